@@ -1,0 +1,245 @@
+"""fp64 CPU oracle for the StreamKL attention-KL primitive.
+
+TEST INFRASTRUCTURE ONLY. Nothing in the product path may import or call this
+module; only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
+``bench.py`` do. It shares no code with the CUDA library.
+
+What it computes ("StreamKL: Fast and Memory-Efficient KL Divergence for
+Boosting Attention Distillation", abstract): attention distillation minimises
+the row-wise KL divergence between a teacher attention distribution and a
+student attention distribution. Written out for one (batch, head):
+
+    s_T[i, j] = scale_T * <q_T[i], k_T[j]>        s_S[i, j] = scale_S * <q_S[i], k_S[j]>
+    J(i)      = { j < N_K : not causal  or  j <= i + N_K - N_Q }   (bottom-right causal)
+    P_X[i, :] = softmax over J(i) of s_X[i, :]                      (X = T, S)
+    KL[i]     = sum_{j in J(i)} P_T[i, j] * (log P_T[i, j] - log P_S[i, j])
+    LSE_X[i]  = log sum_{j in J(i)} exp(s_X[i, j])
+
+The method's claim is that it is exact (it removes the materialisation, not the
+arithmetic), so the oracle *does* materialise both distributions - the baseline
+the abstract describes - one block of query rows at a time, in float64, from the
+bf16 inputs converted exactly to float64. The KL is taken in the materialised
+form above, not through the online identity, so that tests check the identity
+instead of assuming it.
+
+Backward (teacher frozen; g[i] = dLoss/dKL[i]):
+
+    dKL[i]/ds_S[i, j] = P_S[i, j] - P_T[i, j]          (on J(i), else 0)
+    dS[i, j]  = g[i] * scale_S * (P_S[i, j] - P_T[i, j])   (gradient w.r.t. <q_S[i], k_S[j]>)
+    dQ_S      = dS @ K_S            dK_S = dS^T @ Q_S
+
+Readings where the pages are silent (each is listed in the design doc):
+* causal alignment for N_Q != N_K is bottom-right (j <= i + N_K - N_Q);
+* a row with an empty J(i) has KL = 0, LSE = -inf and zero gradient;
+* KL is reported raw (no clamp at 0); LSE is the natural-log value.
+
+Every function below is pinned by tests/test_oracle_pins.py against brute force,
+a library routine (torch log_softmax/kl_div + autograd), closed forms,
+invariances and finite differences.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, List, Sequence, Tuple
+
+import torch
+
+F64 = torch.float64
+NEG_INF = float("-inf")
+
+
+def _f64(x: torch.Tensor) -> torch.Tensor:
+    return x.detach().to("cpu").to(F64)
+
+
+def allowed(i: torch.Tensor, n_q: int, n_k: int, causal: bool) -> torch.Tensor:
+    """Boolean [len(i), N_K] mask of J(i) for the query indices ``i``."""
+    j = torch.arange(n_k)
+    if not causal:
+        return torch.ones(len(i), n_k, dtype=torch.bool)
+    return j[None, :] <= (i[:, None] + (n_k - n_q))
+
+
+def _row_block_stats(qt, kt, qs, ks, rows, scale_t, scale_s, causal, n_q):
+    """Scores, mask, LSEs and log-probabilities for a block of query rows.
+
+    qt/qs: [R, d] fp64 query rows; kt/ks: [N_K, d] fp64 keys; rows: [R] indices.
+    """
+    n_k = kt.shape[0]
+    mask = allowed(rows, n_q, n_k, causal)
+    s_t = scale_t * (qt @ kt.T)
+    s_s = scale_s * (qs @ ks.T)
+    s_t = torch.where(mask, s_t, torch.full_like(s_t, NEG_INF))
+    s_s = torch.where(mask, s_s, torch.full_like(s_s, NEG_INF))
+    lse_t = _logsumexp(s_t)
+    lse_s = _logsumexp(s_s)
+    return s_t, s_s, mask, lse_t, lse_s
+
+
+def _logsumexp(s: torch.Tensor) -> torch.Tensor:
+    """log sum_j exp(s[:, j]) written as max + log(sum(exp(s - max))); -inf for empty rows."""
+    m = s.max(dim=1).values
+    empty = torch.isinf(m) & (m < 0)
+    m_safe = torch.where(empty, torch.zeros_like(m), m)
+    tot = torch.exp(s - m_safe[:, None]).sum(dim=1)
+    out = m_safe + torch.log(tot)
+    return torch.where(empty, torch.full_like(out, NEG_INF), out)
+
+
+def _probs(s: torch.Tensor, lse: torch.Tensor, mask: torch.Tensor):
+    """P = exp(s - LSE) on J(i), 0 elsewhere; log P on J(i), 0 elsewhere."""
+    lse_safe = torch.where(torch.isinf(lse), torch.zeros_like(lse), lse)
+    logp = torch.where(mask, s - lse_safe[:, None], torch.zeros_like(s))
+    p = torch.where(mask, torch.exp(logp), torch.zeros_like(s))
+    return p, logp
+
+
+def _block_kl(s_t, s_s, mask, lse_t, lse_s):
+    p_t, logp_t = _probs(s_t, lse_t, mask)
+    p_s, logp_s = _probs(s_s, lse_s, mask)
+    kl = (p_t * (logp_t - logp_s)).sum(dim=1)
+    return kl, p_t, p_s
+
+
+def oracle_fwd(q_t, k_t, q_s, k_s, scale_t: float, scale_s: float, causal: bool,
+               row_block: int = 1024):
+    """Per-row KL(P_T || P_S), LSE_T and LSE_S, float64 tensors of shape [B, H, N_Q]."""
+    B, H, n_q, _ = q_t.shape
+    n_k = k_t.shape[2]
+    kl = torch.empty(B, H, n_q, dtype=F64)
+    lse_t = torch.empty(B, H, n_q, dtype=F64)
+    lse_s = torch.empty(B, H, n_q, dtype=F64)
+    for b in range(B):
+        for h in range(H):
+            kt, ks = _f64(k_t[b, h]), _f64(k_s[b, h])
+            for r0 in range(0, n_q, row_block):
+                rows = torch.arange(r0, min(n_q, r0 + row_block))
+                st, ss, mask, lt, ls = _row_block_stats(
+                    _f64(q_t[b, h, rows]), kt, _f64(q_s[b, h, rows]), ks,
+                    rows, scale_t, scale_s, causal, n_q)
+                k_row, _, _ = _block_kl(st, ss, mask, lt, ls)
+                kl[b, h, rows] = k_row
+                lse_t[b, h, rows] = lt
+                lse_s[b, h, rows] = ls
+    return kl, lse_t, lse_s
+
+
+def oracle_bwd(q_t, k_t, q_s, k_s, scale_t: float, scale_s: float, causal: bool, g,
+               row_block: int = 1024):
+    """dQ_S [B,H,N_Q,d_S] and dK_S [B,H,N_K,d_S] (float64) of sum_i g[i] * KL[i]."""
+    B, H, n_q, d_s = q_s.shape
+    n_k = k_s.shape[2]
+    dq = torch.zeros(B, H, n_q, d_s, dtype=F64)
+    dk = torch.zeros(B, H, n_k, d_s, dtype=F64)
+    for b in range(B):
+        for h in range(H):
+            kt, ks = _f64(k_t[b, h]), _f64(k_s[b, h])
+            for r0 in range(0, n_q, row_block):
+                rows = torch.arange(r0, min(n_q, r0 + row_block))
+                qs = _f64(q_s[b, h, rows])
+                st, ss, mask, lt, ls = _row_block_stats(
+                    _f64(q_t[b, h, rows]), kt, qs, ks, rows, scale_t, scale_s, causal, n_q)
+                _, p_t, p_s = _block_kl(st, ss, mask, lt, ls)
+                gi = _f64(g[b, h, rows])
+                ds = gi[:, None] * scale_s * (p_s - p_t)
+                dq[b, h, rows] = ds @ ks
+                dk[b, h] += ds.T @ qs
+    return dq, dk
+
+
+def oracle_rows(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g,
+                rows: Sequence[Tuple[int, int]]):
+    """KL, LSE_T, LSE_S and the dQ_S row for selected (bh, i) query rows.
+
+    Each row needs only its own scores, so this is the per-row definition
+    evaluated on a sample (used for parity at full size).
+    Returns (kl [R], lse_t [R], lse_s [R], dq [R, d_S]) in float64.
+    """
+    B, H, n_q, _ = q_t.shape
+    n_k = k_t.shape[2]
+    qt2 = q_t.reshape(B * H, n_q, -1)
+    kt2 = k_t.reshape(B * H, n_k, -1)
+    qs2 = q_s.reshape(B * H, n_q, -1)
+    ks2 = k_s.reshape(B * H, n_k, -1)
+    g2 = g.reshape(B * H, n_q)
+    kl, lt_o, ls_o, dq = [], [], [], []
+    by_head = {}
+    for bh, i in rows:
+        by_head.setdefault(bh, []).append(i)
+    order = []
+    for bh, idx in by_head.items():
+        rr = torch.tensor(idx)
+        kt, ks = _f64(kt2[bh]), _f64(ks2[bh])
+        st, ss, mask, lt, ls = _row_block_stats(
+            _f64(qt2[bh, rr]), kt, _f64(qs2[bh, rr]), ks, rr, scale_t, scale_s, causal, n_q)
+        k_row, p_t, p_s = _block_kl(st, ss, mask, lt, ls)
+        ds = _f64(g2[bh, rr])[:, None] * scale_s * (p_s - p_t)
+        kl.append(k_row); lt_o.append(lt); ls_o.append(ls); dq.append(ds @ ks)
+        order += [(bh, i) for i in idx]
+    pos = {r: n for n, r in enumerate(order)}
+    perm = torch.tensor([pos[tuple(r)] for r in rows])
+    cat = lambda xs: torch.cat(xs)[perm]
+    return cat(kl), cat(lt_o), cat(ls_o), cat(dq)
+
+
+def oracle_dk_rows(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g, bh: int,
+                   keys: Sequence[int], row_block: int = 2048):
+    """dK_S rows for selected keys of one head (float64 [len(keys), d_S]).
+
+    dK_S[j] = sum_i dS[i, j] q_S[i] needs P_T[i, j] and P_S[i, j] for every
+    query row i, so every row's LSE is computed here from the full row.
+    """
+    B, H, n_q, d_s = q_s.shape
+    n_k = k_s.shape[2]
+    qt = q_t.reshape(B * H, n_q, -1)[bh]
+    qs = q_s.reshape(B * H, n_q, -1)[bh]
+    kt = _f64(k_t.reshape(B * H, n_k, -1)[bh])
+    ks = _f64(k_s.reshape(B * H, n_k, -1)[bh])
+    gg = g.reshape(B * H, n_q)[bh]
+    sel = torch.tensor(list(keys))
+    out = torch.zeros(len(sel), d_s, dtype=F64)
+    for r0 in range(0, n_q, row_block):
+        rows = torch.arange(r0, min(n_q, r0 + row_block))
+        qsr = _f64(qs[rows])
+        st, ss, mask, lt, ls = _row_block_stats(
+            _f64(qt[rows]), kt, qsr, ks, rows, scale_t, scale_s, causal, n_q)
+        _, p_t, p_s = _block_kl(st, ss, mask, lt, ls)
+        ds = _f64(gg[rows])[:, None] * scale_s * (p_s - p_t)
+        out += ds[:, sel].T @ qsr
+    return out
+
+
+def oracle_row_work(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g,
+                    rows: Sequence[Tuple[int, int]]):
+    """Whole forward + backward work of selected query rows (CPU-baseline timing).
+
+    For each sampled row: its KL and LSEs, its dQ_S row, and its contribution
+    dS[i, :]^T q_S[i] to dK_S. Returns (kl, dq, dk_contrib_sum) so nothing is
+    optimised away.
+    """
+    kl, _, _, dq = oracle_rows(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g, rows)
+    B, H, n_q, d_s = q_s.shape
+    n_k = k_s.shape[2]
+    qs2 = q_s.reshape(B * H, n_q, -1)
+    qt2 = q_t.reshape(B * H, n_q, -1)
+    kt2 = k_t.reshape(B * H, n_k, -1)
+    ks2 = k_s.reshape(B * H, n_k, -1)
+    g2 = g.reshape(B * H, n_q)
+    dk_acc = torch.zeros(n_k, d_s, dtype=F64)
+    for bh, i in rows:
+        rr = torch.tensor([i])
+        qsr = _f64(qs2[bh, rr])
+        st, ss, mask, lt, ls = _row_block_stats(
+            _f64(qt2[bh, rr]), _f64(kt2[bh]), qsr, _f64(ks2[bh]), rr,
+            scale_t, scale_s, causal, n_q)
+        _, p_t, p_s = _block_kl(st, ss, mask, lt, ls)
+        ds = _f64(g2[bh, rr])[:, None] * scale_s * (p_s - p_t)
+        dk_acc += ds.T @ qsr
+    return kl, dq, dk_acc
+
+
+def row_pair_count(n_q: int, n_k: int, causal: bool, i: int) -> int:
+    """|J(i)|: number of keys query row i attends to."""
+    if not causal:
+        return n_k
+    return max(0, min(n_k, i + n_k - n_q + 1))

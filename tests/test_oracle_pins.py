@@ -1,0 +1,337 @@
+"""Pins for the fp64 oracle, against things other than itself (CPU only).
+
+Each test states what fixes the expected value: brute force from the
+definition, a library routine (torch log_softmax / kl_div + autograd), closed
+forms, invariances, finite differences. Together they make a dropped term, a
+wrong sign, a wrong index, a wrong causal alignment or a transposed operand in
+the oracle fail at least one test (see test_planted_mistakes_are_caught).
+"""
+import math
+
+import pytest
+import torch
+
+from oracle import streamkl_oracle as O
+from workloads import WORKLOADS, make_inputs
+
+F64 = torch.float64
+
+
+def rand_case(B, H, nq, nk, dt, ds, seed, bf16=True, spread=1.0):
+    g = torch.Generator().manual_seed(seed)
+    mk = lambda *s: (spread * torch.randn(*s, generator=g, dtype=torch.float32))
+    q_t, k_t = mk(B, H, nq, dt), mk(B, H, nk, dt)
+    q_s, k_s = mk(B, H, nq, ds), mk(B, H, nk, ds)
+    gg = torch.rand(B, H, nq, generator=g) + 0.5
+    if bf16:
+        q_t, k_t, q_s, k_s = (x.to(torch.bfloat16) for x in (q_t, k_t, q_s, k_s))
+    return q_t, k_t, q_s, k_s, gg
+
+
+# ---------------------------------------------------------------- brute force
+
+def brute_force(q_t, k_t, q_s, k_s, st, ss, causal, g):
+    """Pure-Python loops straight from the definition (no max shift, no matmul).
+
+    KL_i = sum_j p_T log(p_T / p_S) with p = exp(s) / sum exp(s) over the keys
+    j <= i + N_K - N_Q (causal) or all keys. dQ_S and dK_S are the derivatives
+    of sum_i g_i KL_i, using dKL_i/ds_S[i,j] = p_S - p_T.
+    """
+    B, H, nq, dt = q_t.shape
+    nk, ds_ = k_t.shape[2], q_s.shape[3]
+    L = lambda t: t.double().tolist()
+    QT, KT, QS, KS, G = L(q_t), L(k_t), L(q_s), L(k_s), L(g)
+    kl = [[[0.0] * nq for _ in range(H)] for _ in range(B)]
+    lt = [[[0.0] * nq for _ in range(H)] for _ in range(B)]
+    ls = [[[0.0] * nq for _ in range(H)] for _ in range(B)]
+    dq = [[[[0.0] * ds_ for _ in range(nq)] for _ in range(H)] for _ in range(B)]
+    dk = [[[[0.0] * ds_ for _ in range(nk)] for _ in range(H)] for _ in range(B)]
+    for b in range(B):
+        for h in range(H):
+            for i in range(nq):
+                js = [j for j in range(nk) if (not causal) or j <= i + nk - nq]
+                if not js:
+                    lt[b][h][i] = ls[b][h][i] = float("-inf")
+                    continue
+                sT = {j: st * sum(QT[b][h][i][c] * KT[b][h][j][c] for c in range(dt)) for j in js}
+                sS = {j: ss * sum(QS[b][h][i][c] * KS[b][h][j][c] for c in range(ds_)) for j in js}
+                zT = sum(math.exp(v) for v in sT.values())
+                zS = sum(math.exp(v) for v in sS.values())
+                pT = {j: math.exp(sT[j]) / zT for j in js}
+                pS = {j: math.exp(sS[j]) / zS for j in js}
+                kl[b][h][i] = sum(pT[j] * math.log(pT[j] / pS[j]) for j in js)
+                lt[b][h][i], ls[b][h][i] = math.log(zT), math.log(zS)
+                for j in js:
+                    dsij = G[b][h][i] * ss * (pS[j] - pT[j])
+                    for c in range(ds_):
+                        dq[b][h][i][c] += dsij * KS[b][h][j][c]
+                        dk[b][h][j][c] += dsij * QS[b][h][i][c]
+    T = lambda x: torch.tensor(x, dtype=F64)
+    return T(kl), T(lt), T(ls), T(dq), T(dk)
+
+
+@pytest.mark.parametrize("nq,nk,causal", [(5, 5, False), (5, 5, True), (6, 3, True),
+                                          (3, 6, True), (4, 7, False), (1, 1, True)])
+def test_brute_force_tiny(nq, nk, causal):
+    q_t, k_t, q_s, k_s, g = rand_case(2, 2, nq, nk, 3, 2, seed=nq * 31 + nk + causal)
+    st, ss = 0.7, 1.3
+    ref = brute_force(q_t, k_t, q_s, k_s, st, ss, causal, g)
+    kl, lt, ls = O.oracle_fwd(q_t, k_t, q_s, k_s, st, ss, causal, row_block=2)
+    dq, dk = O.oracle_bwd(q_t, k_t, q_s, k_s, st, ss, causal, g, row_block=2)
+    for got, want in zip((kl, lt, ls, dq, dk), ref):
+        fin = torch.isfinite(want)
+        assert torch.equal(fin, torch.isfinite(got))
+        assert torch.equal(got[~fin], want[~fin])
+        torch.testing.assert_close(got[fin], want[fin], rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------- library routine
+
+def library_kl(q_t, k_t, q_s, k_s, st, ss, causal, g):
+    """torch log_softmax + kl_div (log_target) in fp64, autograd for the gradients."""
+    qs = q_s.double().requires_grad_(True)
+    ks = k_s.double().requires_grad_(True)
+    nq, nk = q_t.shape[2], k_t.shape[2]
+    s_t = st * q_t.double() @ k_t.double().transpose(-1, -2)
+    s_s = ss * qs @ ks.transpose(-1, -2)
+    if causal:
+        i = torch.arange(nq)[:, None]
+        j = torch.arange(nk)[None, :]
+        bad = j > i + nk - nq
+        s_t = s_t.masked_fill(bad, float("-inf"))
+        s_s = s_s.masked_fill(bad, float("-inf"))
+    lp_t = torch.log_softmax(s_t, -1)
+    lp_s = torch.log_softmax(s_s, -1)
+    # kl_div(input=log q, target=log p, log_target=True) = p * (log p - log q)
+    terms = torch.nn.functional.kl_div(lp_s, lp_t, reduction="none", log_target=True)
+    terms = torch.nan_to_num(terms, nan=0.0)
+    kl = terms.sum(-1)
+    (kl * g.double()).sum().backward()
+    return kl.detach(), torch.logsumexp(s_t, -1).detach(), torch.logsumexp(s_s, -1).detach(), qs.grad, ks.grad
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dims", [(8, 8, 16, 16), (16, 9, 8, 4), (9, 16, 4, 8)])
+def test_against_library(causal, dims):
+    nq, nk, dt, ds = dims
+    q_t, k_t, q_s, k_s, g = rand_case(1, 3, nq, nk, dt, ds, seed=sum(dims) + causal)
+    st, ss = 1 / math.sqrt(dt), 1 / math.sqrt(ds)
+    kl_r, lt_r, ls_r, dq_r, dk_r = library_kl(q_t, k_t, q_s, k_s, st, ss, causal, g)
+    kl, lt, ls = O.oracle_fwd(q_t, k_t, q_s, k_s, st, ss, causal, row_block=5)
+    dq, dk = O.oracle_bwd(q_t, k_t, q_s, k_s, st, ss, causal, g, row_block=5)
+    ok = torch.isfinite(lt_r)
+    torch.testing.assert_close(kl[ok], kl_r[ok], rtol=1e-12, atol=1e-12)
+    torch.testing.assert_close(lt[ok], lt_r[ok], rtol=1e-12, atol=1e-12)
+    torch.testing.assert_close(ls[ok], ls_r[ok], rtol=1e-12, atol=1e-12)
+    torch.testing.assert_close(dq, torch.nan_to_num(dq_r), rtol=1e-10, atol=1e-12)
+    torch.testing.assert_close(dk, torch.nan_to_num(dk_r), rtol=1e-10, atol=1e-12)
+
+
+# ------------------------------------------------------------- closed forms
+
+def test_two_key_bernoulli_closed_form():
+    """Two keys: softmax over two scores is a Bernoulli law; KL and dS are closed-form."""
+    # d = 2, keys e1 and e2, so s[i, j] = scale * q[i, j].
+    q_t = torch.tensor([[[[1.5, -0.5], [0.25, 2.0], [0.0, 0.0]]]], dtype=F64)
+    q_s = torch.tensor([[[[0.5, 0.5], [-1.0, 1.0], [3.0, -2.0]]]], dtype=F64)
+    k = torch.tensor([[[[1.0, 0.0], [0.0, 1.0]]]], dtype=F64)
+    st, ss = 0.8, 1.7
+    g = torch.tensor([[[1.0, 0.5, 2.0]]], dtype=F64)
+    kl, lt, ls = O.oracle_fwd(q_t, k, q_s, k, st, ss, False)
+    dq, dk = O.oracle_bwd(q_t, k, q_s, k, st, ss, False, g)
+    sig = lambda x: 1.0 / (1.0 + math.exp(-x))
+    for i in range(3):
+        a = sig(st * (q_t[0, 0, i, 0] - q_t[0, 0, i, 1]).item())
+        b = sig(ss * (q_s[0, 0, i, 0] - q_s[0, 0, i, 1]).item())
+        want = a * math.log(a / b) + (1 - a) * math.log((1 - a) / (1 - b))
+        assert abs(kl[0, 0, i].item() - want) < 1e-13 * max(1.0, abs(want))
+        want_lt = math.log(math.exp(st * q_t[0, 0, i, 0].item()) + math.exp(st * q_t[0, 0, i, 1].item()))
+        assert abs(lt[0, 0, i].item() - want_lt) < 1e-13 * max(1.0, abs(want_lt))
+        # dKL/ds_S[i,0] = b - a, dKL/ds_S[i,1] = a - b; dQ_S[i] = g*scale_S*(b-a, a-b)
+        gi = g[0, 0, i].item()
+        torch.testing.assert_close(dq[0, 0, i], torch.tensor([gi * ss * (b - a), gi * ss * (a - b)], dtype=F64),
+                                   rtol=1e-13, atol=1e-15)
+
+
+def test_uniform_student_closed_form():
+    """scale_S = 0 makes P_S uniform on J(i): KL = log|J(i)| - H(P_T)."""
+    q_t, k_t, q_s, k_s, g = rand_case(1, 2, 12, 12, 8, 8, seed=7)
+    for causal in (False, True):
+        kl, lt, ls = O.oracle_fwd(q_t, k_t, q_s, k_s, 0.9, 0.0, causal)
+        for h in range(2):
+            for i in range(12):
+                n = O.row_pair_count(12, 12, causal, i)
+                s = [0.9 * float(q_t[0, h, i].double() @ k_t[0, h, j].double()) for j in range(n)]
+                z = sum(math.exp(v) for v in s)
+                p = [math.exp(v) / z for v in s]
+                ent = -sum(x * math.log(x) for x in p)
+                assert abs(kl[0, h, i].item() - (math.log(n) - ent)) < 1e-12
+                assert abs(ls[0, h, i].item() - math.log(n)) < 1e-12
+
+
+def test_both_scales_zero_gives_zero():
+    q_t, k_t, q_s, k_s, g = rand_case(1, 1, 9, 9, 4, 4, seed=3)
+    kl, _, _ = O.oracle_fwd(q_t, k_t, q_s, k_s, 0.0, 0.0, True)
+    assert torch.all(kl.abs() < 1e-15)
+
+
+def test_causal_row_zero_single_key():
+    """Causal with N_Q = N_K: row 0 sees key 0 only, so KL = 0, LSE = s[0,0], dQ row 0 = 0."""
+    q_t, k_t, q_s, k_s, g = rand_case(1, 2, 10, 10, 4, 4, seed=11)
+    kl, lt, ls = O.oracle_fwd(q_t, k_t, q_s, k_s, 0.5, 0.5, True)
+    dq, dk = O.oracle_bwd(q_t, k_t, q_s, k_s, 0.5, 0.5, True, g)
+    assert torch.all(kl[:, :, 0] == 0)
+    want = 0.5 * (q_t[0, :, 0].double() * k_t[0, :, 0].double()).sum(-1)
+    torch.testing.assert_close(lt[0, :, 0], want, rtol=1e-14, atol=1e-14)
+    assert torch.all(dq[:, :, 0] == 0)
+
+
+def test_empty_rows_when_more_queries_than_keys():
+    """Causal, N_Q > N_K: rows i < N_Q - N_K see no key (KL 0, LSE -inf, zero gradient)."""
+    q_t, k_t, q_s, k_s, g = rand_case(1, 1, 7, 4, 4, 4, seed=5)
+    kl, lt, ls = O.oracle_fwd(q_t, k_t, q_s, k_s, 0.5, 0.5, True)
+    dq, dk = O.oracle_bwd(q_t, k_t, q_s, k_s, 0.5, 0.5, True, g)
+    assert torch.all(kl[0, 0, :3] == 0)
+    assert torch.all(torch.isneginf(lt[0, 0, :3])) and torch.all(torch.isneginf(ls[0, 0, :3]))
+    assert torch.all(torch.isfinite(lt[0, 0, 3:]))
+    assert torch.all(dq[0, 0, :3] == 0)
+    assert torch.all(kl[0, 0, 3] == 0)  # row 3 sees key 0 only
+
+
+# --------------------------------------------------------------- invariants
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gibbs_nonnegative(causal):
+    for seed in range(4):
+        q_t, k_t, q_s, k_s, g = rand_case(2, 2, 33, 29, 16, 8, seed=seed, spread=2.0)
+        kl, _, _ = O.oracle_fwd(q_t, k_t, q_s, k_s, 0.3, 0.4, causal, row_block=7)
+        assert torch.all(kl >= -1e-13)
+        assert kl.max() > 0.01
+
+
+def test_identical_inputs_give_zero():
+    q_t, k_t, _, _, g = rand_case(1, 2, 20, 20, 8, 8, seed=9)
+    for causal in (False, True):
+        kl, lt, ls = O.oracle_fwd(q_t, k_t, q_t, k_t, 0.35, 0.35, causal)
+        dq, dk = O.oracle_bwd(q_t, k_t, q_t, k_t, 0.35, 0.35, causal, g)
+        assert torch.all(kl == 0)
+        assert torch.equal(lt, ls)
+        assert torch.all(dq == 0) and torch.all(dk == 0)
+
+
+def test_key_shift_invariance_and_dk_sums_to_zero():
+    """Adding one vector c to every student key shifts each row's student scores
+    by a constant, which softmax ignores: KL is unchanged. Because sum_j dS[i,j] = 0
+    for every row, sum_j dK_S[j] = sum_i (sum_j dS[i,j]) q_S[i] = 0."""
+    q_t, k_t, q_s, k_s, g = rand_case(1, 2, 15, 15, 8, 8, seed=21, bf16=False)
+    q_t, k_t, q_s, k_s = (x.double() for x in (q_t, k_t, q_s, k_s))
+    c = torch.randn(8, generator=torch.Generator().manual_seed(1), dtype=F64)
+    for causal in (False, True):
+        kl1, _, _ = O.oracle_fwd(q_t, k_t, q_s, k_s, 0.4, 0.6, causal)
+        kl2, _, _ = O.oracle_fwd(q_t, k_t, q_s, k_s + c, 0.4, 0.6, causal)
+        torch.testing.assert_close(kl1, kl2, rtol=1e-11, atol=1e-12)
+        dq, dk = O.oracle_bwd(q_t, k_t, q_s, k_s, 0.4, 0.6, causal, g)
+        assert dk.sum(dim=2).abs().max() < 1e-12
+        assert dk.abs().max() > 1e-3
+
+
+def test_online_identity_matches_materialised_form():
+    """KL_i = E_{P_T}[s_T - s_S] - LSE_T + LSE_S (the identity the forward streams)."""
+    q_t, k_t, q_s, k_s, g = rand_case(1, 2, 17, 17, 8, 8, seed=2)
+    st, ss = 0.5, 0.7
+    for causal in (False, True):
+        kl, lt, ls = O.oracle_fwd(q_t, k_t, q_s, k_s, st, ss, causal)
+        for h in range(2):
+            s_t = st * q_t[0, h].double() @ k_t[0, h].double().T
+            s_s = ss * q_s[0, h].double() @ k_s[0, h].double().T
+            for i in range(17):
+                n = O.row_pair_count(17, 17, causal, i)
+                p = torch.exp(s_t[i, :n] - lt[0, h, i])
+                e = (p * (s_t[i, :n] - s_s[i, :n])).sum()
+                assert abs((e - lt[0, h, i] + ls[0, h, i]).item() - kl[0, h, i].item()) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_finite_differences(causal):
+    """Central differences of sum_i g_i KL_i w.r.t. entries of Q_S and K_S."""
+    q_t, k_t, q_s, k_s, g = rand_case(1, 1, 6, 7, 4, 3, seed=13, bf16=False)
+    q_t, k_t, q_s, k_s = (x.double() for x in (q_t, k_t, q_s, k_s))
+    g = g.double()
+    st, ss = 0.6, 0.9
+    dq, dk = O.oracle_bwd(q_t, k_t, q_s, k_s, st, ss, causal, g)
+    loss = lambda qs, ks: float((O.oracle_fwd(q_t, k_t, qs, ks, st, ss, causal)[0] * g).sum())
+    h = 1e-6
+    for (i, c) in [(0, 0), (2, 1), (5, 2), (3, 0)]:
+        e = torch.zeros_like(q_s); e[0, 0, i, c] = h
+        fd = (loss(q_s + e, k_s) - loss(q_s - e, k_s)) / (2 * h)
+        assert abs(fd - dq[0, 0, i, c].item()) <= 1e-6 * max(1.0, abs(fd))
+    for (j, c) in [(0, 0), (3, 2), (6, 1)]:
+        e = torch.zeros_like(k_s); e[0, 0, j, c] = h
+        fd = (loss(q_s, k_s + e) - loss(q_s, k_s - e)) / (2 * h)
+        assert abs(fd - dk[0, 0, j, c].item()) <= 1e-6 * max(1.0, abs(fd))
+
+
+# ------------------------------------------------------ sampled-row helpers
+
+def test_sampled_rows_match_full():
+    w = WORKLOADS["tiny_n256_d64"].with_sizes(H=3, N_Q=70, N_K=70, causal=True)
+    x = make_inputs(w)
+    args = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S, w.causal)
+    kl, lt, ls = O.oracle_fwd(*args, row_block=16)
+    dq, dk = O.oracle_bwd(*args, x["g"], row_block=16)
+    rows = [(0, 0), (2, 69), (1, 33), (0, 5)]
+    kl_r, lt_r, ls_r, dq_r = O.oracle_rows(*args, x["g"], rows)
+    for n, (bh, i) in enumerate(rows):
+        assert kl_r[n] == kl.view(-1, 70)[bh, i]
+        assert lt_r[n] == lt.view(-1, 70)[bh, i]
+        torch.testing.assert_close(dq_r[n], dq.view(3, 70, -1)[bh, i], rtol=1e-13, atol=1e-15)
+    keys = [0, 17, 69]
+    dk_r = O.oracle_dk_rows(*args, x["g"], 1, keys, row_block=16)
+    torch.testing.assert_close(dk_r, dk.view(3, 70, -1)[1, keys], rtol=1e-12, atol=1e-14)
+
+
+# --------------------------------------------------- planted mistakes (CPU)
+
+def _mutants():
+    """Plausible one-line mistakes, each planted in a copy of one oracle helper."""
+    orig_stats = O._row_block_stats
+
+    def wrong_causal(i, n_q, n_k, causal):  # top-left alignment instead of bottom-right
+        j = torch.arange(n_k)
+        if not causal:
+            return torch.ones(len(i), n_k, dtype=torch.bool)
+        return j[None, :] <= i[:, None]
+
+    def lse_no_max(s):  # drops the max term of the log-sum-exp
+        m = s.max(dim=1).values
+        return torch.log(torch.exp(s - m[:, None]).sum(dim=1))
+
+    def probs_sign(s, lse, mask):  # wrong sign: exp(s + LSE)
+        logp = torch.where(mask, s + lse[:, None], torch.zeros_like(s))
+        return torch.where(mask, torch.exp(logp), torch.zeros_like(s)), logp
+
+    def kl_dropped_term(s_t, s_s, mask, lse_t, lse_s):  # drops the -log P_S term
+        p_t, logp_t = O._probs(s_t, lse_t, mask)
+        p_s, _ = O._probs(s_s, lse_s, mask)
+        return (p_t * logp_t).sum(dim=1), p_t, p_s
+
+    def teacher_keys_for_student(qt, kt, qs, ks, rows, st, ss, causal, n_q):  # wrong operand
+        return orig_stats(qt, kt, qs, kt[:, : ks.shape[1]], rows, st, ss, causal, n_q)
+
+    return [("allowed", wrong_causal), ("_logsumexp", lse_no_max), ("_probs", probs_sign),
+            ("_block_kl", kl_dropped_term), ("_row_block_stats", teacher_keys_for_student)]
+
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    """Each planted oracle mistake must break the brute-force pin (N_Q != N_K, causal)."""
+    q_t, k_t, q_s, k_s, g = rand_case(1, 1, 4, 6, 3, 2, seed=99)
+    ref = brute_force(q_t, k_t, q_s, k_s, 0.7, 1.1, True, g)
+    mutants = _mutants()
+    for name, fn in mutants:
+        with monkeypatch.context() as m:
+            m.setattr(O, name, fn)
+            kl, lt, ls = O.oracle_fwd(q_t, k_t, q_s, k_s, 0.7, 1.1, True)
+            dq, dk = O.oracle_bwd(q_t, k_t, q_s, k_s, 0.7, 1.1, True, g)
+            same = all(torch.allclose(a, b, rtol=1e-9, atol=1e-12, equal_nan=True)
+                       for a, b in zip((kl, lt, ls, dq, dk), ref))
+            assert not same, f"planted mistake in {name} was not caught"
