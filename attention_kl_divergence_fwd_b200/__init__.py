@@ -1,0 +1,148 @@
+"""Python binding of the StreamKL C ABI (include/streamkl.h).
+
+Argument marshalling only: every step of the forward and backward runs in the CUDA
+library ``lib/libstreamkl.so``. PyTorch supplies device memory and the stream. There
+is no CPU fallback: if the library is missing, importing the functions raises.
+
+    kl, lse_t, lse_s = streamkl_fwd(q_t, k_t, q_s, k_s, scale_T, scale_S, causal)
+    dq_s, dk_s = streamkl_bwd(q_t, k_t, q_s, k_s, scale_T, scale_S, causal, lse_t, lse_s, g)
+
+Tensors: bf16 [B, H, N, d] contiguous on one CUDA device (d in {64, 128}); row
+statistics and g fp32 [B, H, N_Q]; gradients fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libstreamkl.so")
+
+STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "MISALIGNED", 4: "LAUNCH", 5: "TIMEOUT"}
+EXPORTS = ("streamkl_fwd", "streamkl_bwd", "streamkl_status_string", "streamkl_device_status",
+           "streamkl_version")
+
+
+class StreamKLError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {status_string(status)}")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"StreamKL CUDA library not built: {path} "
+                      "(run python -m attention_kl_divergence_fwd_b200.build)")
+    lib = ctypes.CDLL(path)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.streamkl_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, f, i, vp, vp, vp, vp]
+    lib.streamkl_fwd.restype = i
+    lib.streamkl_bwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, f, i, vp, vp, vp, vp, vp, vp]
+    lib.streamkl_bwd.restype = i
+    lib.streamkl_status_string.argtypes = [i]
+    lib.streamkl_status_string.restype = ctypes.c_char_p
+    lib.streamkl_device_status.argtypes = [vp]
+    lib.streamkl_device_status.restype = i
+    lib.streamkl_version.argtypes = []
+    lib.streamkl_version.restype = i
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().streamkl_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise StreamKLError(status, where)
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _shape(q_t, k_t, q_s, k_s):
+    import torch
+    for name, t in (("q_t", q_t), ("k_t", k_t), ("q_s", q_s), ("k_s", k_s)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor [B,H,N,d]")
+    B, H, n_q, d_t = q_t.shape
+    n_k = k_t.shape[2]
+    d_s = q_s.shape[3]
+    if tuple(k_t.shape) != (B, H, n_k, d_t) or tuple(q_s.shape) != (B, H, n_q, d_s) or \
+            tuple(k_s.shape) != (B, H, n_k, d_s):
+        raise ValueError("inconsistent shapes")
+    return B, H, n_q, n_k, d_t, d_s
+
+
+def streamkl_fwd_raw(q_t: int, k_t: int, q_s: int, k_s: int, B: int, H: int, N_Q: int, N_K: int,
+                     d_T: int, d_S: int, scale_T: float, scale_S: float, causal: bool,
+                     kl: int, lse_t: int, lse_s: int, stream: int = 0) -> int:
+    """The C entry point with plain pointers; returns the status code."""
+    return load_library().streamkl_fwd(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S,
+                                       float(scale_T), float(scale_S), int(bool(causal)),
+                                       kl, lse_t, lse_s, stream)
+
+
+def streamkl_bwd_raw(q_t: int, k_t: int, q_s: int, k_s: int, B: int, H: int, N_Q: int, N_K: int,
+                     d_T: int, d_S: int, scale_T: float, scale_S: float, causal: bool,
+                     lse_t: int, lse_s: int, g: int, dq_s: int, dk_s: int, stream: int = 0) -> int:
+    return load_library().streamkl_bwd(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S,
+                                       float(scale_T), float(scale_S), int(bool(causal)),
+                                       lse_t, lse_s, g, dq_s, dk_s, stream)
+
+
+def streamkl_fwd(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
+                 kl=None, lse_t=None, lse_s=None, stream=None):
+    """Per-row KL(P_T || P_S), LSE_T, LSE_S (fp32 [B,H,N_Q]) on the current stream."""
+    import torch
+    B, H, n_q, n_k, d_t, d_s = _shape(q_t, k_t, q_s, k_s)
+    dev = q_t.device
+    kl = torch.empty(B, H, n_q, device=dev, dtype=torch.float32) if kl is None else kl
+    lse_t = torch.empty_like(kl) if lse_t is None else lse_t
+    lse_s = torch.empty_like(kl) if lse_s is None else lse_s
+    st = streamkl_fwd_raw(q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(),
+                          B, H, n_q, n_k, d_t, d_s, scale_T, scale_S, causal,
+                          kl.data_ptr(), lse_t.data_ptr(), lse_s.data_ptr(), _stream_ptr(stream))
+    _check(st, "streamkl_fwd")
+    return kl, lse_t, lse_s
+
+
+def streamkl_bwd(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
+                 lse_t, lse_s, g, dq_s=None, dk_s=None, stream=None):
+    """dQ_S [B,H,N_Q,d_S] and dK_S [B,H,N_K,d_S] (fp32) of sum_i g_i KL_i."""
+    import torch
+    B, H, n_q, n_k, d_t, d_s = _shape(q_t, k_t, q_s, k_s)
+    dev = q_t.device
+    for name, t in (("lse_t", lse_t), ("lse_s", lse_s), ("g", g)):
+        if t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != (B, H, n_q):
+            raise ValueError(f"{name} must be contiguous fp32 [B,H,N_Q]")
+    dq_s = torch.empty(B, H, n_q, d_s, device=dev, dtype=torch.float32) if dq_s is None else dq_s
+    dk_s = torch.empty(B, H, n_k, d_s, device=dev, dtype=torch.float32) if dk_s is None else dk_s
+    st = streamkl_bwd_raw(q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(),
+                          B, H, n_q, n_k, d_t, d_s, scale_T, scale_S, causal,
+                          lse_t.data_ptr(), lse_s.data_ptr(), g.data_ptr(),
+                          dq_s.data_ptr(), dk_s.data_ptr(), _stream_ptr(stream))
+    _check(st, "streamkl_bwd")
+    return dq_s, dk_s
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the library's device error status."""
+    return load_library().streamkl_device_status(_stream_ptr(stream))
+
+
+def version() -> int:
+    return load_library().streamkl_version()

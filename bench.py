@@ -1,0 +1,367 @@
+"""StreamKL benchmark: forward + backward throughput on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one StreamKL forward (KL, LSE_T, LSE_S per row) + one backward (dQ_S, dK_S)
+over the whole workload, inputs resident in HBM. Default workload: B=1, H=32,
+N_Q=N_K=16384, d=128, causal (long context). Multi-GPU runs (torchrun) are weak
+scaling: every rank runs its own copy of the workload (heads are independent, so
+there is no data-path collective); time is the max over ranks.
+
+Prints one JSON line (rank 0). FLOPs are counted per head as 2*N_Q*N_K*(d_T+d_S)
+forward and 2*N_Q*N_K*(d_T+3*d_S) backward, halved when causal.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, flops_bwd, flops_fwd, make_inputs  # noqa: E402
+
+METRIC = "fwd/bwd TFLOP/s and % of B200 bf16 peak at N=16K,d=128; ms per fwd+bwd"
+DEFAULT_WORKLOAD = "long_b1h32_n16384_d128_causal"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_baseline(w, budget_s: float = 12.0, seed: int = 77):
+    """The fp64 oracle as it stands, timed on this host's cores on sampled query rows.
+
+    Each sampled row does its full forward + backward work: its KL and LSEs, its dQ_S
+    row and its contribution to dK_S. FLOPs are counted with the same convention as
+    the GPU (2*|J(i)|*(d_T+d_S) + 2*|J(i)|*(d_T+3*d_S) per row)."""
+    from oracle import oracle_row_work, row_pair_count
+    x = make_inputs(w) if w.bh * w.N_Q * (w.d_T + w.d_S) * 2 < (3 << 30) else None
+    if x is None:
+        raise RuntimeError("workload too large for the CPU baseline")
+    gen = torch.Generator().manual_seed(seed)
+    args = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S, w.causal, x["g"])
+    done_rows, flops, elapsed = 0, 0.0, 0.0
+    batch = 16
+    while elapsed < budget_s:
+        flat = torch.randint(0, w.bh * w.N_Q, (batch,), generator=gen).tolist()
+        rows = [(f // w.N_Q, f % w.N_Q) for f in flat]
+        t0 = time.perf_counter()
+        oracle_row_work(*args, rows)
+        elapsed += time.perf_counter() - t0
+        for _, i in rows:
+            n = row_pair_count(w.N_Q, w.N_K, w.causal, i)
+            flops += 2.0 * n * (w.d_T + w.d_S) + 2.0 * n * (w.d_T + 3 * w.d_S)
+        done_rows += batch
+    cores = torch.get_num_threads()
+    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done_rows} uniformly sampled query rows of {w.name} (fwd + bwd work of "
+                      f"each row, fp64, torch CPU ops), {elapsed:.1f} s",
+            "seconds": elapsed, "host_cores": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the fp64 oracle on the host cores (rank 0 only)."""
+    w = WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(w, budget_s=min(per_step, 3.0), seed=11)
+    vals, secs = [], 0.0
+    for k in range(args.steps):
+        cb = cpu_baseline(w, budget_s=per_step, seed=100 + k)
+        vals.append(cb["value"])
+        secs += cb["seconds"]
+    value = statistics.mean(vals)
+    cb["value"] = value
+    cb["sample"] = f"{args.steps} steps, each {cb['sample']}"
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": config_of(w, world), "cpu_baseline": cb,
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def config_of(w, world):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N_Q": w.N_Q, "N_K": w.N_K, "d_T": w.d_T,
+            "d_S": w.d_S, "causal": w.causal, "scale_T": w.scale_T, "scale_S": w.scale_S,
+            "per_rank": "full workload per rank (heads are independent)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "no flush: each step reads 4 bf16 input tensors larger than the 126 MB L2"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    import attention_kl_divergence_fwd_b200 as skl
+    skl.load_library()
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    x = make_inputs(w)
+    d = {k: v.to(dev) for k, v in x.items()}
+    B, H, nq, nk = w.B, w.H, w.N_Q, w.N_K
+    kl = torch.empty(B, H, nq, device=dev)
+    lt, ls = torch.empty_like(kl), torch.empty_like(kl)
+    dq = torch.empty(B, H, nq, w.d_S, device=dev)
+    dk = torch.empty(B, H, nk, w.d_S, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        skl.streamkl_fwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal,
+                         kl=kl, lse_t=lt, lse_s=ls)
+        if ev is not None:
+            ev[1].record(stream)
+        skl.streamkl_bwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal,
+                         lt, ls, d["g"], dq_s=dq, dk_s=dk)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if skl.device_status() != 0:
+        raise RuntimeError("kernel watchdog fired during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    if skl.device_status() != 0:
+        raise RuntimeError("kernel watchdog fired during the timed region")
+
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    fwd_ms = max_over_ranks(fwd_ms, world)
+    bwd_ms = max_over_ranks(bwd_ms, world)
+    ms_step = total_ms / args.steps
+    ff, fb = flops_fwd(w), flops_bwd(w)
+    value = world * (ff + fb) * args.steps / (total_ms * 1e-3) / 1e12
+
+    peaks, peak_kind = load_peaks()
+    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    fwd_tf = ff / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = fb / (bwd_ms * 1e-3) / 1e12
+    dominant = "bwd" if bwd_ms >= fwd_ms else "fwd"
+    traffic = load_traffic(w.name, dominant)
+    roof = {"kernel": f"streamkl_{dominant}_kernel", "bound": "tensor",
+            "achieved": bwd_tf if dominant == "bwd" else fwd_tf,
+            "peak": peak_sus, "unit": "TFLOP/s",
+            "frac": (bwd_tf if dominant == "bwd" else fwd_tf) / peak_sus,
+            "traffic": traffic,
+            "peak_kind": f"{peak_kind} bf16 dense, sustained (kernel timed inside a long loop)"}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(skl, w, x, dev, stream, args.steps, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+               "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+               "dtype": "bf16", "data": "synthetic", "config": config_of(w, world),
+               "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+               "fwd_frac_peak": fwd_tf / peak_sus, "bwd_frac_peak": bwd_tf / peak_sus,
+               "fwd_frac_burst_peak": fwd_tf / peak_burst,
+               "bwd_frac_burst_peak": bwd_tf / peak_burst,
+               "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+               "gpu_launches": 2 * args.steps,
+               "extra_hbm_bytes": 3 * 4 * w.bh * w.N_Q,
+               "impl": "ours"}
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(skl, w, x, dev, stream, steps, world):
+    """Same metric through the public API from pinned host buffers: every step copies
+    the inputs host->device, runs forward + backward, and reads the KL rows back."""
+    host = {k: v.pin_memory() for k, v in x.items()}
+    d = {k: torch.empty_like(v, device=dev) for k, v in x.items()}
+    kl_h = torch.empty(w.B, w.H, w.N_Q, dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = kl_h.numel() * 4
+
+    def one():
+        for k in d:
+            d[k].copy_(host[k], non_blocking=True)
+        kl, lt, ls = skl.streamkl_fwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T,
+                                      w.scale_S, w.causal)
+        skl.streamkl_bwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S,
+                         w.causal, lt, ls, d["g"])
+        kl_h.copy_(kl, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    value = world * (flops_fwd(w) + flops_bwd(w)) * steps / (ms * 1e-3) / 1e12
+    return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps}
+
+
+def load_traffic(workload: str, which: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d.get(workload, {}).get(which)
+    except Exception:
+        return None
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,108 @@
+/*
+ * streamkl.h - C ABI of the StreamKL attention-KL library for NVIDIA B200 (sm_100a).
+ *
+ * The operation ("StreamKL: Fast and Memory-Efficient KL Divergence for Boosting
+ * Attention Distillation", abstract): for every batch b, head h and query row i,
+ *
+ *   s_T[i,j] = scale_T * <q_T[i], k_T[j]>,   s_S[i,j] = scale_S * <q_S[i], k_S[j]>
+ *   J(i)     = { j < N_K : !causal || j <= i + N_K - N_Q }     (bottom-right causal)
+ *   P_X[i,:] = softmax over J(i) of s_X[i,:]                   (X = T teacher, S student)
+ *   KL[i]    = sum_{j in J(i)} P_T[i,j] * (log P_T[i,j] - log P_S[i,j])
+ *
+ * computed without materialising either N_Q x N_K matrix. The forward streams key
+ * tiles past a resident query tile and keeps an online state per row (the abstract's
+ * "online formulation for the coupled two-distribution KL reduction" and "single
+ * one-pass forward kernel"). The backward recomputes both probability tiles from the
+ * saved log-sum-exps (the abstract's "recomputes attention probabilities
+ * tile-by-tile"). The teacher is frozen: only the student gets gradients.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All pointers are DEVICE pointers on the current CUDA device, owned by the caller.
+ *   The library allocates no device memory. Extra device memory beyond the caller's
+ *   inputs and outputs is O(1) (one error word per device); the only state passed
+ *   from forward to backward is the caller's O(B*H*N_Q) row statistics.
+ * - Layout: q_t [B,H,N_Q,d_T], k_t [B,H,N_K,d_T], q_s [B,H,N_Q,d_S], k_s [B,H,N_K,d_S],
+ *   contiguous row-major bf16 (d innermost). Row statistics and g are contiguous fp32
+ *   [B,H,N_Q]. Gradients are contiguous fp32.
+ * - Supported: d_T, d_S in {64, 128}; B, H, N_Q, N_K >= 1; B*H*max(N_Q,N_K) < 2^31;
+ *   any finite scale_T, scale_S. N_Q and N_K need not be multiples of any tile size.
+ * - Every input/output pointer must be 16-byte aligned.
+ * - Calls are asynchronous on `stream`: argument checks happen on the host before any
+ *   launch and return a status without touching device memory; launch failures are
+ *   reported through cudaGetLastError as STREAMKL_ERR_LAUNCH. A kernel that hits its
+ *   internal watchdog (a pipeline wait that exceeds its bound) stops early and records
+ *   STREAMKL_ERR_TIMEOUT in a device-side error word, read with
+ *   streamkl_device_status(); it never traps.
+ * - Rows with an empty J(i) (only causal with N_Q > N_K) get KL = 0, LSE = -inf and a
+ *   zero gradient. KL is reported unclamped (rounding can make it slightly negative).
+ */
+#ifndef STREAMKL_H
+#define STREAMKL_H
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  STREAMKL_OK = 0,
+  STREAMKL_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, non-finite scale */
+  STREAMKL_ERR_UNSUPPORTED = 2, /* head dim outside {64,128} or sizes beyond the limits */
+  STREAMKL_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned */
+  STREAMKL_ERR_LAUNCH = 4,      /* the CUDA runtime rejected a launch or a set-up call */
+  STREAMKL_ERR_TIMEOUT = 5      /* a kernel watchdog fired (see streamkl_device_status) */
+} streamkl_status;
+
+/*
+ * Forward. Online coupled statistics per query row (running maxima m_T, m_S, sums
+ * l_T, l_S and A = sum_j 2^(t_T - m_T) (t_T - t_S) in base-2 units), finalised as
+ *   LSE_X = ln2 * (m_X + log2 l_X),   KL = ln2 * A / l_T - LSE_T + LSE_S,
+ * i.e. KL = E_{P_T}[s_T - s_S] - LSE_T + LSE_S.
+ *
+ * Outputs (caller-allocated fp32 [B,H,N_Q], fully overwritten):
+ *   kl     per-row KL(P_T || P_S) in nats;
+ *   lse_t  per-row natural-log log-sum-exp of s_T over J(i);
+ *   lse_s  per-row natural-log log-sum-exp of s_S over J(i).
+ * lse_t / lse_s are the only state streamkl_bwd needs.
+ */
+streamkl_status streamkl_fwd(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
+                             int B, int H, int N_Q, int N_K, int d_T, int d_S,
+                             float scale_T, float scale_S, int causal,
+                             float* kl, float* lse_t, float* lse_s, cudaStream_t stream);
+
+/*
+ * Backward (teacher frozen). With g[i] = dLoss/dKL[i] (fp32 [B,H,N_Q]) and the forward's
+ * lse_t / lse_s, recomputes P_T = exp(s_T - LSE_T) and P_S = exp(s_S - LSE_S) tile by
+ * tile and forms
+ *   dS[i,j] = g[i] * scale_S * (P_S[i,j] - P_T[i,j])   on J(i), 0 elsewhere,
+ *   dq_s = dS K_S   (fp32 [B,H,N_Q,d_S], fully overwritten: zeroed on `stream` first),
+ *   dk_s = dS^T Q_S (fp32 [B,H,N_K,d_S], fully overwritten).
+ * dq_s is accumulated with fp32 atomic reductions, so its low bits can differ between
+ * runs; dk_s is deterministic.
+ */
+streamkl_status streamkl_bwd(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
+                             int B, int H, int N_Q, int N_K, int d_T, int d_S,
+                             float scale_T, float scale_S, int causal,
+                             const float* lse_t, const float* lse_s, const float* g,
+                             float* dq_s, float* dk_s, cudaStream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char* streamkl_status_string(streamkl_status status);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error word.
+ * Returns STREAMKL_OK, STREAMKL_ERR_TIMEOUT if a kernel watchdog fired since the last
+ * call, or STREAMKL_ERR_LAUNCH if the stream reports a CUDA error.
+ */
+streamkl_status streamkl_device_status(cudaStream_t stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int streamkl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STREAMKL_H */

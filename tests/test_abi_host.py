@@ -1,0 +1,92 @@
+"""C-ABI library: loads, exports every declared symbol, host-side argument checks.
+
+No CUDA call is made here: every case below is rejected on the host before any
+launch, so these run on a machine without a GPU.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import attention_kl_divergence_fwd_b200 as skl
+from attention_kl_divergence_fwd_b200 import build as skl_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "streamkl.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    skl_build.build()
+    return skl.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(streamkl_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_exports():
+    assert declared_functions() == sorted(skl.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", skl.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (streamkl_[a-z_]+)\b", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert skl.status_string(code)
+    assert skl.version() >= 100
+
+
+P = 1 << 12  # a fake, 16-byte aligned, non-null address: never dereferenced on these paths
+
+
+def fwd(**kw):
+    a = dict(q_t=P, k_t=P, q_s=P, k_s=P, B=1, H=1, N_Q=128, N_K=128, d_T=128, d_S=128,
+             scale_T=0.1, scale_S=0.1, causal=False, kl=P, lse_t=P, lse_s=P, stream=0)
+    a.update(kw)
+    return skl.streamkl_fwd_raw(**a)
+
+
+def bwd(**kw):
+    a = dict(q_t=P, k_t=P, q_s=P, k_s=P, B=1, H=1, N_Q=128, N_K=128, d_T=128, d_S=128,
+             scale_T=0.1, scale_S=0.1, causal=False, lse_t=P, lse_s=P, g=P, dq_s=P, dk_s=P,
+             stream=0)
+    a.update(kw)
+    return skl.streamkl_bwd_raw(**a)
+
+
+@pytest.mark.parametrize("fn", [fwd, bwd])
+def test_host_validation(lib, fn):
+    assert fn(q_t=0) == 1
+    assert fn(k_s=0) == 1
+    assert fn(B=0) == 1
+    assert fn(N_Q=0) == 1
+    assert fn(N_K=-5) == 1
+    assert fn(scale_T=float("nan")) == 1
+    assert fn(scale_S=float("inf")) == 1
+    assert fn(d_T=96) == 2
+    assert fn(d_S=32) == 2
+    assert fn(d_T=256) == 2
+    assert fn(B=1 << 12, H=1 << 12) == 2          # B*H beyond the grid limit
+    assert fn(H=4096, N_Q=1 << 20) == 2            # B*H*N beyond int32 row indices
+    assert fn(q_t=P + 8) == 3
+    assert fn(k_s=P + 2) == 3
+
+
+def test_host_validation_outputs(lib):
+    assert fwd(kl=0) == 1
+    assert fwd(lse_s=P + 4) == 3
+    assert bwd(g=0) == 1
+    assert bwd(dk_s=P + 12) == 3
+    assert bwd(lse_t=0) == 1

@@ -1,0 +1,187 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI (needs a B200).
+
+Tolerances (bf16 inputs, fp32 accumulation, bf16 dS operand in the backward):
+  KL    : |GPU - ref| <= 1e-4 or <= 2e-3 * |ref| per row
+  LSE   : |GPU - ref| <= 1e-4 + 1e-5 * |ref| per row
+  dQ_S, dK_S : relative Frobenius error <= 1e-2
+Small cases compare every output; the five full-size workloads run in the same
+launch configuration as bench.py and compare sampled rows the oracle computes one
+by one, plus properties that hold at any size.
+"""
+import math
+
+import pytest
+import torch
+
+import attention_kl_divergence_fwd_b200 as skl
+from oracle import oracle_bwd, oracle_dk_rows, oracle_fwd, oracle_rows
+from workloads import WORKLOADS, WORKLOAD_LIST, make_inputs, sample_keys, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+KL_ABS, KL_REL = 1e-4, 2e-3
+LSE_ABS, LSE_REL = 1e-4, 1e-5
+GRAD_REL = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from attention_kl_divergence_fwd_b200 import build
+    build.build()
+    skl.load_library()
+
+
+def to_dev(x):
+    return {k: v.cuda() for k, v in x.items()}
+
+
+def run_gpu(w, x, with_bwd=True):
+    d = to_dev(x)
+    kl, lt, ls = skl.streamkl_fwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S,
+                                  w.causal)
+    out = {"kl": kl, "lse_t": lt, "lse_s": ls}
+    if with_bwd:
+        dq, dk = skl.streamkl_bwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S,
+                                  w.causal, lt, ls, d["g"])
+        out.update(dq=dq, dk=dk)
+    assert skl.device_status() == 0
+    return {k: v.cpu().double() for k, v in out.items()}
+
+
+def check_kl(got, ref):
+    err = (got - ref).abs()
+    ok = (err <= KL_ABS) | (err <= KL_REL * ref.abs())
+    assert bool(ok.all()), f"KL mismatch: max abs err {err.max().item():.3e}"
+
+
+def check_lse(got, ref):
+    fin = torch.isfinite(ref)
+    assert torch.equal(fin, torch.isfinite(got)), "LSE finiteness differs"
+    assert torch.equal(got[~fin], ref[~fin])
+    err = (got[fin] - ref[fin]).abs()
+    assert bool((err <= LSE_ABS + LSE_REL * ref[fin].abs()).all()), f"LSE err {err.max():.3e}"
+
+
+def rel_fro(got, ref):
+    n = ref.norm().item()
+    return (got - ref).norm().item() / (n if n > 0 else 1.0)
+
+
+def check_full(w, x, with_bwd=True):
+    g = run_gpu(w, x, with_bwd)
+    args = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S, w.causal)
+    kl, lt, ls = oracle_fwd(*args)
+    check_kl(g["kl"], kl)
+    check_lse(g["lse_t"], lt)
+    check_lse(g["lse_s"], ls)
+    if with_bwd:
+        dq, dk = oracle_bwd(*args, x["g"])
+        assert rel_fro(g["dq"], dq) <= GRAD_REL, rel_fro(g["dq"], dq)
+        assert rel_fro(g["dk"], dk) <= GRAD_REL, rel_fro(g["dk"], dk)
+    return g
+
+
+# ---------------------------------------------------------------- small cases
+
+def test_tiny_workload_full():
+    w = WORKLOADS["tiny_n256_d64"]
+    check_full(w, make_inputs(w))
+
+
+BASE = WORKLOADS["b2h16_n4096_d128_causal"]
+
+
+@pytest.mark.parametrize("nq,nk,dt,ds,causal", [
+    (300, 300, 128, 128, True),      # ragged tail, diagonal tiles
+    (300, 300, 128, 128, False),
+    (333, 517, 128, 64, False),      # mismatched head dims, ragged keys
+    (517, 333, 64, 128, True),       # N_Q > N_K: empty rows at the top
+    (200, 700, 64, 64, True),        # N_Q < N_K: bottom-right causal
+    (1, 1, 128, 128, True),
+    (1, 1000, 64, 64, False),
+    (777, 1, 128, 128, True),
+    (640, 640, 128, 128, True),      # exact multiples of every tile
+])
+def test_shapes_full(nq, nk, dt, ds, causal):
+    w = BASE.with_sizes(B=1, H=2, N_Q=nq, N_K=nk, d_T=dt, d_S=ds, causal=causal,
+                        scale_T=1 / math.sqrt(dt), scale_S=1 / math.sqrt(ds),
+                        student="independent" if dt != ds else "perturb")
+    check_full(w, make_inputs(w, seed=nq * 7 + nk))
+
+
+def test_negative_and_zero_scales():
+    w = BASE.with_sizes(B=1, H=2, N_Q=260, N_K=260, scale_T=-0.09, scale_S=0.0, causal=True)
+    check_full(w, make_inputs(w, seed=5))
+    w = BASE.with_sizes(B=1, H=1, N_Q=130, N_K=390, scale_T=0.2, scale_S=-0.05, causal=False)
+    check_full(w, make_inputs(w, seed=6))
+
+
+def test_large_scores():
+    """Peaked distributions (|s| up to ~50): exercises the online max and rescaling."""
+    w = BASE.with_sizes(B=1, H=2, N_Q=384, N_K=384, scale_T=0.5, scale_S=0.4, causal=True,
+                        student="independent")
+    check_full(w, make_inputs(w, seed=8))
+
+
+def test_identical_inputs_exact_zero():
+    w = BASE.with_sizes(B=2, H=2, N_Q=333, N_K=333, causal=True)
+    x = make_inputs(w, seed=3)
+    x["q_s"], x["k_s"] = x["q_t"].clone(), x["k_t"].clone()
+    g = run_gpu(w, x)
+    assert torch.all(g["kl"] == 0)
+    assert torch.equal(g["lse_t"], g["lse_s"])
+    assert torch.all(g["dq"] == 0) and torch.all(g["dk"] == 0)
+
+
+def test_repeatable_and_no_allocation():
+    """The library allocates no device memory; dK and KL are bitwise repeatable."""
+    w = BASE.with_sizes(B=1, H=4, N_Q=1000, N_K=1000, causal=True)
+    d = to_dev(make_inputs(w, seed=4))
+    a = (d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal)
+    kl, lt, ls = skl.streamkl_fwd(*a)
+    dq, dk = skl.streamkl_bwd(*a, lt, ls, d["g"])
+    outs = [torch.empty_like(kl) for _ in range(3)] + [torch.full_like(dq, 7.0),
+                                                        torch.full_like(dk, 7.0)]
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        kl2, lt2, ls2 = skl.streamkl_fwd(*a, kl=outs[0], lse_t=outs[1], lse_s=outs[2])
+        dq2, dk2 = skl.streamkl_bwd(*a, lt, ls, d["g"], dq_s=outs[3], dk_s=outs[4])
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
+    assert skl.device_status() == 0
+    assert torch.equal(kl, kl2) and torch.equal(lt, lt2) and torch.equal(dk, dk2)
+    assert rel_fro(dq2.double(), dq.double()) < 1e-5
+    # every buffer above existed before free0; the library adds nothing on the device
+    assert free1 == free0
+
+
+# ----------------------------------------------------------- full-size workloads
+
+def _sampled(w, rows_n=256, dk_heads=2, dk_keys=64):
+    x = make_inputs(w)
+    g = run_gpu(w, x)
+    args = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S, w.causal, x["g"])
+    rows = sample_rows(w, rows_n)
+    kl, lt, ls, dq = oracle_rows(*args, rows)
+    idx = torch.tensor([bh * w.N_Q + i for bh, i in rows])
+    check_kl(g["kl"].reshape(-1)[idx], kl)
+    check_lse(g["lse_t"].reshape(-1)[idx], lt)
+    check_lse(g["lse_s"].reshape(-1)[idx], ls)
+    assert rel_fro(g["dq"].reshape(-1, w.d_S)[idx], dq) <= GRAD_REL
+    for bh, keys in sample_keys(w, dk_heads, dk_keys):
+        ref = oracle_dk_rows(*args, bh, keys, row_block=512)
+        got = g["dk"].reshape(w.bh, w.N_K, w.d_S)[bh, keys]
+        assert rel_fro(got, ref) <= GRAD_REL
+    # properties that hold at any size
+    assert g["kl"].min().item() >= -1e-5
+    assert torch.isfinite(g["kl"]).all() and torch.isfinite(g["dq"]).all()
+    col = g["dk"].reshape(w.bh, w.N_K, w.d_S).sum(dim=1).abs().max().item()
+    assert col <= 4e-3 * g["dk"].abs().max().item() * math.sqrt(w.N_K)
+    return g
+
+
+@pytest.mark.parametrize("name", [w.name for w in WORKLOAD_LIST[1:]])
+def test_full_size_workload(name):
+    w = WORKLOADS[name]
+    _sampled(w, dk_heads=1 if w.N_K > 20000 else 2)
