@@ -8,18 +8,21 @@
 //     dS[i,j] = g[i] * scale_S * (P_S[i,j] - P_T[i,j]),   P_X = 2^(t_X - LSE_X*log2 e)
 //     dQ_S = dS K_S,   dK_S = dS^T Q_S.
 //
-// CTA = one tile of 128 keys of one (batch, head), resident in shared memory. It
-// walks the 128-row query tiles that can see those keys. Per query tile:
-//   1. tensor core: S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T into TMEM (keys on lanes);
-//   2. two warpgroups (one thread per key, 64 query columns each) recompute P_T, P_S,
-//      form dS^T in registers and store it to shared memory as bf16;
-//   3. tensor core: dK_S += dS^T Q_S (TMEM accumulator over all query tiles) and
-//      dQ_part = dS K_S (TMEM);
-//   4. the same warpgroups add dQ_part into dq_s with fp32 vector reductions.
-// The score tiles of step s+1 are computed while the warpgroups work on step s.
+// CTA = one tile of 128 keys of one (batch, head), resident in shared memory. It walks
+// the 64-row query tiles ("steps") that can see those keys. Per step s:
+//   1. tensor core: S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T into TMEM buffer s&1
+//      (keys on the 128 lanes, 64 query columns);
+//   2. warpgroup s&1 (one thread per key) recomputes P_T, P_S, forms dS^T in registers
+//      and stores it as bf16 into shared-memory buffer s&1;
+//   3. tensor core: dK_S += dS^T Q_S (TMEM accumulator over all steps) and
+//      dQ^T_part = K_S^T dS^T into TMEM buffer s&1 (d_S on the lanes, queries on columns);
+//   4. the same warpgroup adds dQ^T_part into dq_s: one fp32 reduction per lane, 32
+//      consecutive d values (one 128-byte line) per warp instruction.
+// Score tiles, dS tiles and dQ parts are double-buffered, so the two warpgroups work on
+// alternate steps while the tensor core computes the next ones.
 //
-// Warp roles (320 threads): warps 0-3 and 4-7 statistics/dS (query columns 0-63 and
-// 64-127), warp 8 TMA producer + row-statistics loader, warp 9 TMEM allocator + MMA.
+// Warp roles (320 threads): warps 0-3 even steps, warps 4-7 odd steps, warp 8 TMA
+// producer + row-statistics loader, warp 9 TMEM allocator + MMA issuer.
 #pragma once
 
 #include "ptx.cuh"
@@ -33,7 +36,7 @@ struct BwdArgs {
   float cT, cS;     // |scale| * log2(e)
   float scale_S;    // signed student scale (folded into G = g * scale_S)
   int n_ktiles;     // ceil(N_K / 128)
-  int n_qtiles;     // ceil(N_Q / 128)
+  int n_qtiles;     // ceil(N_Q / 64)
   const float* lse_t;
   const float* lse_s;
   const float* g;
@@ -44,36 +47,39 @@ struct BwdArgs {
 template <int DT, int DS>
 struct BwdCfg {
   static constexpr int BN = 128;  // keys per CTA (TMEM lanes)
-  static constexpr int BM = 128;  // queries per step
+  static constexpr int BM = 64;   // queries per step
+  static constexpr int NQST = 3;  // query-tile stages
   static constexpr int KT_TILE = BN * DT * 2;
   static constexpr int KS_TILE = BN * DS * 2;
   static constexpr int QT_TILE = BM * DT * 2;
   static constexpr int QS_TILE = BM * DS * 2;
-  static constexpr int DS_TILE = BN * BM * 2;
-  static constexpr int STATS = 3 * BM * 4;  // -LSE_T*log2e, -LSE_S*log2e, g*scale_S
+  static constexpr int Q_STAGE = QT_TILE + QS_TILE;
+  static constexpr int DS_TILE = BN * BM * 2;  // bf16 dS^T [128 keys][64 queries]
+  static constexpr int STATS = 3 * BM * 4;     // -LSE_T*log2e, -LSE_S*log2e, g*scale_S
   static constexpr int OFF_KT = 0;
   static constexpr int OFF_KS = OFF_KT + KT_TILE;
-  static constexpr int OFF_QT = OFF_KS + KS_TILE;
-  static constexpr int OFF_QS = OFF_QT + QT_TILE;        // two slots
-  static constexpr int OFF_DS = OFF_QS + 2 * QS_TILE;
-  static constexpr int OFF_ST = OFF_DS + DS_TILE;         // two slots
-  static constexpr int OFF_BAR = OFF_ST + 2 * STATS;
+  static constexpr int OFF_Q = OFF_KS + KS_TILE;           // NQST stages {Q_T, Q_S}
+  static constexpr int OFF_DS = OFF_Q + NQST * Q_STAGE;    // two dS tiles
+  static constexpr int OFF_ST = OFF_DS + 2 * DS_TILE;      // NQST statistics slots
+  static constexpr int OFF_BAR = OFF_ST + NQST * STATS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = 1024 + OFF_BAR + BAR_BYTES;
   static constexpr int THREADS = 320;
-  // TMEM columns
-  static constexpr int TM_ST = 0, TM_SS = 128, TM_DK = 256, TM_DQ = 384;
+  // TMEM columns: S_T^T / S_S^T per buffer, dK_S, dQ^T per buffer.
+  static constexpr int TM_S = 0;          // buffer b: [128b, 128b+64) S_T, [+64, +128) S_S
+  static constexpr int TM_DK = 256;       // d_S columns
+  static constexpr int TM_DQ = 256 + DS;  // buffer b: + 64 b
+  static constexpr int DQ_M = DS;         // M of the dQ^T MMA (64 uses half the lanes)
+  static_assert(TM_DQ + 2 * BM <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 struct BwdBars {
   uint64_t k_full;
-  uint64_t qt_full, qt_empty;
-  uint64_t qs_full[2], qs_empty[2];
-  uint64_t st_full[2], st_empty[2];
-  uint64_t s_full, s_free;
-  uint64_t ds_full, ds_empty;
-  uint64_t dq_full, dq_free;
+  uint64_t q_full[3], q_empty[3], st_full[3];
+  uint64_t s_full[2], s_free[2];
+  uint64_t ds_full[2], ds_empty[2];
+  uint64_t dq_full[2], dq_free[2];
   uint64_t dk_full;
   uint64_t drain;
   uint32_t tmem_base;
@@ -118,20 +124,19 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->k_full), 1);
-    mbar_init(smem_u32(&bars->qt_full), 1);
-    mbar_init(smem_u32(&bars->qt_empty), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bars->qs_full[i]), 1);
-      mbar_init(smem_u32(&bars->qs_empty[i]), 1);
+    for (int i = 0; i < C::NQST; ++i) {
+      mbar_init(smem_u32(&bars->q_full[i]), 1);
+      mbar_init(smem_u32(&bars->q_empty[i]), 1);
       mbar_init(smem_u32(&bars->st_full[i]), 32);
-      mbar_init(smem_u32(&bars->st_empty[i]), 8);
     }
-    mbar_init(smem_u32(&bars->s_full), 1);
-    mbar_init(smem_u32(&bars->s_free), 8);
-    mbar_init(smem_u32(&bars->ds_full), 8);
-    mbar_init(smem_u32(&bars->ds_empty), 1);
-    mbar_init(smem_u32(&bars->dq_full), 1);
-    mbar_init(smem_u32(&bars->dq_free), 8);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bars->s_full[b]), 1);
+      mbar_init(smem_u32(&bars->s_free[b]), 4);
+      mbar_init(smem_u32(&bars->ds_full[b]), 4);
+      mbar_init(smem_u32(&bars->ds_empty[b]), 1);
+      mbar_init(smem_u32(&bars->dq_full[b]), 1);
+      mbar_init(smem_u32(&bars->dq_free[b]), 4);
+    }
     mbar_init(smem_u32(&bars->dk_full), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort_flag = 0;
@@ -149,7 +154,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   if (warp == 8) {
     // --------------------------------------- TMA producer + row-statistics loader
     const uint64_t keep = l2_policy_evict_last();
-    int qt_issued = 0, qs_issued = 0;
+    int issued = 0;
     bool ok = true;
     if (lane == 0) {
       tma_prefetch_desc(&map_qt);
@@ -164,37 +169,30 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         tma_load_3d(sb + C::OFF_KS + blk * (C::BN * 128), &map_ks, kb, blk * 64, k0, bh, keep);
     }
     const float LOG2E = 1.4426950408889634f;
-    for (int s = 0; s < n_steps && ok; ++s) {
+    for (int s = 0; s < n_steps; ++s) {
+      const int st = s % C::NQST;
       const int i0 = (jq_begin + s) * C::BM;
-      // Lane 0 does every wait of this warp and issues the copies; the verdict is
-      // then shared so the whole warp leaves the loop together.
+      // Lane 0 does the waits and issues the copies; the verdict is shared so the warp
+      // leaves the loop together (the shuffle also orders the slot reuse below).
       if (lane == 0) {
-        if (!mbar_wait(smem_u32(&bars->qt_empty), (s & 1) ^ 1)) {
+        if (!mbar_wait(smem_u32(&bars->q_empty[st]), ((s / C::NQST) & 1) ^ 1)) {
           ok = false;
+          skl_fail_b(abort_flag);
         } else {
-          const uint32_t fb = smem_u32(&bars->qt_full);
-          mbar_arrive_expect_tx(fb, C::QT_TILE);
+          const uint32_t fb = smem_u32(&bars->q_full[st]);
+          const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
+          mbar_arrive_expect_tx(fb, C::Q_STAGE);
           for (int blk = 0; blk < DT / 64; ++blk)
-            tma_load_3d(sb + C::OFF_QT + blk * (C::BM * 128), &map_qt, fb, blk * 64, i0, bh, keep);
-          qt_issued = s + 1;
-        }
-        if (ok && !mbar_wait(smem_u32(&bars->qs_empty[s & 1]), ((s >> 1) & 1) ^ 1)) {
-          ok = false;
-        } else if (ok) {
-          const uint32_t fb = smem_u32(&bars->qs_full[s & 1]);
-          mbar_arrive_expect_tx(fb, C::QS_TILE);
+            tma_load_3d(q_base + blk * (C::BM * 128), &map_qt, fb, blk * 64, i0, bh, keep);
           for (int blk = 0; blk < DS / 64; ++blk)
-            tma_load_3d(sb + C::OFF_QS + (s & 1) * C::QS_TILE + blk * (C::BM * 128), &map_qs, fb,
-                        blk * 64, i0, bh, keep);
-          qs_issued = s + 1;
+            tma_load_3d(q_base + C::QT_TILE + blk * (C::BM * 128), &map_qs, fb, blk * 64, i0, bh,
+                        keep);
+          issued = s + 1;
         }
-        if (ok && !mbar_wait(smem_u32(&bars->st_empty[s & 1]), ((s >> 1) & 1) ^ 1)) ok = false;
-        if (!ok) skl_fail_b(abort_flag);
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      // Row statistics of this query tile: -LSE_T*log2e, -LSE_S*log2e, g*scale_S.
-      float* st = stats + (s & 1) * (3 * C::BM);
+      float* sts = stats + st * (3 * C::BM);
 #pragma unroll
       for (int r = 0; r < C::BM / 32; ++r) {
         const int qi = r * 32 + lane;
@@ -210,83 +208,76 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
             gs = args.g[o] * args.scale_S;
           }
         }
-        st[qi] = nlt;
-        st[C::BM + qi] = nls;
-        st[2 * C::BM + qi] = gs;
+        sts[qi] = nlt;
+        sts[C::BM + qi] = nls;
+        sts[2 * C::BM + qi] = gs;
       }
-      mbar_arrive(smem_u32(&bars->st_full[s & 1]));
+      mbar_arrive(smem_u32(&bars->st_full[st]));
     }
     if (lane == 0 && *abort_flag) {
+      // Let every copy this thread started land before the CTA can exit.
       mbar_wait(smem_u32(&bars->k_full), 0);
-      if (qt_issued > 0) mbar_wait(smem_u32(&bars->qt_full), (qt_issued - 1) & 1);
-      for (int s = max(0, qs_issued - 2); s < qs_issued; ++s)
-        mbar_wait(smem_u32(&bars->qs_full[s & 1]), (s >> 1) & 1);
+      for (int s = max(0, issued - C::NQST); s < issued; ++s)
+        mbar_wait(smem_u32(&bars->q_full[s % C::NQST]), (s / C::NQST) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (elect_one()) {
-      const uint32_t t_st = tmem + C::TM_ST, t_ss = tmem + C::TM_SS;
-      const uint32_t t_dk = tmem + C::TM_DK, t_dq = tmem + C::TM_DQ;
-      const uint32_t s_kt = sb + C::OFF_KT, s_ks = sb + C::OFF_KS, s_qt = sb + C::OFF_QT;
-      const uint32_t s_ds = sb + C::OFF_DS;
+      const uint32_t s_kt = sb + C::OFF_KT, s_ks = sb + C::OFF_KS;
       bool ok = mbar_wait(smem_u32(&bars->k_full), 0);
-      // Score tiles of step s: S_T^T = K_T Q_T^T, S_S^T = K_S Q_S^T (keys on lanes).
+      // S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T of step s into TMEM buffer s&1.
       auto issue_scores = [&](int s) -> bool {
-        if (!mbar_wait(smem_u32(&bars->qt_full), s & 1)) return false;
-        if (!mbar_wait(smem_u32(&bars->qs_full[s & 1]), (s >> 1) & 1)) return false;
-        if (!mbar_wait(smem_u32(&bars->s_free), (s & 1) ^ 1)) return false;
+        const int st = s % C::NQST, b = s & 1;
+        if (!mbar_wait(smem_u32(&bars->q_full[st]), (s / C::NQST) & 1)) return false;
+        if (!mbar_wait(smem_u32(&bars->s_free[b]), ((s >> 1) & 1) ^ 1)) return false;
         tc_fence_after();
+        const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
+        const uint32_t d_t = tmem + C::TM_S + b * 128, d_s = d_t + 64;
 #pragma unroll
         for (int kk = 0; kk < DT / 16; ++kk) {
-          const uint32_t o = (kk >> 2) * (C::BN * 128) + (kk & 3) * 32;
-          umma_bf16_ss(t_st, sdesc_sw128(s_kt + o, 16, 1024), sdesc_sw128(s_qt + o, 16, 1024),
+          const uint32_t ka = (kk >> 2) * (C::BN * 128) + (kk & 3) * 32;
+          const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
+          umma_bf16_ss(d_t, sdesc_sw128(s_kt + ka, 16, 1024), sdesc_sw128(q_base + qa, 16, 1024),
                        idesc_st, kk > 0);
         }
-        umma_commit(smem_u32(&bars->qt_empty));
-        const uint32_t s_qs = sb + C::OFF_QS + (s & 1) * C::QS_TILE;
 #pragma unroll
         for (int kk = 0; kk < DS / 16; ++kk) {
-          const uint32_t o = (kk >> 2) * (C::BN * 128) + (kk & 3) * 32;
-          umma_bf16_ss(t_ss, sdesc_sw128(s_ks + o, 16, 1024), sdesc_sw128(s_qs + o, 16, 1024),
-                       idesc_ss, kk > 0);
+          const uint32_t ka = (kk >> 2) * (C::BN * 128) + (kk & 3) * 32;
+          const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
+          umma_bf16_ss(d_s, sdesc_sw128(s_ks + ka, 16, 1024),
+                       sdesc_sw128(q_base + C::QT_TILE + qa, 16, 1024), idesc_ss, kk > 0);
         }
-        umma_commit(smem_u32(&bars->s_full));
+        umma_commit(smem_u32(&bars->s_full[b]));
         return true;
       };
       if (ok && n_steps > 0) ok = issue_scores(0);
-      for (int s = 0; ok && s < n_steps; ++s) {
-        if (s + 1 < n_steps && !issue_scores(s + 1)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait(smem_u32(&bars->ds_full), s & 1)) {
-          ok = false;
-          break;
-        }
+      if (ok && n_steps > 1) ok = issue_scores(1);
+      for (int p = 0; ok && p < n_steps; ++p) {
+        const int pb = p & 1, pst = p % C::NQST;
+        if (!mbar_wait(smem_u32(&bars->ds_full[pb]), (p >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t s_qs = sb + C::OFF_QS + (s & 1) * C::QS_TILE;
-        // dK_S += dS^T Q_S : A = dS^T (keys x queries, K-major), B = Q_S (d x queries, MN-major)
+        const uint32_t s_ds = sb + C::OFF_DS + pb * C::DS_TILE;
+        const uint32_t s_qs = sb + C::OFF_Q + pst * C::Q_STAGE + C::QT_TILE;
+        // dK_S += dS^T Q_S : A = dS^T [keys][queries] K-major, B = Q_S [queries][d] MN-major.
 #pragma unroll
         for (int kk = 0; kk < C::BM / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(s_ds + (kk >> 2) * (C::BN * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sdesc_sw128(s_qs + kk * 2048, C::BM * 128, 1024);
-          umma_bf16_ss(t_dk, a, b, idesc_dk, (s > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ss(tmem + C::TM_DK, sdesc_sw128(s_ds + kk * 32, 16, 1024),
+                       sdesc_sw128(s_qs + kk * 2048, C::BM * 128, 1024), idesc_dk,
+                       (p > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(smem_u32(&bars->qs_empty[s & 1]));
-        if (!mbar_wait(smem_u32(&bars->dq_free), (s & 1) ^ 1)) {
-          ok = false;
-          break;
-        }
+        umma_commit(smem_u32(&bars->q_empty[pst]));
+        if (!mbar_wait(smem_u32(&bars->dq_free[pb]), ((p >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        // dQ_part = dS K_S : A = dS (queries x keys, MN-major), B = K_S (d x keys, MN-major)
+        // dQ^T = K_S^T dS^T : A = K_S [keys][d] MN-major, B = dS^T [keys][queries] MN-major.
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(s_ds + kk * 2048, C::BN * 128, 1024);
-          const uint64_t b = sdesc_sw128(s_ks + kk * 2048, C::BN * 128, 1024);
-          umma_bf16_ss(t_dq, a, b, idesc_dq, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tmem + C::TM_DQ + pb * C::BM,
+                       sdesc_sw128(s_ks + kk * 2048, C::BN * 128, 1024),
+                       sdesc_sw128(s_ds + kk * 2048, C::BN * 128, 1024), idesc_dq, kk > 0 ? 1u : 0u);
         }
-        umma_commit(smem_u32(&bars->ds_empty));
-        umma_commit(smem_u32(&bars->dq_full));
+        umma_commit(smem_u32(&bars->ds_empty[pb]));
+        umma_commit(smem_u32(&bars->dq_full[pb]));
+        if (p + 2 < n_steps && !issue_scores(p + 2)) { ok = false; break; }
       }
       if (!ok) skl_fail_b(abort_flag);
       umma_commit(smem_u32(&bars->dk_full));
@@ -295,123 +286,126 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     }
   } else {
     // ------------------------------------------------- dS / reduction warpgroups
-    const int half = warp >> 2;       // query columns [64*half, 64*half + 64) of each step
+    const int wg = warp >> 2;            // steps s with s&1 == wg
     const int quarter = warp & 3;
     const int kl = quarter * 32 + lane;  // key row within the tile = TMEM lane
     const int key = k0 + kl;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float cT = args.cT, cS = args.cS;
-    const uint32_t s_ds = sb + C::OFF_DS + half * (C::BN * 128) + (kl >> 3) * 1024 + (kl & 7) * 128;
-    constexpr int DQH = DS / 2;  // dQ / dK columns handled by this warpgroup
+    const uint32_t s_ds_row = sb + C::OFF_DS + wg * C::DS_TILE + kl * 128;
+    // dQ^T lanes are d: all 32 lanes of a quarter for d_S = 128; for d_S = 64 the M=64
+    // layout puts rows 16w..16w+15 on lanes 32w..32w+15.
+    const bool dq_lane_ok = (C::DQ_M == 128) || lane < 16;
+    const int dq_d = (C::DQ_M == 128) ? kl : quarter * 16 + lane;
 
-    auto drain_dq = [&](int s) -> bool {
-      if (!mbar_wait(smem_u32(&bars->dq_full), s & 1)) return false;
+    auto drain_dq = [&](int p) -> bool {
+      if (!mbar_wait(smem_u32(&bars->dq_full[wg]), (p >> 1) & 1)) return false;
       tc_fence_after();
-      uint32_t v[DQH];
-      if constexpr (DQH == 64) {
-        tmem_ld_2x32_wait(tmem + lane_off + C::TM_DQ + half * DQH,
-                          tmem + lane_off + C::TM_DQ + half * DQH + 32, v);
-      } else {
-        tmem_ld_32_wait(tmem + lane_off + C::TM_DQ + half * DQH, v);
-      }
+      uint32_t v[64];
+      tmem_ld_2x32_wait(tmem + lane_off + C::TM_DQ + wg * C::BM,
+                        tmem + lane_off + C::TM_DQ + wg * C::BM + 32, v);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->dq_free));
-      const int row = (jq_begin + s) * C::BM + kl;  // dQ lanes are query rows
-      if (row < args.N_Q) {
-        float* dst = args.dq_s + ((size_t)bh * args.N_Q + row) * DS + half * DQH;
+      if (lane == 0) mbar_arrive(smem_u32(&bars->dq_free[wg]));
+      if (dq_lane_ok) {
+        const int i0 = (jq_begin + p) * C::BM;
+        const int nrows = min(C::BM, args.N_Q - i0);
+        float* dst = args.dq_s + ((size_t)bh * args.N_Q + i0) * DS + dq_d;
 #pragma unroll
-        for (int c = 0; c < DQH; c += 4)
-          red_add_v4(dst + c, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                     __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+        for (int c = 0; c < C::BM; ++c)
+          if (c < nrows) red_add_f32(dst + (size_t)c * DS, __uint_as_float(v[c]));
       }
       return true;
     };
 
     bool ok = true;
-    for (int s = 0; s < n_steps; ++s) {
-      const int i0 = (jq_begin + s) * C::BM + half * 64;  // first query column of this thread
-      if (!mbar_wait(smem_u32(&bars->s_full), s & 1)) { ok = false; break; }
+    int last = -1;
+    for (int s = wg; s < n_steps; s += 2) {
+      const int st = s % C::NQST;
+      const int i0 = (jq_begin + s) * C::BM;  // first query column of this step
+      if (!mbar_wait(smem_u32(&bars->s_full[wg]), (s >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      uint32_t vt[64], vs[64];
-      tmem_ld_2x32_wait(tmem + lane_off + C::TM_ST + half * 64,
-                        tmem + lane_off + C::TM_ST + half * 64 + 32, vt);
-      tmem_ld_2x32_wait(tmem + lane_off + C::TM_SS + half * 64,
-                        tmem + lane_off + C::TM_SS + half * 64 + 32, vs);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->s_free));
-
-      if (!mbar_wait(smem_u32(&bars->st_full[s & 1]), (s >> 1) & 1)) { ok = false; break; }
-      const float* st = stats + (s & 1) * (3 * C::BM) + half * 64;
+      if (!mbar_wait(smem_u32(&bars->st_full[st]), (s / C::NQST) & 1)) { ok = false; break; }
+      const float* sts = stats + st * (3 * C::BM);
 
       // Query column c is allowed for this key iff i0 + c >= key - off.
       const bool need_mask = args.causal && (i0 + args.off < k0 + C::BN - 1);
       const int cmin = need_mask ? (key - args.off - i0) : -1;
       uint32_t packed[32];  // dS^T row of this key, 64 bf16 values
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {  // 8 query columns = one 16-byte chunk per iteration
-        const float4 nlt0 = *reinterpret_cast<const float4*>(st + u * 8);
-        const float4 nlt1 = *reinterpret_cast<const float4*>(st + u * 8 + 4);
-        const float4 nls0 = *reinterpret_cast<const float4*>(st + C::BM + u * 8);
-        const float4 nls1 = *reinterpret_cast<const float4*>(st + C::BM + u * 8 + 4);
-        const float4 g0 = *reinterpret_cast<const float4*>(st + 2 * C::BM + u * 8);
-        const float4 g1 = *reinterpret_cast<const float4*>(st + 2 * C::BM + u * 8 + 4);
-        const float nlt[8] = {nlt0.x, nlt0.y, nlt0.z, nlt0.w, nlt1.x, nlt1.y, nlt1.z, nlt1.w};
-        const float nls[8] = {nls0.x, nls0.y, nls0.z, nls0.w, nls1.x, nls1.y, nls1.z, nls1.w};
-        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-        float d[8];
+      for (int h = 0; h < 2; ++h) {  // 32 query columns of S_T and S_S per pass
+        uint32_t v[64];             // v[0..31] teacher scores, v[32..63] student scores
+        tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + wg * 128 + 32 * h,
+                          tmem + lane_off + C::TM_S + wg * 128 + 64 + 32 * h, v);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int c = u * 8 + e;
-          const float pT = ex2_approx(fmaf(__uint_as_float(vt[c]), cT, nlt[e]));
-          const float pS = ex2_approx(fmaf(__uint_as_float(vs[c]), cS, nls[e]));
-          float ds = gg[e] * (pS - pT);
-          if (need_mask && c < cmin) ds = 0.f;
-          d[e] = ds;
+        for (int u4 = 0; u4 < 4; ++u4) {  // 8 query columns = one 16-byte chunk
+          const int u = 4 * h + u4;
+          const float4 nlt0 = *reinterpret_cast<const float4*>(sts + u * 8);
+          const float4 nlt1 = *reinterpret_cast<const float4*>(sts + u * 8 + 4);
+          const float4 nls0 = *reinterpret_cast<const float4*>(sts + C::BM + u * 8);
+          const float4 nls1 = *reinterpret_cast<const float4*>(sts + C::BM + u * 8 + 4);
+          const float4 g0 = *reinterpret_cast<const float4*>(sts + 2 * C::BM + u * 8);
+          const float4 g1 = *reinterpret_cast<const float4*>(sts + 2 * C::BM + u * 8 + 4);
+          const float nlt[8] = {nlt0.x, nlt0.y, nlt0.z, nlt0.w, nlt1.x, nlt1.y, nlt1.z, nlt1.w};
+          const float nls[8] = {nls0.x, nls0.y, nls0.z, nls0.w, nls1.x, nls1.y, nls1.z, nls1.w};
+          const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+          float d[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = u * 8 + e;
+            const float pT = ex2_approx(fmaf(__uint_as_float(v[u4 * 8 + e]), cT, nlt[e]));
+            const float pS = ex2_approx(fmaf(__uint_as_float(v[32 + u4 * 8 + e]), cS, nls[e]));
+            float ds = gg[e] * (pS - pT);
+            if (need_mask && c < cmin) ds = 0.f;
+            d[e] = ds;
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) packed[u * 4 + e] = pack_bf16x2(d[2 * e], d[2 * e + 1]);
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) packed[u * 4 + e] = pack_bf16x2(d[2 * e], d[2 * e + 1]);
       }
+      // The score buffer can take step s+2 once every lane has read it.
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->st_empty[s & 1]));
-      // The dS buffer is free once the previous step's dK/dQ MMAs have read it.
-      if (!mbar_wait(smem_u32(&bars->ds_empty), (s & 1) ^ 1)) { ok = false; break; }
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[wg]));
+      // The dS buffer is free once the dK/dQ MMAs of step s-2 have read it.
+      if (!mbar_wait(smem_u32(&bars->ds_empty[wg]), ((s >> 1) & 1) ^ 1)) { ok = false; break; }
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        st_shared_v4(s_ds + ((u ^ (kl & 7)) << 4), packed[4 * u], packed[4 * u + 1],
+        st_shared_v4(s_ds_row + ((u ^ (kl & 7)) << 4), packed[4 * u], packed[4 * u + 1],
                      packed[4 * u + 2], packed[4 * u + 3]);
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->ds_full));
-      if (s > 0 && !drain_dq(s - 1)) { ok = false; break; }
+      if (lane == 0) mbar_arrive(smem_u32(&bars->ds_full[wg]));
+      if (last >= 0 && !drain_dq(last)) { ok = false; break; }
+      last = s;
     }
-    if (ok && n_steps > 0 && !drain_dq(n_steps - 1)) ok = false;
+    if (ok && last >= 0 && !drain_dq(last)) ok = false;
 
     // dK_S rows of this key tile (TMEM lanes = keys); zero when no query sees them.
+    constexpr int DKH = DS / 2;  // dK columns handled by this warpgroup
     if (ok) {
-      uint32_t v[DQH];
+      uint32_t v[DKH];
       if (n_steps > 0) {
         if (!mbar_wait(smem_u32(&bars->dk_full), 0)) {
           ok = false;
         } else {
           tc_fence_after();
-          if constexpr (DQH == 64) {
-            tmem_ld_2x32_wait(tmem + lane_off + C::TM_DK + half * DQH,
-                              tmem + lane_off + C::TM_DK + half * DQH + 32, v);
+          if constexpr (DKH == 64) {
+            tmem_ld_2x32_wait(tmem + lane_off + C::TM_DK + wg * DKH,
+                              tmem + lane_off + C::TM_DK + wg * DKH + 32, v);
           } else {
-            tmem_ld_32_wait(tmem + lane_off + C::TM_DK + half * DQH, v);
+            tmem_ld_32_wait(tmem + lane_off + C::TM_DK + wg * DKH, v);
           }
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < DQH; ++c) v[c] = 0u;
+        for (int c = 0; c < DKH; ++c) v[c] = 0u;
       }
       if (ok && key < args.N_K) {
         float4* dst = reinterpret_cast<float4*>(args.dk_s + ((size_t)bh * args.N_K + key) * DS +
-                                                half * DQH);
+                                                wg * DKH);
 #pragma unroll
-        for (int c = 0; c < DQH; c += 4)
+        for (int c = 0; c < DKH; c += 4)
           dst[c / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
                                    __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
       }

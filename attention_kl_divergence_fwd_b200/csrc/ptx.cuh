@@ -246,6 +246,10 @@ __device__ __forceinline__ void red_add_v4(float* gaddr, float a, float b, float
                : "memory");
 }
 
+__device__ __forceinline__ void red_add_f32(float* gaddr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(gaddr), "f"(a) : "memory");
+}
+
 // Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

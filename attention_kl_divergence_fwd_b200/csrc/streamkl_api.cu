@@ -98,8 +98,8 @@ streamkl_status launch_bwd(const CUtensorMap* maps, const skl::BwdArgs& a, bool 
   if (!set_smem(kern, C::SMEM)) return STREAMKL_ERR_LAUNCH;
   const uint32_t i_st = skl::idesc_bf16_f32(128, C::BM, false, false, negT);
   const uint32_t i_ss = skl::idesc_bf16_f32(128, C::BM, false, false, negS);
-  const uint32_t i_dk = skl::idesc_bf16_f32(128, DS, false, true);
-  const uint32_t i_dq = skl::idesc_bf16_f32(128, DS, true, true);
+  const uint32_t i_dk = skl::idesc_bf16_f32(128, DS, false, true);   // dS^T Q_S
+  const uint32_t i_dq = skl::idesc_bf16_f32(DS, C::BM, true, true);  // K_S^T dS^T
   const long long grid = (long long)a.n_ktiles * a.BH;
   kern<<<dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream>>>(
       maps[0], maps[1], maps[2], maps[3], a, i_st, i_ss, i_dk, i_dq);
@@ -154,8 +154,8 @@ streamkl_status streamkl_bwd(const void* q_t, const void* k_t, const void* q_s, 
     return STREAMKL_ERR_MISALIGNED;
   const int bh = B * H;
   CUtensorMap maps[4];
-  if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 128) || !make_map(&maps[1], k_t, d_T, N_K, bh, 128) ||
-      !make_map(&maps[2], q_s, d_S, N_Q, bh, 128) || !make_map(&maps[3], k_s, d_S, N_K, bh, 128))
+  if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 64) || !make_map(&maps[1], k_t, d_T, N_K, bh, 128) ||
+      !make_map(&maps[2], q_s, d_S, N_Q, bh, 64) || !make_map(&maps[3], k_s, d_S, N_K, bh, 128))
     return STREAMKL_ERR_LAUNCH;
   if (cudaMemsetAsync(dq_s, 0, (size_t)bh * N_Q * d_S * sizeof(float), stream) != cudaSuccess)
     return STREAMKL_ERR_LAUNCH;
@@ -169,7 +169,7 @@ streamkl_status streamkl_bwd(const void* q_t, const void* k_t, const void* q_s, 
   a.cS = std::fabs(scale_S) * kLog2e;
   a.scale_S = scale_S;
   a.n_ktiles = (N_K + 127) / 128;
-  a.n_qtiles = (N_Q + 127) / 128;
+  a.n_qtiles = (N_Q + 63) / 64;
   a.lse_t = lse_t;
   a.lse_s = lse_s;
   a.g = g;
