@@ -21,8 +21,9 @@
 // Score tiles, dS tiles and dQ parts are double-buffered, so the two warpgroups work on
 // alternate steps while the tensor core computes the next ones.
 //
-// Warp roles (320 threads): warps 0-3 even steps, warps 4-7 odd steps, warp 8 TMA
-// producer + row-statistics loader, warp 9 TMEM allocator + MMA issuer.
+// Warp roles (352 threads): warps 0-3 even steps, warps 4-7 odd steps, warp 8 TMA
+// producer, warp 9 TMEM allocator + MMA issuer, warp 10 row-statistics loader (global
+// loads issued several steps ahead so their latency never reaches the pipeline).
 #pragma once
 
 #include "ptx.cuh"
@@ -48,7 +49,8 @@ template <int DT, int DS>
 struct BwdCfg {
   static constexpr int BN = 128;  // keys per CTA (TMEM lanes)
   static constexpr int BM = 64;   // queries per step
-  static constexpr int NQST = 3;  // query-tile stages
+  static constexpr int NQST = 4;  // query-tile stages
+  static constexpr int NSTS = 2;  // row-statistics slots
   static constexpr int KT_TILE = BN * DT * 2;
   static constexpr int KS_TILE = BN * DS * 2;
   static constexpr int QT_TILE = BM * DT * 2;
@@ -60,11 +62,11 @@ struct BwdCfg {
   static constexpr int OFF_KS = OFF_KT + KT_TILE;
   static constexpr int OFF_Q = OFF_KS + KS_TILE;           // NQST stages {Q_T, Q_S}
   static constexpr int OFF_DS = OFF_Q + NQST * Q_STAGE;    // two dS tiles
-  static constexpr int OFF_ST = OFF_DS + 2 * DS_TILE;      // NQST statistics slots
-  static constexpr int OFF_BAR = OFF_ST + NQST * STATS;
+  static constexpr int OFF_ST = OFF_DS + 2 * DS_TILE;      // NSTS statistics slots
+  static constexpr int OFF_BAR = OFF_ST + NSTS * STATS;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = 1024 + OFF_BAR + BAR_BYTES;
-  static constexpr int THREADS = 320;
+  static constexpr int SMEM = OFF_BAR + BAR_BYTES;  // the dynamic base is 1024-byte aligned
+  static constexpr int THREADS = 352;
   // TMEM columns: S_T^T / S_S^T per buffer, dK_S, dQ^T per buffer.
   static constexpr int TM_S = 0;          // buffer b: [128b, 128b+64) S_T, [+64, +128) S_S
   static constexpr int TM_DK = 256;       // d_S columns
@@ -76,7 +78,7 @@ struct BwdCfg {
 
 struct BwdBars {
   uint64_t k_full;
-  uint64_t q_full[3], q_empty[3], st_full[3];
+  uint64_t q_full[4], q_empty[4], st_full[2], st_empty[2];
   uint64_t s_full[2], s_free[2];
   uint64_t ds_full[2], ds_empty[2];
   uint64_t dq_full[2], dq_free[2];
@@ -92,7 +94,7 @@ __device__ __forceinline__ void skl_fail_b(volatile int* abort_flag) {
 }
 
 template <int DT, int DS>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
 streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                     const __grid_constant__ CUtensorMap map_kt,
                     const __grid_constant__ CUtensorMap map_qs,
@@ -100,10 +102,13 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                     const uint32_t idesc_st, const uint32_t idesc_ss, const uint32_t idesc_dk,
                     const uint32_t idesc_dq) {
   using C = BwdCfg<DT, DS>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sb = smem_u32(smem);
+  if (sb & 1023u) {  // the swizzled tiles need 1024-byte alignment; never expected to fire
+    if (threadIdx.x == 0) atomicOr(&g_skl_error, 4u);
+    return;
+  }
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::OFF_BAR);
   float* stats = reinterpret_cast<float*>(smem + C::OFF_ST);
   volatile int* abort_flag = &bars->abort_flag;
@@ -127,7 +132,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     for (int i = 0; i < C::NQST; ++i) {
       mbar_init(smem_u32(&bars->q_full[i]), 1);
       mbar_init(smem_u32(&bars->q_empty[i]), 1);
+    }
+    for (int i = 0; i < C::NSTS; ++i) {
       mbar_init(smem_u32(&bars->st_full[i]), 32);
+      mbar_init(smem_u32(&bars->st_empty[i]), 4);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&bars->s_full[b]), 1);
@@ -152,11 +160,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 8) {
-    // --------------------------------------- TMA producer + row-statistics loader
-    const uint64_t keep = l2_policy_evict_last();
-    int issued = 0;
-    bool ok = true;
+    // ----------------------------------------------------------- TMA producer
     if (lane == 0) {
+      const uint64_t keep = l2_policy_evict_last();
+      int issued = 0;
       tma_prefetch_desc(&map_qt);
       tma_prefetch_desc(&map_kt);
       tma_prefetch_desc(&map_qs);
@@ -167,58 +174,82 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         tma_load_3d(sb + C::OFF_KT + blk * (C::BN * 128), &map_kt, kb, blk * 64, k0, bh, keep);
       for (int blk = 0; blk < DS / 64; ++blk)
         tma_load_3d(sb + C::OFF_KS + blk * (C::BN * 128), &map_ks, kb, blk * 64, k0, bh, keep);
-    }
-    const float LOG2E = 1.4426950408889634f;
-    for (int s = 0; s < n_steps; ++s) {
-      const int st = s % C::NQST;
-      const int i0 = (jq_begin + s) * C::BM;
-      // Lane 0 does the waits and issues the copies; the verdict is shared so the warp
-      // leaves the loop together (the shuffle also orders the slot reuse below).
-      if (lane == 0) {
+      for (int s = 0; s < n_steps; ++s) {
+        const int st = s % C::NQST;
+        const int i0 = (jq_begin + s) * C::BM;
         if (!mbar_wait(smem_u32(&bars->q_empty[st]), ((s / C::NQST) & 1) ^ 1)) {
-          ok = false;
           skl_fail_b(abort_flag);
-        } else {
-          const uint32_t fb = smem_u32(&bars->q_full[st]);
-          const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
-          mbar_arrive_expect_tx(fb, C::Q_STAGE);
-          for (int blk = 0; blk < DT / 64; ++blk)
-            tma_load_3d(q_base + blk * (C::BM * 128), &map_qt, fb, blk * 64, i0, bh, keep);
-          for (int blk = 0; blk < DS / 64; ++blk)
-            tma_load_3d(q_base + C::QT_TILE + blk * (C::BM * 128), &map_qs, fb, blk * 64, i0, bh,
-                        keep);
-          issued = s + 1;
+          break;
         }
+        const uint32_t fb = smem_u32(&bars->q_full[st]);
+        const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
+        mbar_arrive_expect_tx(fb, C::Q_STAGE);
+        for (int blk = 0; blk < DT / 64; ++blk)
+          tma_load_3d(q_base + blk * (C::BM * 128), &map_qt, fb, blk * 64, i0, bh, keep);
+        for (int blk = 0; blk < DS / 64; ++blk)
+          tma_load_3d(q_base + C::QT_TILE + blk * (C::BM * 128), &map_qs, fb, blk * 64, i0, bh,
+                      keep);
+        issued = s + 1;
+      }
+      if (*abort_flag) {
+        // Let every copy this thread started land before the CTA can exit.
+        mbar_wait(smem_u32(&bars->k_full), 0);
+        for (int s = max(0, issued - C::NQST); s < issued; ++s)
+          mbar_wait(smem_u32(&bars->q_full[s % C::NQST]), (s / C::NQST) & 1);
+      }
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------ row-statistics loader
+    // Each lane owns query rows lane and lane+32 of every step. Raw LSE_T, LSE_S and g
+    // are loaded kStatAhead steps before they are needed and kept in registers.
+    constexpr int kStatAhead = 3;
+    const float LOG2E = 1.4426950408889634f;
+    float r_lt[kStatAhead][2], r_ls[kStatAhead][2], r_g[kStatAhead][2];
+    auto load_step = [&](int s, float (&lt)[2], float (&ls)[2], float (&gg)[2]) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = (jq_begin + s) * C::BM + r * 32 + lane;
+        lt[r] = -INFINITY;
+        ls[r] = -INFINITY;
+        gg[r] = 0.f;
+        if (s < n_steps && row < args.N_Q) {
+          const size_t o = (size_t)bh * args.N_Q + row;
+          lt[r] = __ldg(args.lse_t + o);
+          ls[r] = __ldg(args.lse_s + o);
+          gg[r] = __ldg(args.g + o);
+        }
+      }
+    };
+#pragma unroll
+    for (int k = 0; k < kStatAhead; ++k) load_step(k, r_lt[k], r_ls[k], r_g[k]);
+    bool ok = true;
+    for (int s = 0; s < n_steps; ++s) {
+      if (lane == 0 && !mbar_wait(smem_u32(&bars->st_empty[s & 1]), ((s >> 1) & 1) ^ 1)) {
+        ok = false;
+        skl_fail_b(abort_flag);
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      float* sts = stats + st * (3 * C::BM);
+      // Slot s&1: -LSE_T*log2e, -LSE_S*log2e, g*scale_S (rows without keys: -inf, -inf, 0).
+      float* sts = stats + (s & 1) * (3 * C::BM);
 #pragma unroll
-      for (int r = 0; r < C::BM / 32; ++r) {
-        const int qi = r * 32 + lane;
-        const int row = i0 + qi;
-        float nlt = -INFINITY, nls = -INFINITY, gs = 0.f;
-        if (row < args.N_Q) {
-          const size_t o = (size_t)bh * args.N_Q + row;
-          const float lt = args.lse_t[o];
-          const float ls = args.lse_s[o];
-          if (lt != -INFINITY && ls != -INFINITY) {
-            nlt = -lt * LOG2E;
-            nls = -ls * LOG2E;
-            gs = args.g[o] * args.scale_S;
-          }
-        }
-        sts[qi] = nlt;
-        sts[C::BM + qi] = nls;
-        sts[2 * C::BM + qi] = gs;
+      for (int r = 0; r < 2; ++r) {
+        const float lt = r_lt[0][r], ls = r_ls[0][r];
+        const bool live = lt != -INFINITY && ls != -INFINITY;
+        sts[r * 32 + lane] = live ? -lt * LOG2E : -INFINITY;
+        sts[C::BM + r * 32 + lane] = live ? -ls * LOG2E : -INFINITY;
+        sts[2 * C::BM + r * 32 + lane] = live ? r_g[0][r] * args.scale_S : 0.f;
       }
-      mbar_arrive(smem_u32(&bars->st_full[st]));
-    }
-    if (lane == 0 && *abort_flag) {
-      // Let every copy this thread started land before the CTA can exit.
-      mbar_wait(smem_u32(&bars->k_full), 0);
-      for (int s = max(0, issued - C::NQST); s < issued; ++s)
-        mbar_wait(smem_u32(&bars->q_full[s % C::NQST]), (s / C::NQST) & 1);
+      mbar_arrive(smem_u32(&bars->st_full[s & 1]));
+#pragma unroll
+      for (int k = 0; k + 1 < kStatAhead; ++k)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          r_lt[k][r] = r_lt[k + 1][r];
+          r_ls[k][r] = r_ls[k + 1][r];
+          r_g[k][r] = r_g[k + 1][r];
+        }
+      load_step(s + kStatAhead, r_lt[kStatAhead - 1], r_ls[kStatAhead - 1], r_g[kStatAhead - 1]);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
@@ -254,6 +285,15 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       if (ok && n_steps > 1) ok = issue_scores(1);
       for (int p = 0; ok && p < n_steps; ++p) {
         const int pb = p & 1, pst = p % C::NQST;
+        // The score tiles of step p+2 reuse buffer pb, which the warpgroup frees as soon as
+        // it has read step p's scores; issue them ahead of dK/dQ(p) when their query tile
+        // has landed, so the warpgroup finds them ready when it finishes step p.
+        bool early = false;
+        if (p + 2 < n_steps && mbar_try_wait(smem_u32(&bars->q_full[(p + 2) % C::NQST]),
+                                             ((p + 2) / C::NQST) & 1)) {
+          if (!issue_scores(p + 2)) { ok = false; break; }
+          early = true;
+        }
         if (!mbar_wait(smem_u32(&bars->ds_full[pb]), (p >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s_ds = sb + C::OFF_DS + pb * C::DS_TILE;
@@ -277,7 +317,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         }
         umma_commit(smem_u32(&bars->ds_empty[pb]));
         umma_commit(smem_u32(&bars->dq_full[pb]));
-        if (p + 2 < n_steps && !issue_scores(p + 2)) { ok = false; break; }
+        if (!early && p + 2 < n_steps && !issue_scores(p + 2)) { ok = false; break; }
       }
       if (!ok) skl_fail_b(abort_flag);
       umma_commit(smem_u32(&bars->dk_full));
@@ -325,54 +365,50 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       const int i0 = (jq_begin + s) * C::BM;  // first query column of this step
       if (!mbar_wait(smem_u32(&bars->s_full[wg]), (s >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      if (!mbar_wait(smem_u32(&bars->st_full[st]), (s / C::NQST) & 1)) { ok = false; break; }
-      const float* sts = stats + st * (3 * C::BM);
+      uint32_t vt[64], vs[64];  // raw teacher / student scores of this key, 64 query columns
+      tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + wg * 128,
+                        tmem + lane_off + C::TM_S + wg * 128 + 32, vt);
+      tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + wg * 128 + 64,
+                        tmem + lane_off + C::TM_S + wg * 128 + 96, vs);
+      // The score buffer can take step s+2 as soon as every lane has read it.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[wg]));
+      if (!mbar_wait(smem_u32(&bars->st_full[s & 1]), (s >> 1) & 1)) { ok = false; break; }
+      const float* sts = stats + (s & 1) * (3 * C::BM);
+      // The dS buffer is free once the dK/dQ MMAs of step s-2 have read it (they were
+      // issued before this step's scores, so this wait normally returns at once).
+      if (!mbar_wait(smem_u32(&bars->ds_empty[wg]), ((s >> 1) & 1) ^ 1)) { ok = false; break; }
 
       // Query column c is allowed for this key iff i0 + c >= key - off.
       const bool need_mask = args.causal && (i0 + args.off < k0 + C::BN - 1);
       const int cmin = need_mask ? (key - args.off - i0) : -1;
-      uint32_t packed[32];  // dS^T row of this key, 64 bf16 values
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {  // 32 query columns of S_T and S_S per pass
-        uint32_t v[64];             // v[0..31] teacher scores, v[32..63] student scores
-        tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + wg * 128 + 32 * h,
-                          tmem + lane_off + C::TM_S + wg * 128 + 64 + 32 * h, v);
+      for (int u = 0; u < 8; ++u) {  // 8 query columns = one 16-byte chunk of dS^T
+        const float4 nlt0 = *reinterpret_cast<const float4*>(sts + u * 8);
+        const float4 nlt1 = *reinterpret_cast<const float4*>(sts + u * 8 + 4);
+        const float4 nls0 = *reinterpret_cast<const float4*>(sts + C::BM + u * 8);
+        const float4 nls1 = *reinterpret_cast<const float4*>(sts + C::BM + u * 8 + 4);
+        const float4 g0 = *reinterpret_cast<const float4*>(sts + 2 * C::BM + u * 8);
+        const float4 g1 = *reinterpret_cast<const float4*>(sts + 2 * C::BM + u * 8 + 4);
+        const float nlt[8] = {nlt0.x, nlt0.y, nlt0.z, nlt0.w, nlt1.x, nlt1.y, nlt1.z, nlt1.w};
+        const float nls[8] = {nls0.x, nls0.y, nls0.z, nls0.w, nls1.x, nls1.y, nls1.z, nls1.w};
+        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        float d[8];
 #pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {  // 8 query columns = one 16-byte chunk
-          const int u = 4 * h + u4;
-          const float4 nlt0 = *reinterpret_cast<const float4*>(sts + u * 8);
-          const float4 nlt1 = *reinterpret_cast<const float4*>(sts + u * 8 + 4);
-          const float4 nls0 = *reinterpret_cast<const float4*>(sts + C::BM + u * 8);
-          const float4 nls1 = *reinterpret_cast<const float4*>(sts + C::BM + u * 8 + 4);
-          const float4 g0 = *reinterpret_cast<const float4*>(sts + 2 * C::BM + u * 8);
-          const float4 g1 = *reinterpret_cast<const float4*>(sts + 2 * C::BM + u * 8 + 4);
-          const float nlt[8] = {nlt0.x, nlt0.y, nlt0.z, nlt0.w, nlt1.x, nlt1.y, nlt1.z, nlt1.w};
-          const float nls[8] = {nls0.x, nls0.y, nls0.z, nls0.w, nls1.x, nls1.y, nls1.z, nls1.w};
-          const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-          float d[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int c = u * 8 + e;
-            const float pT = ex2_approx(fmaf(__uint_as_float(v[u4 * 8 + e]), cT, nlt[e]));
-            const float pS = ex2_approx(fmaf(__uint_as_float(v[32 + u4 * 8 + e]), cS, nls[e]));
-            float ds = gg[e] * (pS - pT);
-            if (need_mask && c < cmin) ds = 0.f;
-            d[e] = ds;
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) packed[u * 4 + e] = pack_bf16x2(d[2 * e], d[2 * e + 1]);
+        for (int e = 0; e < 8; ++e) {
+          const int c = u * 8 + e;
+          const float pT = ex2_approx(fmaf(__uint_as_float(vt[c]), cT, nlt[e]));
+          const float pS = ex2_approx(fmaf(__uint_as_float(vs[c]), cS, nls[e]));
+          float ds = gg[e] * (pS - pT);
+          if (need_mask && c < cmin) ds = 0.f;
+          d[e] = ds;
         }
+        st_shared_v4(s_ds_row + ((u ^ (kl & 7)) << 4), pack_bf16x2(d[0], d[1]),
+                     pack_bf16x2(d[2], d[3]), pack_bf16x2(d[4], d[5]), pack_bf16x2(d[6], d[7]));
       }
-      // The score buffer can take step s+2 once every lane has read it.
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[wg]));
-      // The dS buffer is free once the dK/dQ MMAs of step s-2 have read it.
-      if (!mbar_wait(smem_u32(&bars->ds_empty[wg]), ((s >> 1) & 1) ^ 1)) { ok = false; break; }
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        st_shared_v4(s_ds_row + ((u ^ (kl & 7)) << 4), packed[4 * u], packed[4 * u + 1],
-                     packed[4 * u + 2], packed[4 * u + 3]);
+      if (lane == 0) mbar_arrive(smem_u32(&bars->st_empty[s & 1]));
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->ds_full[wg]));
