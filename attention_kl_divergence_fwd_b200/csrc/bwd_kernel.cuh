@@ -16,14 +16,16 @@
 //      and stores it as bf16 into shared-memory buffer s&1;
 //   3. tensor core: dK_S += dS^T Q_S (TMEM accumulator over all steps) and
 //      dQ^T_part = K_S^T dS^T into TMEM buffer s&1 (d_S on the lanes, queries on columns);
-//   4. the same warpgroup adds dQ^T_part into dq_s: one fp32 reduction per lane, 32
-//      consecutive d values (one 128-byte line) per warp instruction.
+//   4. the same warpgroup copies dQ^T_part from TMEM into a shared-memory staging tile
+//      laid out as dq_s rows, and one thread adds the tile into dq_s with a bulk tensor
+//      reduce-add (the fp32 adds happen in L2).
 // Score tiles, dS tiles and dQ parts are double-buffered, so the two warpgroups work on
 // alternate steps while the tensor core computes the next ones.
 //
-// Warp roles (352 threads): warps 0-3 even steps, warps 4-7 odd steps, warp 8 TMA
+// Warp roles (384 threads): warps 0-3 even steps, warps 4-7 odd steps, warp 8 TMA
 // producer, warp 9 TMEM allocator + MMA issuer, warp 10 row-statistics loader (global
-// loads issued several steps ahead so their latency never reaches the pipeline).
+// loads issued several steps ahead so their latency never reaches the pipeline), warp 11
+// issues the dQ reduce-adds.
 #pragma once
 
 #include "ptx.cuh"
@@ -49,7 +51,7 @@ template <int DT, int DS>
 struct BwdCfg {
   static constexpr int BN = 128;  // keys per CTA (TMEM lanes)
   static constexpr int BM = 64;   // queries per step
-  static constexpr int NQST = 4;  // query-tile stages
+  static constexpr int NQST = 3;  // query-tile stages
   static constexpr int NSTS = 2;  // row-statistics slots
   static constexpr int KT_TILE = BN * DT * 2;
   static constexpr int KS_TILE = BN * DS * 2;
@@ -62,11 +64,13 @@ struct BwdCfg {
   static constexpr int OFF_KS = OFF_KT + KT_TILE;
   static constexpr int OFF_Q = OFF_KS + KS_TILE;           // NQST stages {Q_T, Q_S}
   static constexpr int OFF_DS = OFF_Q + NQST * Q_STAGE;    // two dS tiles
-  static constexpr int OFF_ST = OFF_DS + 2 * DS_TILE;      // NSTS statistics slots
+  static constexpr int STG_TILE = BM * DS * 4;             // fp32 dQ staging tile
+  static constexpr int OFF_STG = OFF_DS + 2 * DS_TILE;
+  static constexpr int OFF_ST = OFF_STG + STG_TILE;        // NSTS statistics slots
   static constexpr int OFF_BAR = OFF_ST + NSTS * STATS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES;  // the dynamic base is 1024-byte aligned
-  static constexpr int THREADS = 352;
+  static constexpr int THREADS = 384;
   // TMEM columns: S_T^T / S_S^T per buffer, dK_S, dQ^T per buffer.
   static constexpr int TM_S = 0;          // buffer b: [128b, 128b+64) S_T, [+64, +128) S_S
   static constexpr int TM_DK = 256;       // d_S columns
@@ -78,7 +82,8 @@ struct BwdCfg {
 
 struct BwdBars {
   uint64_t k_full;
-  uint64_t q_full[4], q_empty[4], st_full[2], st_empty[2];
+  uint64_t q_full[3], q_empty[3], st_full[2], st_empty[2];
+  uint64_t stg_full[2], stg_free[2];  // indexed by step parity
   uint64_t s_full[2], s_free[2];
   uint64_t ds_full[2], ds_empty[2];
   uint64_t dq_full[2], dq_free[2];
@@ -94,11 +99,12 @@ __device__ __forceinline__ void skl_fail_b(volatile int* abort_flag) {
 }
 
 template <int DT, int DS>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
 streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                     const __grid_constant__ CUtensorMap map_kt,
                     const __grid_constant__ CUtensorMap map_qs,
-                    const __grid_constant__ CUtensorMap map_ks, const BwdArgs args,
+                    const __grid_constant__ CUtensorMap map_ks,
+                    const __grid_constant__ CUtensorMap map_dq, const BwdArgs args,
                     const uint32_t idesc_st, const uint32_t idesc_ss, const uint32_t idesc_dk,
                     const uint32_t idesc_dq) {
   using C = BwdCfg<DT, DS>;
@@ -144,6 +150,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       mbar_init(smem_u32(&bars->ds_empty[b]), 1);
       mbar_init(smem_u32(&bars->dq_full[b]), 1);
       mbar_init(smem_u32(&bars->dq_free[b]), 4);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bars->stg_full[b]), 4);
+      mbar_init(smem_u32(&bars->stg_free[b]), 1);
     }
     mbar_init(smem_u32(&bars->dk_full), 1);
     mbar_init(smem_u32(&bars->drain), 1);
@@ -251,6 +261,25 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         }
       load_step(s + kStatAhead, r_lt[kStatAhead - 1], r_ls[kStatAhead - 1], r_g[kStatAhead - 1]);
     }
+  } else if (warp == 11) {
+    // ------------------------------------------------------- dQ reduce issuer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_dq);
+      for (int p = 0; p < n_steps; ++p) {
+        if (!mbar_wait(smem_u32(&bars->stg_full[p & 1]), (p >> 1) & 1)) {
+          skl_fail_b(abort_flag);
+          break;
+        }
+        const int i0 = (jq_begin + p) * C::BM;
+#pragma unroll
+        for (int db = 0; db < DS / 32; ++db)
+          tma_reduce_add_3d(&map_dq, sb + C::OFF_STG + db * (C::BM * 128), db * 32, i0, bh);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        mbar_arrive(smem_u32(&bars->stg_free[p & 1]));
+      }
+      bulk_wait_group0();
+    }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (elect_one()) {
@@ -338,6 +367,8 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     const bool dq_lane_ok = (C::DQ_M == 128) || lane < 16;
     const int dq_d = (C::DQ_M == 128) ? kl : quarter * 16 + lane;
 
+    // dQ^T part of step p (TMEM) -> staging tile (dq_s row layout: 32-column boxes of
+    // 64 rows x 128 bytes, 128-byte swizzle) -> one bulk reduce-add by warp 11.
     auto drain_dq = [&](int p) -> bool {
       if (!mbar_wait(smem_u32(&bars->dq_full[wg]), (p >> 1) & 1)) return false;
       tc_fence_after();
@@ -347,14 +378,21 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->dq_free[wg]));
+      // The staging tile is free once the reduce of step p-1 has read it. Barriers are
+      // split by step parity so this wait is never more than one phase ahead: the
+      // previous wait of this warpgroup (step p-2) already covered step p-3.
+      if (p > 0 && !mbar_wait(smem_u32(&bars->stg_free[(p - 1) & 1]), ((p - 1) >> 1) & 1))
+        return false;
       if (dq_lane_ok) {
-        const int i0 = (jq_begin + p) * C::BM;
-        const int nrows = min(C::BM, args.N_Q - i0);
-        float* dst = args.dq_s + ((size_t)bh * args.N_Q + i0) * DS + dq_d;
+        const uint32_t col = sb + C::OFF_STG + (dq_d >> 5) * (C::BM * 128) + ((dq_d & 3) << 2);
+        const uint32_t chunk = (dq_d & 31) >> 2;
 #pragma unroll
         for (int c = 0; c < C::BM; ++c)
-          if (c < nrows) red_add_f32(dst + (size_t)c * DS, __uint_as_float(v[c]));
+          st_shared_f32(col + c * 128 + ((chunk ^ (c & 7)) << 4), __uint_as_float(v[c]));
       }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->stg_full[p & 1]));
       return true;
     };
 

@@ -51,6 +51,20 @@ bool make_map(CUtensorMap* m, const void* base, int d, int n, int bh, int box_ro
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over the fp32 [BH, N_Q, d] dQ accumulator: box of 32 columns x 64 rows x 1.
+bool make_map_f32(CUtensorMap* m, void* base, int d, int n, int bh) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)bh};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)n * d * 4};
+  const cuuint32_t box[3] = {32, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 streamkl_status check_common(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
@@ -102,7 +116,7 @@ streamkl_status launch_bwd(const CUtensorMap* maps, const skl::BwdArgs& a, bool 
   const uint32_t i_dq = skl::idesc_bf16_f32(DS, C::BM, true, true);  // K_S^T dS^T
   const long long grid = (long long)a.n_ktiles * a.BH;
   kern<<<dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream>>>(
-      maps[0], maps[1], maps[2], maps[3], a, i_st, i_ss, i_dk, i_dq);
+      maps[0], maps[1], maps[2], maps[3], maps[4], a, i_st, i_ss, i_dk, i_dq);
   return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
 }
 
@@ -153,9 +167,10 @@ streamkl_status streamkl_bwd(const void* q_t, const void* k_t, const void* q_s, 
       !aligned16(dk_s))
     return STREAMKL_ERR_MISALIGNED;
   const int bh = B * H;
-  CUtensorMap maps[4];
+  CUtensorMap maps[5];
   if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 64) || !make_map(&maps[1], k_t, d_T, N_K, bh, 128) ||
-      !make_map(&maps[2], q_s, d_S, N_Q, bh, 64) || !make_map(&maps[3], k_s, d_S, N_K, bh, 128))
+      !make_map(&maps[2], q_s, d_S, N_Q, bh, 64) || !make_map(&maps[3], k_s, d_S, N_K, bh, 128) ||
+      !make_map_f32(&maps[4], dq_s, d_S, N_Q, bh))
     return STREAMKL_ERR_LAUNCH;
   if (cudaMemsetAsync(dq_s, 0, (size_t)bh * N_Q * d_S * sizeof(float), stream) != cudaSuccess)
     return STREAMKL_ERR_LAUNCH;
