@@ -5,18 +5,18 @@
 // two-distribution KL reduction, streaming query-key tiles through on-chip memory).
 //
 // CTA = two 128-row query tiles of one (batch, head). Key tiles of 64 rows stream
-// through a TMA ring. Per key tile and query tile the tensor core computes the
-// teacher and student score tiles into TMEM (double-buffered per query tile), and
-// one warpgroup per query tile (one thread per query row) folds them into the
-// online state
+// through a TMA ring. Per key tile and query tile the tensor core computes the teacher
+// and student score tiles into TMEM (two buffers per query tile). Each query tile has
+// two warpgroups, one thread per query row, taking the even and the odd key tiles; each
+// folds its tiles into its own online state
 //     m_T, m_S   running maxima of t = s * log2(e)
 //     l_T, l_S   running sums of 2^(t - m)
 //     A          running sum of 2^(t_T - m_T) * (t_T - t_S)
-// so that KL = ln2 * A / l_T - LSE_T + LSE_S at the end. Nothing of size N_Q x N_K
-// ever leaves the SM.
+// and the two states of a row are merged at the end (the state is associative), so
+// KL = ln2 * A / l_T - LSE_T + LSE_S. Nothing of size N_Q x N_K ever leaves the SM.
 //
-// Warp roles (320 threads): warps 0-3 query tile 0, warps 4-7 query tile 1,
-// warp 8 TMA producer, warp 9 TMEM allocator + MMA issuer.
+// Warp roles (576 threads): warps 0-15 statistics (warpgroup w: query tile w>>1, key
+// tiles of parity w&1), warp 16 TMA producer, warp 17 TMEM allocator + MMA issuer.
 #pragma once
 
 #include "ptx.cuh"
@@ -47,10 +47,10 @@ struct FwdCfg {
   static constexpr int QBYTES = NQ * (QT_TILE + QS_TILE);
   static constexpr int SMEM_MAX = 232448;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int NST_FIT = (SMEM_MAX - 1024 - BAR_BYTES - QBYTES) / STAGE;
+  static constexpr int NST_FIT = (SMEM_MAX - BAR_BYTES - QBYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
-  static constexpr int SMEM = 1024 + QBYTES + NST * STAGE + BAR_BYTES;
-  static constexpr int THREADS = 320;
+  static constexpr int SMEM = QBYTES + NST * STAGE + BAR_BYTES;  // base is 1024-aligned
+  static constexpr int THREADS = 576;
   static_assert(NST >= 2, "key ring needs two stages");
   static_assert(SMEM <= SMEM_MAX, "shared memory budget");
 };
@@ -71,18 +71,93 @@ __device__ __forceinline__ void skl_fail(volatile int* abort_flag) {
   *abort_flag = 1;
 }
 
+// Online state of one query row over the keys one warpgroup has seen (base-2 units).
+struct RowState {
+  float mT, mS, lT, lS, A;
+};
+
+// Folds 32 keys (v[0..31] teacher scores, v[32..63] student scores, raw dot products)
+// into the row state. Columns c > lim are masked. Every fourth exponential (c % 4 == 3)
+// runs on the FMA pipe (exp2_fma) so the MUFU is not the only unit doing them.
+template <bool MASK>
+__device__ __forceinline__ void fold_chunk(RowState& st, const uint32_t (&v)[64], float cT,
+                                           float cS, int lim) {
+  float mxT, mxS;
+  {
+    float a[32], b[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      a[c] = (!MASK || c <= lim) ? __uint_as_float(v[c]) : -INFINITY;
+      b[c] = (!MASK || c <= lim) ? __uint_as_float(v[32 + c]) : -INFINITY;
+    }
+    mxT = max_tree32(a);
+    mxS = max_tree32(b);
+  }
+  const float mT_new = fmaxf(st.mT, cT * mxT);  // NaN (cT=0, all masked) keeps the old max
+  const float mS_new = fmaxf(st.mS, cS * mxS);
+  const float mT_use = (mT_new == -INFINITY) ? 0.f : mT_new;
+  const float mS_use = (mS_new == -INFINITY) ? 0.f : mS_new;
+  // Rescale the running sums only when some row of the warp raised its maximum.
+  if (__any_sync(0xffffffffu, (mT_new > st.mT) || (mS_new > st.mS))) {
+    const float aT = ex2_approx(st.mT - mT_use);  // -inf - x -> 0
+    const float aS = ex2_approx(st.mS - mS_use);
+    st.lT *= aT;
+    st.A *= aT;
+    st.lS *= aS;
+  }
+  float sT0 = 0.f, sT1 = 0.f, sS0 = 0.f, sS1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    const float xT0 = fmaf(__uint_as_float(v[c]), cT, -mT_use);
+    const float xT1 = fmaf(__uint_as_float(v[c + 1]), cT, -mT_use);
+    const float xS0 = fmaf(__uint_as_float(v[32 + c]), cS, -mS_use);
+    const float xS1 = fmaf(__uint_as_float(v[32 + c + 1]), cS, -mS_use);
+    float eT0 = ex2_approx(xT0);
+    float eS0 = ex2_approx(xS0);
+    float eT1, eS1;
+    if ((c & 3) == 2) {
+      eT1 = exp2_fma(xT1);
+      eS1 = exp2_fma(xS1);
+    } else {
+      eT1 = ex2_approx(xT1);
+      eS1 = ex2_approx(xS1);
+    }
+    if (MASK) {
+      eT0 = c <= lim ? eT0 : 0.f;
+      eS0 = c <= lim ? eS0 : 0.f;
+      eT1 = c + 1 <= lim ? eT1 : 0.f;
+      eS1 = c + 1 <= lim ? eS1 : 0.f;
+    }
+    sT0 += eT0;
+    sT1 += eT1;
+    sS0 += eS0;
+    sS1 += eS1;
+    b0 = fmaf(eT0, xT0 - xS0, b0);
+    b1 = fmaf(eT1, xT1 - xS1, b1);
+  }
+  const float sumT = sT0 + sT1;
+  st.lT += sumT;
+  st.lS += sS0 + sS1;
+  st.A += (b0 + b1) + (mT_use - mS_use) * sumT;
+  st.mT = mT_new;
+  st.mS = mS_new;
+}
+
 template <int DT, int DS>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(576, 1)
 streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                     const __grid_constant__ CUtensorMap map_kt,
                     const __grid_constant__ CUtensorMap map_qs,
                     const __grid_constant__ CUtensorMap map_ks,
                     const FwdArgs args, const uint32_t idesc_t, const uint32_t idesc_s) {
   using C = FwdCfg<DT, DS>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t s_base = smem_u32(smem);
+  if (s_base & 1023u) {  // the swizzled tiles need 1024-byte alignment; never expected to fire
+    if (threadIdx.x == 0) atomicOr(&g_skl_error, 4u);
+    return;
+  }
   const uint32_t s_qt = s_base;                               // [NQ][DT/64][128][64]
   const uint32_t s_qs = s_base + C::NQ * C::QT_TILE;          // [NQ][DS/64][128][64]
   const uint32_t s_k = s_base + C::QBYTES;                    // [NST]{K_T, K_S}
@@ -131,7 +206,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 17) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
   }
@@ -140,7 +215,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
       tma_prefetch_desc(&map_qt);
@@ -183,7 +258,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           mbar_wait(smem_u32(&bars->full[j % C::NST]), (j / C::NST) & 1);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ------------------------------------------------------------- MMA issuer
     if (elect_one()) {
       bool ok = mbar_wait(smem_u32(&bars->q_full), 0);
@@ -235,32 +310,26 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     }
   } else {
     // --------------------------------------------------- statistics warpgroups
-    const int q = warp >> 2;          // query tile of this warpgroup
+    const int wg = warp >> 2;
+    const int q = wg >> 1;            // query tile
+    const int par = wg & 1;           // key tiles j with j & 1 == par (TMEM buffer par)
     const int quarter = warp & 3;     // TMEM lane quarter of this warp
-    const int row = q0 + q * C::BM + quarter * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int rloc = quarter * 32 + lane;
+    const int row = q0 + q * C::BM + rloc;
+    const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + q * 256 + par * 128;
     const float cT = args.cT, cS = args.cS;
     const int first_row = q0 + q * C::BM;
+    const int nkq = nk[q];
 
-    float mT = -INFINITY, mS = -INFINITY, lT = 0.f, lS = 0.f, A = 0.f;
+    RowState st{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
     bool ok = true;
-    for (int j = 0; j < nk[q]; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(smem_u32(&bars->s_full[q][b]), (j >> 1) & 1)) {
+    for (int j = par; j < nkq; j += 2) {
+      if (!mbar_wait(smem_u32(&bars->s_full[q][par]), (j >> 1) & 1)) {
         skl_fail(abort_flag);
         ok = false;
         break;
       }
       tc_fence_after();
-      // Raw teacher / student scores of keys 64j..64j+63 for this thread's row.
-      const uint32_t ta = tmem + lane_off + q * 256 + b * 128;
-      uint32_t vt_u[64], vs_u[64];
-      tmem_ld_2x32_wait(ta, ta + 32, vt_u);
-      tmem_ld_2x32_wait(ta + 64, ta + 96, vs_u);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[q][b]));
-
       const int k0 = j * C::BN;
       const bool need_mask =
           (k0 + C::BN > args.N_K) || (args.causal && k0 + C::BN - 1 > first_row + args.off);
@@ -270,68 +339,50 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         if (args.causal) last = min(last, row + args.off);
         lim = last - k0;
       }
-
-      float mxT = -INFINITY, mxS = -INFINITY;
-      if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < C::BN; ++c) {
-          const bool ok_c = c <= lim;
-          mxT = fmaxf(mxT, ok_c ? __uint_as_float(vt_u[c]) : -INFINITY);
-          mxS = fmaxf(mxS, ok_c ? __uint_as_float(vs_u[c]) : -INFINITY);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[64];  // keys 64j+32h .. +31: v[0..31] teacher, v[32..63] student
+        tmem_ld_2x32_wait(ta + 32 * h, ta + 64 + 32 * h, v);
+        if (h == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[q][par]));
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < C::BN; ++c) {
-          mxT = fmaxf(mxT, __uint_as_float(vt_u[c]));
-          mxS = fmaxf(mxS, __uint_as_float(vs_u[c]));
-        }
+        if (need_mask)
+          fold_chunk<true>(st, v, cT, cS, lim - 32 * h);
+        else
+          fold_chunk<false>(st, v, cT, cS, 0);
       }
-      const float mT_new = fmaxf(mT, cT * mxT);
-      const float mS_new = fmaxf(mS, cS * mxS);
-      const float mT_use = (mT_new == -INFINITY) ? 0.f : mT_new;
-      const float mS_use = (mS_new == -INFINITY) ? 0.f : mS_new;
-      const float aT = ex2_approx(mT - mT_use);
-      const float aS = ex2_approx(mS - mS_use);
-
-      float sT0 = 0.f, sT1 = 0.f, sS0 = 0.f, sS1 = 0.f, b0 = 0.f, b1 = 0.f;
-      if (need_mask) {
-#pragma unroll
-        for (int c = 0; c < C::BN; c += 2) {
-          const float xT0 = fmaf(__uint_as_float(vt_u[c]), cT, -mT_use);
-          const float xT1 = fmaf(__uint_as_float(vt_u[c + 1]), cT, -mT_use);
-          const float xS0 = fmaf(__uint_as_float(vs_u[c]), cS, -mS_use);
-          const float xS1 = fmaf(__uint_as_float(vs_u[c + 1]), cS, -mS_use);
-          const float eT0 = c <= lim ? ex2_approx(xT0) : 0.f;
-          const float eT1 = c + 1 <= lim ? ex2_approx(xT1) : 0.f;
-          const float eS0 = c <= lim ? ex2_approx(xS0) : 0.f;
-          const float eS1 = c + 1 <= lim ? ex2_approx(xS1) : 0.f;
-          sT0 += eT0; sT1 += eT1; sS0 += eS0; sS1 += eS1;
-          b0 = fmaf(eT0, xT0 - xS0, b0);
-          b1 = fmaf(eT1, xT1 - xS1, b1);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < C::BN; c += 2) {
-          const float xT0 = fmaf(__uint_as_float(vt_u[c]), cT, -mT_use);
-          const float xT1 = fmaf(__uint_as_float(vt_u[c + 1]), cT, -mT_use);
-          const float xS0 = fmaf(__uint_as_float(vs_u[c]), cS, -mS_use);
-          const float xS1 = fmaf(__uint_as_float(vs_u[c + 1]), cS, -mS_use);
-          const float eT0 = ex2_approx(xT0), eT1 = ex2_approx(xT1);
-          const float eS0 = ex2_approx(xS0), eS1 = ex2_approx(xS1);
-          sT0 += eT0; sT1 += eT1; sS0 += eS0; sS1 += eS1;
-          b0 = fmaf(eT0, xT0 - xS0, b0);
-          b1 = fmaf(eT1, xT1 - xS1, b1);
-        }
-      }
-      const float sumT = sT0 + sT1;
-      lT = fmaf(aT, lT, sumT);
-      lS = fmaf(aS, lS, sS0 + sS1);
-      A = fmaf(aT, A, (b0 + b1) + (mT_use - mS_use) * sumT);
-      mT = mT_new;
-      mS = mS_new;
     }
 
-    if (ok && row < args.N_Q) {
+    // Merge the odd-tile state into the even-tile warpgroup. The merge area is this
+    // query tile's Q_T buffer, free once every MMA of the tile has completed.
+    float* merge = reinterpret_cast<float*>(smem + q * C::QT_TILE);
+    bool ready = ok && mbar_wait(smem_u32(&bars->q_full), 0);
+    if (ready && nkq > 0) {
+      const int jl = nkq - 1;
+      ready = mbar_wait(smem_u32(&bars->s_full[q][jl & 1]), (jl >> 1) & 1);
+    }
+    if (!ready && ok) skl_fail(abort_flag);
+    fence_async_smem();
+    if (par == 1 && ready) {
+      merge[0 * C::BM + rloc] = st.mT;
+      merge[1 * C::BM + rloc] = st.mS;
+      merge[2 * C::BM + rloc] = st.lT;
+      merge[3 * C::BM + rloc] = st.lS;
+      merge[4 * C::BM + rloc] = st.A;
+    }
+    named_bar_sync(1 + q, 256);
+    if (par == 0 && ready && row < args.N_Q) {
+      const float mT1 = merge[0 * C::BM + rloc], mS1 = merge[1 * C::BM + rloc];
+      const float mT = fmaxf(st.mT, mT1), mS = fmaxf(st.mS, mS1);
+      const float mT_use = (mT == -INFINITY) ? 0.f : mT;
+      const float mS_use = (mS == -INFINITY) ? 0.f : mS;
+      const float a0T = ex2_approx(st.mT - mT_use), a1T = ex2_approx(mT1 - mT_use);
+      const float a0S = ex2_approx(st.mS - mS_use), a1S = ex2_approx(mS1 - mS_use);
+      const float lT = a0T * st.lT + a1T * merge[2 * C::BM + rloc];
+      const float lS = a0S * st.lS + a1S * merge[3 * C::BM + rloc];
+      const float A = a0T * st.A + a1T * merge[4 * C::BM + rloc];
       const float LN2 = 0.69314718055994530942f;
       float kl, lse_t, lse_s;
       if (lT > 0.f) {
@@ -354,7 +405,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -227,6 +227,44 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Maximum of 32 values as a shallow tree of three-input max instructions.
+__device__ __forceinline__ float max_tree32(const float (&a)[32]) {
+  float l1[12];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) l1[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  l1[10] = a[30];
+  l1[11] = a[31];
+  const float l2a = fmax3(l1[0], l1[1], l1[2]), l2b = fmax3(l1[3], l1[4], l1[5]);
+  const float l2c = fmax3(l1[6], l1[7], l1[8]), l2d = fmax3(l1[9], l1[10], l1[11]);
+  return fmaxf(fmax3(l2a, l2b, l2c), l2d);
+}
+
+// 2^x on the FMA pipe, for x <= 0 (inputs below -125 give 2^-125; callers only add the
+// result to sums that are at least 1). Method: Cody-Waite style range reduction
+// x = n + f, n = round-to-nearest(x) taken with the 1.5*2^23 shifter, f in [-1/2, 1/2];
+// 2^f from a degree-5 polynomial fitted by this project (minimax relative error on
+// [-1/2, 1/2] by linear programming, see fit_exp2_poly.py): max relative error 1.9e-7
+// in fp32 Horner form; n is added straight into the exponent field.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.0f);
+  const float kShift = 12582912.0f;
+  const float y = __fadd_rn(x, kShift);
+  const float f = __fsub_rn(x, __fsub_rn(y, kShift));
+  float p = 0.001325405784882605f;
+  p = fmaf(p, f, 0.00967527274042368f);
+  p = fmaf(p, f, 0.055507827550172806f);
+  p = fmaf(p, f, 0.2402212917804718f);
+  p = fmaf(p, f, 0.6931469440460205f);
+  p = fmaf(p, f, 1.0000001192092896f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
