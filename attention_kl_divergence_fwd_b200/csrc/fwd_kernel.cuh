@@ -6,17 +6,20 @@
 //
 // CTA = two 128-row query tiles of one (batch, head). Key tiles of 64 rows stream
 // through a TMA ring. Per key tile and query tile the tensor core computes the teacher
-// and student score tiles into TMEM (two buffers per query tile). Each query tile has
-// two warpgroups, one thread per query row, taking the even and the odd key tiles; each
-// folds its tiles into its own online state
+// and student score tiles into TMEM (two buffers per query tile, so the next tile is
+// computed while the current one is folded). One warpgroup per query tile, one thread
+// per query row, folds each tile into the row's online state
 //     m_T, m_S   running maxima of t = s * log2(e)
 //     l_T, l_S   running sums of 2^(t - m)
 //     A          running sum of 2^(t_T - m_T) * (t_T - t_S)
-// and the two states of a row are merged at the end (the state is associative), so
-// KL = ln2 * A / l_T - LSE_T + LSE_S. Nothing of size N_Q x N_K ever leaves the SM.
+// so that KL = ln2 * A / l_T - LSE_T + LSE_S at the end. Per tile: one pass over TMEM
+// for the row maxima, a second pass (two 32-key halves) for the exponentials, with the
+// fp32 work issued as packed pairs and a share of the exponentials on the FMA pipe.
+// Nothing of size N_Q x N_K ever leaves the SM.
 //
-// Warp roles (576 threads): warps 0-15 statistics (warpgroup w: query tile w>>1, key
-// tiles of parity w&1), warp 16 TMA producer, warp 17 TMEM allocator + MMA issuer.
+// Warp roles (384 threads): warps 0-3 query tile 0, warps 4-7 query tile 1 (224 registers
+// each), warp 8 TMA producer, warp 9 TMEM allocator + MMA issuer, warps 10-11 idle (the
+// control warpgroup runs with 56 registers).
 #pragma once
 
 #include "ptx.cuh"
@@ -50,7 +53,7 @@ struct FwdCfg {
   static constexpr int NST_FIT = (SMEM_MAX - BAR_BYTES - QBYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
   static constexpr int SMEM = QBYTES + NST * STAGE + BAR_BYTES;  // base is 1024-aligned
-  static constexpr int THREADS = 576;
+  static constexpr int THREADS = 384;
   static_assert(NST >= 2, "key ring needs two stages");
   static_assert(SMEM <= SMEM_MAX, "shared memory budget");
 };
@@ -76,28 +79,22 @@ struct RowState {
   float mT, mS, lT, lS, A;
 };
 
-// Folds 32 keys (v[0..31] teacher scores, v[32..63] student scores, raw dot products)
-// into the row state. Columns c > lim are masked. Every fourth exponential (c % 4 == 3)
-// runs on the FMA pipe (exp2_fma) so the MUFU is not the only unit doing them.
-template <bool MASK>
-__device__ __forceinline__ void fold_chunk(RowState& st, const uint32_t (&v)[64], float cT,
-                                           float cS, int lim) {
-  float mxT, mxS;
-  {
-    float a[32], b[32];
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      a[c] = (!MASK || c <= lim) ? __uint_as_float(v[c]) : -INFINITY;
-      b[c] = (!MASK || c <= lim) ? __uint_as_float(v[32 + c]) : -INFINITY;
-    }
-    mxT = max_tree32(a);
-    mxS = max_tree32(b);
-  }
+// Which column pairs (c, c+1) of a 32-key chunk send their second exponential of both
+// distributions to the FMA pipe: pairs 1, 3, 5, 7 of every 8 (25 % of the exponentials),
+// plus pair 6 when kPolyHeavy (37.5 %).
+constexpr bool kPolyHeavy = true;
+__host__ __device__ constexpr bool poly_pair(int pair) {
+  return (pair & 1) || (kPolyHeavy && (pair & 7) == 6);
+}
+
+// New running maxima from a tile's raw maxima; rescales the sums when any row of the
+// warp raised its maximum. Returns the reference maxima (0 while still -inf).
+__device__ __forceinline__ void update_max(RowState& st, float mxT, float mxS, float cT, float cS,
+                                           float& mT_use, float& mS_use) {
   const float mT_new = fmaxf(st.mT, cT * mxT);  // NaN (cT=0, all masked) keeps the old max
   const float mS_new = fmaxf(st.mS, cS * mxS);
-  const float mT_use = (mT_new == -INFINITY) ? 0.f : mT_new;
-  const float mS_use = (mS_new == -INFINITY) ? 0.f : mS_new;
-  // Rescale the running sums only when some row of the warp raised its maximum.
+  mT_use = (mT_new == -INFINITY) ? 0.f : mT_new;
+  mS_use = (mS_new == -INFINITY) ? 0.f : mS_new;
   if (__any_sync(0xffffffffu, (mT_new > st.mT) || (mS_new > st.mS))) {
     const float aT = ex2_approx(st.mT - mT_use);  // -inf - x -> 0
     const float aS = ex2_approx(st.mS - mS_use);
@@ -105,46 +102,90 @@ __device__ __forceinline__ void fold_chunk(RowState& st, const uint32_t (&v)[64]
     st.A *= aT;
     st.lS *= aS;
   }
-  float sT0 = 0.f, sT1 = 0.f, sS0 = 0.f, sS1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll
-  for (int c = 0; c < 32; c += 2) {
-    const float xT0 = fmaf(__uint_as_float(v[c]), cT, -mT_use);
-    const float xT1 = fmaf(__uint_as_float(v[c + 1]), cT, -mT_use);
-    const float xS0 = fmaf(__uint_as_float(v[32 + c]), cS, -mS_use);
-    const float xS1 = fmaf(__uint_as_float(v[32 + c + 1]), cS, -mS_use);
-    float eT0 = ex2_approx(xT0);
-    float eS0 = ex2_approx(xS0);
-    float eT1, eS1;
-    if ((c & 3) == 2) {
-      eT1 = exp2_fma(xT1);
-      eS1 = exp2_fma(xS1);
-    } else {
-      eT1 = ex2_approx(xT1);
-      eS1 = ex2_approx(xS1);
-    }
-    if (MASK) {
-      eT0 = c <= lim ? eT0 : 0.f;
-      eS0 = c <= lim ? eS0 : 0.f;
-      eT1 = c + 1 <= lim ? eT1 : 0.f;
-      eS1 = c + 1 <= lim ? eS1 : 0.f;
-    }
-    sT0 += eT0;
-    sT1 += eT1;
-    sS0 += eS0;
-    sS1 += eS1;
-    b0 = fmaf(eT0, xT0 - xS0, b0);
-    b1 = fmaf(eT1, xT1 - xS1, b1);
-  }
-  const float sumT = sT0 + sT1;
-  st.lT += sumT;
-  st.lS += sS0 + sS1;
-  st.A += (b0 + b1) + (mT_use - mS_use) * sumT;
   st.mT = mT_new;
   st.mS = mS_new;
 }
 
+// Accumulates 16 keys (v[0..15] teacher scores, v[16..31] student scores, raw dot
+// products) into the packed partial sums. Columns c > lim are masked (MASK).
+template <bool MASK>
+__device__ __forceinline__ void fold_part(const uint32_t (&v)[32], uint64_t cT2, uint64_t cS2,
+                                          uint64_t nmT2, uint64_t nmS2, int lim, int pair0,
+                                          uint64_t& sT2, uint64_t& sS2, uint64_t& b2) {
+#pragma unroll
+  for (int c = 0; c < 16; c += 2) {
+    const uint64_t xT = f2_fma(f2_pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), cT2, nmT2);
+    const uint64_t xS =
+        f2_fma(f2_pack(__uint_as_float(v[16 + c]), __uint_as_float(v[16 + c + 1])), cS2, nmS2);
+    float xT0, xT1, xS0, xS1;
+    f2_unpack(xT, xT0, xT1);
+    f2_unpack(xS, xS0, xS1);
+    float eT0 = ex2_approx(xT0), eS0 = ex2_approx(xS0), eT1, eS1;
+    if (poly_pair(pair0 + (c >> 1))) {
+      f2_unpack(exp2_fma2(f2_pack(xT1, xS1)), eT1, eS1);
+    } else {
+      eT1 = ex2_approx(xT1);
+      eS1 = ex2_approx(xS1);
+    }
+    uint64_t d = f2_sub(xT, xS);
+    if (MASK) {
+      const bool k0 = c <= lim, k1 = c + 1 <= lim;
+      eT0 = k0 ? eT0 : 0.f;
+      eS0 = k0 ? eS0 : 0.f;
+      eT1 = k1 ? eT1 : 0.f;
+      eS1 = k1 ? eS1 : 0.f;
+      float d0, d1;
+      f2_unpack(d, d0, d1);
+      d = f2_pack(k0 ? d0 : 0.f, k1 ? d1 : 0.f);
+    }
+    const uint64_t eT = f2_pack(eT0, eT1);
+    sT2 = f2_add(sT2, eT);
+    sS2 = f2_add(sS2, f2_pack(eS0, eS1));
+    b2 = f2_fma(eT, d, b2);
+  }
+}
+
+// Folds one 64-key tile (TMEM columns: ta .. ta+63 teacher, ta+64 .. ta+127 student)
+// into the row state; releases the TMEM buffer (s_free) once it has been read.
+template <bool MASK>
+__device__ __forceinline__ void fold_tile(RowState& st, uint32_t ta, float cT, float cS, int lim,
+                                          uint32_t s_free, int lane) {
+  float mxT, mxS;
+  {
+    uint32_t v[64];
+    tmem_ld_2x32_wait(ta, ta + 32, v);
+    mxT = fmaxf(max_tree32<MASK>(v, 0, lim), max_tree32<MASK>(v, 32, lim - 32));
+    tmem_ld_2x32_wait(ta + 64, ta + 96, v);
+    mxS = fmaxf(max_tree32<MASK>(v, 0, lim), max_tree32<MASK>(v, 32, lim - 32));
+  }
+  float mT_use, mS_use;
+  update_max(st, mxT, mxS, cT, cS, mT_use, mS_use);
+  const uint64_t cT2 = f2_pack(cT, cT), cS2 = f2_pack(cS, cS);
+  const uint64_t nmT2 = f2_pack(-mT_use, -mT_use), nmS2 = f2_pack(-mS_use, -mS_use);
+  uint64_t sT2 = f2_pack(0.f, 0.f), sS2 = sT2, b2 = sT2;
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    uint32_t v[32];  // keys 16h .. 16h+15: v[0..15] teacher, v[16..31] student
+    tmem_ld_2x16_wait(ta + 16 * h, ta + 64 + 16 * h, v);
+    if (h == 3) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+    }
+    fold_part<MASK>(v, cT2, cS2, nmT2, nmS2, lim - 16 * h, 8 * h, sT2, sS2, b2);
+  }
+  float s0, s1, u0, u1, w0, w1;
+  f2_unpack(sT2, s0, s1);
+  f2_unpack(sS2, u0, u1);
+  f2_unpack(b2, w0, w1);
+  const float sumT = s0 + s1;
+  st.lT += sumT;
+  st.lS += u0 + u1;
+  st.A += (w0 + w1) + (mT_use - mS_use) * sumT;
+}
+
 template <int DT, int DS>
-__global__ void __launch_bounds__(576, 1)
+__global__ void __launch_bounds__(384, 1)
 streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                     const __grid_constant__ CUtensorMap map_kt,
                     const __grid_constant__ CUtensorMap map_qs,
@@ -206,7 +247,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 17) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
   }
@@ -215,116 +256,21 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 16) {
-    // ------------------------------------------------------------ TMA producer
-    if (elect_one()) {
-      tma_prefetch_desc(&map_qt);
-      tma_prefetch_desc(&map_kt);
-      tma_prefetch_desc(&map_qs);
-      tma_prefetch_desc(&map_ks);
-      const uint64_t keep = l2_policy_evict_last();
-      const uint64_t once = l2_policy_evict_first();
-      const uint32_t qb = smem_u32(&bars->q_full);
-      mbar_arrive_expect_tx(qb, C::QBYTES);
-      for (int q = 0; q < C::NQ; ++q) {
-        for (int blk = 0; blk < DT / 64; ++blk)
-          tma_load_3d(s_qt + q * C::QT_TILE + blk * (C::BM * 128), &map_qt, qb, blk * 64,
-                      q0 + q * C::BM, bh, once);
-        for (int blk = 0; blk < DS / 64; ++blk)
-          tma_load_3d(s_qs + q * C::QS_TILE + blk * (C::BM * 128), &map_qs, qb, blk * 64,
-                      q0 + q * C::BM, bh, once);
-      }
-      int issued = 0;
-      for (int j = 0; j < nk_max; ++j) {
-        const int s = j % C::NST;
-        if (!mbar_wait(smem_u32(&bars->empty[s]), ((j / C::NST) & 1) ^ 1)) {
-          skl_fail(abort_flag);
-          break;
-        }
-        const uint32_t fb = smem_u32(&bars->full[s]);
-        mbar_arrive_expect_tx(fb, C::STAGE);
-        const uint32_t st = s_k + s * C::STAGE;
-        for (int blk = 0; blk < DT / 64; ++blk)
-          tma_load_3d(st + blk * (C::BN * 128), &map_kt, fb, blk * 64, j * C::BN, bh, keep);
-        for (int blk = 0; blk < DS / 64; ++blk)
-          tma_load_3d(st + C::KT_TILE + blk * (C::BN * 128), &map_ks, fb, blk * 64, j * C::BN,
-                      bh, keep);
-        issued = j + 1;
-      }
-      if (*abort_flag) {
-        // Let every copy this thread started land before the CTA can exit.
-        mbar_wait(qb, 0);
-        for (int j = max(0, issued - C::NST); j < issued; ++j)
-          mbar_wait(smem_u32(&bars->full[j % C::NST]), (j / C::NST) & 1);
-      }
-    }
-  } else if (warp == 17) {
-    // ------------------------------------------------------------- MMA issuer
-    if (elect_one()) {
-      bool ok = mbar_wait(smem_u32(&bars->q_full), 0);
-      if (!ok) skl_fail(abort_flag);
-      for (int j = 0; ok && j < nk_max; ++j) {
-        const int s = j % C::NST;
-        if (!mbar_wait(smem_u32(&bars->full[s]), (j / C::NST) & 1)) {
-          skl_fail(abort_flag);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t st = s_k + s * C::STAGE;
-#pragma unroll
-        for (int q = 0; q < C::NQ; ++q) {
-          if (j >= nk[q]) continue;
-          const int b = j & 1;
-          if (!mbar_wait(smem_u32(&bars->s_free[q][b]), ((j >> 1) & 1) ^ 1)) {
-            skl_fail(abort_flag);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d_t = tmem + q * 256 + b * 128;
-          const uint32_t d_s = d_t + 64;
-#pragma unroll
-          for (int kk = 0; kk < DT / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;
-            const uint64_t a = sdesc_sw128(s_qt + q * C::QT_TILE + (kk >> 2) * (C::BM * 128) + off,
-                                           16, 1024);
-            const uint64_t bd = sdesc_sw128(st + (kk >> 2) * (C::BN * 128) + off, 16, 1024);
-            umma_bf16_ss(d_t, a, bd, idesc_t, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < DS / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;
-            const uint64_t a = sdesc_sw128(s_qs + q * C::QS_TILE + (kk >> 2) * (C::BM * 128) + off,
-                                           16, 1024);
-            const uint64_t bd =
-                sdesc_sw128(st + C::KT_TILE + (kk >> 2) * (C::BN * 128) + off, 16, 1024);
-            umma_bf16_ss(d_s, a, bd, idesc_s, kk > 0);
-          }
-          umma_commit(smem_u32(&bars->s_full[q][b]));
-        }
-        umma_commit(smem_u32(&bars->empty[s]));
-      }
-      // Every MMA this thread issued must be complete before TMEM is released.
-      umma_commit(smem_u32(&bars->drain));
-      if (!mbar_wait(smem_u32(&bars->drain), 0)) skl_fail(abort_flag);
-    }
-  } else {
+  if (warp < 8) {
+    regs_inc<200>();
     // --------------------------------------------------- statistics warpgroups
-    const int wg = warp >> 2;
-    const int q = wg >> 1;            // query tile
-    const int par = wg & 1;           // key tiles j with j & 1 == par (TMEM buffer par)
+    const int q = warp >> 2;          // query tile of this warpgroup
     const int quarter = warp & 3;     // TMEM lane quarter of this warp
-    const int rloc = quarter * 32 + lane;
-    const int row = q0 + q * C::BM + rloc;
-    const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + q * 256 + par * 128;
+    const int row = q0 + q * C::BM + quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float cT = args.cT, cS = args.cS;
     const int first_row = q0 + q * C::BM;
-    const int nkq = nk[q];
 
     RowState st{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
     bool ok = true;
-    for (int j = par; j < nkq; j += 2) {
-      if (!mbar_wait(smem_u32(&bars->s_full[q][par]), (j >> 1) & 1)) {
+    for (int j = 0; j < nk[q]; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(smem_u32(&bars->s_full[q][b]), (j >> 1) & 1)) {
         skl_fail(abort_flag);
         ok = false;
         break;
@@ -333,64 +279,26 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       const int k0 = j * C::BN;
       const bool need_mask =
           (k0 + C::BN > args.N_K) || (args.causal && k0 + C::BN - 1 > first_row + args.off);
-      int lim = C::BN - 1;  // last allowed column of this tile for this row
+      const uint32_t ta = tmem + lane_off + q * 256 + b * 128;
+      const uint32_t fr = smem_u32(&bars->s_free[q][b]);
       if (need_mask) {
         int last = args.N_K - 1;
         if (args.causal) last = min(last, row + args.off);
-        lim = last - k0;
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t v[64];  // keys 64j+32h .. +31: v[0..31] teacher, v[32..63] student
-        tmem_ld_2x32_wait(ta + 32 * h, ta + 64 + 32 * h, v);
-        if (h == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[q][par]));
-        }
-        if (need_mask)
-          fold_chunk<true>(st, v, cT, cS, lim - 32 * h);
-        else
-          fold_chunk<false>(st, v, cT, cS, 0);
+        fold_tile<true>(st, ta, cT, cS, last - k0, fr, lane);
+      } else {
+        fold_tile<false>(st, ta, cT, cS, C::BN - 1, fr, lane);
       }
     }
 
-    // Merge the odd-tile state into the even-tile warpgroup. The merge area is this
-    // query tile's Q_T buffer, free once every MMA of the tile has completed.
-    float* merge = reinterpret_cast<float*>(smem + q * C::QT_TILE);
-    bool ready = ok && mbar_wait(smem_u32(&bars->q_full), 0);
-    if (ready && nkq > 0) {
-      const int jl = nkq - 1;
-      ready = mbar_wait(smem_u32(&bars->s_full[q][jl & 1]), (jl >> 1) & 1);
-    }
-    if (!ready && ok) skl_fail(abort_flag);
-    fence_async_smem();
-    if (par == 1 && ready) {
-      merge[0 * C::BM + rloc] = st.mT;
-      merge[1 * C::BM + rloc] = st.mS;
-      merge[2 * C::BM + rloc] = st.lT;
-      merge[3 * C::BM + rloc] = st.lS;
-      merge[4 * C::BM + rloc] = st.A;
-    }
-    named_bar_sync(1 + q, 256);
-    if (par == 0 && ready && row < args.N_Q) {
-      const float mT1 = merge[0 * C::BM + rloc], mS1 = merge[1 * C::BM + rloc];
-      const float mT = fmaxf(st.mT, mT1), mS = fmaxf(st.mS, mS1);
-      const float mT_use = (mT == -INFINITY) ? 0.f : mT;
-      const float mS_use = (mS == -INFINITY) ? 0.f : mS;
-      const float a0T = ex2_approx(st.mT - mT_use), a1T = ex2_approx(mT1 - mT_use);
-      const float a0S = ex2_approx(st.mS - mS_use), a1S = ex2_approx(mS1 - mS_use);
-      const float lT = a0T * st.lT + a1T * merge[2 * C::BM + rloc];
-      const float lS = a0S * st.lS + a1S * merge[3 * C::BM + rloc];
-      const float A = a0T * st.A + a1T * merge[4 * C::BM + rloc];
+    if (ok && row < args.N_Q) {
       const float LN2 = 0.69314718055994530942f;
       float kl, lse_t, lse_s;
-      if (lT > 0.f) {
-        const float l2T = log2f(lT), l2S = log2f(lS);
-        lse_t = LN2 * (mT + l2T);
-        lse_s = LN2 * (mS + l2S);
+      if (st.lT > 0.f) {
+        const float l2T = log2f(st.lT), l2S = log2f(st.lS);
+        lse_t = LN2 * (st.mT + l2T);
+        lse_s = LN2 * (st.mS + l2S);
         // Grouped so that identical teacher and student statistics give exactly 0.
-        kl = LN2 * ((A / lT) + ((mS - mT) + (l2S - l2T)));
+        kl = LN2 * ((st.A / st.lT) + ((st.mS - st.mT) + (l2S - l2T)));
       } else {
         kl = 0.f;
         lse_t = -INFINITY;
@@ -401,11 +309,107 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       args.lse_t[o] = lse_t;
       args.lse_s[o] = lse_s;
     }
+  } else {
+    regs_dec<104>();
+    if (warp == 8) {
+      // ------------------------------------------------------------ TMA producer
+      if (elect_one()) {
+        tma_prefetch_desc(&map_qt);
+        tma_prefetch_desc(&map_kt);
+        tma_prefetch_desc(&map_qs);
+        tma_prefetch_desc(&map_ks);
+        const uint64_t keep = l2_policy_evict_last();
+        const uint64_t once = l2_policy_evict_first();
+        const uint32_t qb = smem_u32(&bars->q_full);
+        mbar_arrive_expect_tx(qb, C::QBYTES);
+        for (int q = 0; q < C::NQ; ++q) {
+          for (int blk = 0; blk < DT / 64; ++blk)
+            tma_load_3d(s_qt + q * C::QT_TILE + blk * (C::BM * 128), &map_qt, qb, blk * 64,
+                        q0 + q * C::BM, bh, once);
+          for (int blk = 0; blk < DS / 64; ++blk)
+            tma_load_3d(s_qs + q * C::QS_TILE + blk * (C::BM * 128), &map_qs, qb, blk * 64,
+                        q0 + q * C::BM, bh, once);
+        }
+        int issued = 0;
+        for (int j = 0; j < nk_max; ++j) {
+          const int s = j % C::NST;
+          if (!mbar_wait(smem_u32(&bars->empty[s]), ((j / C::NST) & 1) ^ 1)) {
+            skl_fail(abort_flag);
+            break;
+          }
+          const uint32_t fb = smem_u32(&bars->full[s]);
+          mbar_arrive_expect_tx(fb, C::STAGE);
+          const uint32_t st = s_k + s * C::STAGE;
+          for (int blk = 0; blk < DT / 64; ++blk)
+            tma_load_3d(st + blk * (C::BN * 128), &map_kt, fb, blk * 64, j * C::BN, bh, keep);
+          for (int blk = 0; blk < DS / 64; ++blk)
+            tma_load_3d(st + C::KT_TILE + blk * (C::BN * 128), &map_ks, fb, blk * 64, j * C::BN,
+                        bh, keep);
+          issued = j + 1;
+        }
+        if (*abort_flag) {
+          // Let every copy this thread started land before the CTA can exit.
+          mbar_wait(qb, 0);
+          for (int j = max(0, issued - C::NST); j < issued; ++j)
+            mbar_wait(smem_u32(&bars->full[j % C::NST]), (j / C::NST) & 1);
+        }
+      }
+    } else if (warp == 9) {
+      // ------------------------------------------------------------- MMA issuer
+      if (elect_one()) {
+        bool ok = mbar_wait(smem_u32(&bars->q_full), 0);
+        if (!ok) skl_fail(abort_flag);
+        for (int j = 0; ok && j < nk_max; ++j) {
+          const int s = j % C::NST;
+          if (!mbar_wait(smem_u32(&bars->full[s]), (j / C::NST) & 1)) {
+            skl_fail(abort_flag);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = s_k + s * C::STAGE;
+  #pragma unroll
+          for (int q = 0; q < C::NQ; ++q) {
+            if (j >= nk[q]) continue;
+            const int b = j & 1;
+            if (!mbar_wait(smem_u32(&bars->s_free[q][b]), ((j >> 1) & 1) ^ 1)) {
+              skl_fail(abort_flag);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d_t = tmem + q * 256 + b * 128;
+            const uint32_t d_s = d_t + 64;
+  #pragma unroll
+            for (int kk = 0; kk < DT / 16; ++kk) {
+              const uint32_t off = (kk & 3) * 32;
+              const uint64_t a = sdesc_sw128(s_qt + q * C::QT_TILE + (kk >> 2) * (C::BM * 128) + off,
+                                             16, 1024);
+              const uint64_t bd = sdesc_sw128(st + (kk >> 2) * (C::BN * 128) + off, 16, 1024);
+              umma_bf16_ss(d_t, a, bd, idesc_t, kk > 0);
+            }
+  #pragma unroll
+            for (int kk = 0; kk < DS / 16; ++kk) {
+              const uint32_t off = (kk & 3) * 32;
+              const uint64_t a = sdesc_sw128(s_qs + q * C::QS_TILE + (kk >> 2) * (C::BM * 128) + off,
+                                             16, 1024);
+              const uint64_t bd =
+                  sdesc_sw128(st + C::KT_TILE + (kk >> 2) * (C::BN * 128) + off, 16, 1024);
+              umma_bf16_ss(d_s, a, bd, idesc_s, kk > 0);
+            }
+            umma_commit(smem_u32(&bars->s_full[q][b]));
+          }
+          umma_commit(smem_u32(&bars->empty[s]));
+        }
+        // Every MMA this thread issued must be complete before TMEM is released.
+        umma_commit(smem_u32(&bars->drain));
+        if (!mbar_wait(smem_u32(&bars->drain), 0)) skl_fail(abort_flag);
+      }
+    }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 17) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

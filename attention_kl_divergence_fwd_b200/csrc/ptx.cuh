@@ -206,6 +206,29 @@ __device__ __forceinline__ void tmem_ld_2x32_wait(uint32_t ta, uint32_t tb, uint
       : "memory");
 }
 
+// Two 16-column loads (lanes = this warp's quarter) followed by the wait.
+__device__ __forceinline__ void tmem_ld_2x16_wait(uint32_t ta, uint32_t tb, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : SKL_R8(0), SKL_R8(8), SKL_R8(16), SKL_R8(24)
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_16_wait(uint32_t ta, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : SKL_R8(0), SKL_R8(8)
+      : "r"(ta)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_32_wait(uint32_t ta, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -233,13 +256,18 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// Maximum of 32 values as a shallow tree of three-input max instructions.
-__device__ __forceinline__ float max_tree32(const float (&a)[32]) {
+// Maximum of v[base..base+31] (as floats) as a shallow tree of three-input max
+// instructions; with MASK, entries past `lim` count as -inf.
+template <bool MASK, int N>
+__device__ __forceinline__ float max_tree32(const uint32_t (&v)[N], int base, int lim) {
+  auto at = [&](int c) -> float {
+    return (!MASK || c <= lim) ? __uint_as_float(v[base + c]) : -INFINITY;
+  };
   float l1[12];
 #pragma unroll
-  for (int i = 0; i < 10; ++i) l1[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
-  l1[10] = a[30];
-  l1[11] = a[31];
+  for (int i = 0; i < 10; ++i) l1[i] = fmax3(at(3 * i), at(3 * i + 1), at(3 * i + 2));
+  l1[10] = at(30);
+  l1[11] = at(31);
   const float l2a = fmax3(l1[0], l1[1], l1[2]), l2b = fmax3(l1[3], l1[4], l1[5]);
   const float l2c = fmax3(l1[6], l1[7], l1[8]), l2d = fmax3(l1[9], l1[10], l1[11]);
   return fmaxf(fmax3(l2a, l2b, l2c), l2d);
@@ -263,6 +291,82 @@ __device__ __forceinline__ float exp2_fma(float x) {
   p = fmaf(p, f, 0.6931469440460205f);
   p = fmaf(p, f, 1.0000001192092896f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
+}
+
+// ---- packed fp32 pairs (one instruction for two lanes of work on sm_100)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// exp2_fma on a packed pair: same steps, the fp32 arithmetic issued as f32x2.
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t kShift = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t y = f2_add(x, kShift);
+  const uint64_t f = f2_sub(x, f2_sub(y, kShift));
+  uint64_t p = f2_pack(0.001325405784882605f, 0.001325405784882605f);
+  p = f2_fma(p, f, f2_pack(0.00967527274042368f, 0.00967527274042368f));
+  p = f2_fma(p, f, f2_pack(0.055507827550172806f, 0.055507827550172806f));
+  p = f2_fma(p, f, f2_pack(0.2402212917804718f, 0.2402212917804718f));
+  p = f2_fma(p, f, f2_pack(0.6931469440460205f, 0.6931469440460205f));
+  p = f2_fma(p, f, f2_pack(1.0000001192092896f, 1.0000001192092896f));
+  float p0, p1, y0, y1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(y, y0, y1);
+  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(y0) << 23)),
+                 __int_as_float(__float_as_int(p1) + (__float_as_int(y1) << 23)));
+}
+
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Lower-accuracy pair variant for values that are rounded to bf16 afterwards: degree-3
+// polynomial from the same fit (fit_exp2_poly.py), max relative error 7.5e-5.
+__device__ __forceinline__ uint64_t exp2_fma2_d3(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t kShift = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t y = f2_add(x, kShift);
+  const uint64_t f = f2_sub(x, f2_sub(y, kShift));
+  uint64_t p = f2_pack(0.055171750485897064f, 0.055171750485897064f);
+  p = f2_fma(p, f, f2_pack(0.24261131882667542f, 0.24261131882667542f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, y0, y1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(y, y0, y1);
+  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(y0) << 23)),
+                 __int_as_float(__float_as_int(p1) + (__float_as_int(y1) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -315,6 +419,19 @@ __device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
 
 __device__ __forceinline__ void red_add_f32(float* gaddr, float a) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(gaddr), "f"(a) : "memory");
+}
+
+// Per-warpgroup register budget changes (every warp of the warpgroup executes them).
+// The kernels using them launch 12 warps at 168 registers and move registers from the
+// control warpgroup to the two compute warpgroups, keeping the total: 4*104 + 8*200 = 12*168.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
