@@ -1,0 +1,76 @@
+"""PyTorch autograd wrapper over the StreamKL C ABI, with the usual loss reductions.
+
+    loss = attention_kl_loss(q_t, k_t, q_s, k_s, causal=True, reduction="mean")
+    loss.backward()          # fills q_s.grad and k_s.grad (the teacher is frozen)
+
+The forward calls ``streamkl_fwd`` (per-row KL plus the two log-sum-exps it saves for
+backward); the backward calls ``streamkl_bwd`` with g = dLoss/dKL per row, which the
+reduction determines: 1 for "sum", 1/(B*H*N_Q) for "mean", 1/B for "batchmean". Only
+the O(B*H*N_Q) row vector is touched by PyTorch; every O(N_Q*N_K) step runs in the CUDA
+kernels and nothing of that size is ever allocated.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import streamkl_bwd, streamkl_fwd
+
+REDUCTIONS = ("none", "sum", "mean", "batchmean")
+
+
+class StreamKLFunction(torch.autograd.Function):
+    """Row-wise KL(P_T || P_S) of two attention maps; gradients flow to Q_S and K_S only."""
+
+    @staticmethod
+    def forward(ctx, q_t, k_t, q_s, k_s, scale_t: float, scale_s: float, causal: bool):
+        kl, lse_t, lse_s = streamkl_fwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal)
+        ctx.save_for_backward(q_t, k_t, q_s, k_s, lse_t, lse_s)
+        ctx.params = (scale_t, scale_s, causal)
+        ctx.mark_non_differentiable(lse_t, lse_s)
+        return kl, lse_t, lse_s
+
+    @staticmethod
+    def backward(ctx, g_kl, _g_lse_t=None, _g_lse_s=None):
+        q_t, k_t, q_s, k_s, lse_t, lse_s = ctx.saved_tensors
+        scale_t, scale_s, causal = ctx.params
+        g = g_kl.detach().to(torch.float32).contiguous()
+        dq, dk = streamkl_bwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, lse_t, lse_s, g)
+        return None, None, dq.to(q_s.dtype), dk.to(k_s.dtype), None, None, None
+
+
+def attention_kl(q_t, k_t, q_s, k_s, scale_t: Optional[float] = None,
+                 scale_s: Optional[float] = None, causal: bool = False):
+    """Per-row KL [B, H, N_Q] (fp32), differentiable w.r.t. q_s and k_s.
+
+    Default scales are 1/sqrt(d) of each side. Tensors: bf16 [B, H, N, d] on one GPU.
+    """
+    scale_t = 1.0 / math.sqrt(q_t.shape[-1]) if scale_t is None else float(scale_t)
+    scale_s = 1.0 / math.sqrt(q_s.shape[-1]) if scale_s is None else float(scale_s)
+    kl, _, _ = StreamKLFunction.apply(q_t.contiguous(), k_t.contiguous(), q_s.contiguous(),
+                                      k_s.contiguous(), scale_t, scale_s, bool(causal))
+    return kl
+
+
+def reduce_kl(kl: torch.Tensor, reduction: str = "mean") -> torch.Tensor:
+    """Reduce per-row KL [B, H, N_Q] to a loss; the reduction fixes g = dLoss/dKL."""
+    if reduction == "none":
+        return kl
+    if reduction == "sum":
+        return kl.sum()
+    if reduction == "mean":
+        return kl.mean()
+    if reduction == "batchmean":
+        return kl.sum() / kl.shape[0]
+    raise ValueError(f"reduction must be one of {REDUCTIONS}, got {reduction!r}")
+
+
+def attention_kl_loss(q_t, k_t, q_s, k_s, scale_t: Optional[float] = None,
+                      scale_s: Optional[float] = None, causal: bool = False,
+                      reduction: str = "mean") -> torch.Tensor:
+    """Attention-distillation loss: reduction of the row-wise KL(P_T || P_S)."""
+    if reduction not in REDUCTIONS:
+        raise ValueError(f"reduction must be one of {REDUCTIONS}, got {reduction!r}")
+    return reduce_kl(attention_kl(q_t, k_t, q_s, k_s, scale_t, scale_s, causal), reduction)

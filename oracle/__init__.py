@@ -2,6 +2,7 @@
 from .streamkl_oracle import (  # noqa: F401
     allowed,
     oracle_bwd,
+    oracle_bwd_teacher,
     oracle_dk_rows,
     oracle_fwd,
     oracle_row_work,

@@ -243,3 +243,36 @@ def row_pair_count(n_q: int, n_k: int, causal: bool, i: int) -> int:
     if not causal:
         return n_k
     return max(0, min(n_k, i + n_k - n_q + 1))
+
+
+def oracle_bwd_teacher(q_t, k_t, q_s, k_s, scale_t: float, scale_s: float, causal: bool, g,
+                       row_block: int = 1024):
+    """dQ_T [B,H,N_Q,d_T] and dK_T [B,H,N_K,d_T] (float64) of sum_i g[i] * KL[i].
+
+    For a trainable teacher. With the student fixed, KL_i = sum_j P_T (s_T - log P_S) - LSE_T,
+    so dKL_i/ds_T[i,j] = P_T[i,j] * ((s_T - s_S)[i,j] - E_i) with
+    E_i = sum_j P_T[i,j] (s_T - s_S)[i,j] (= KL_i + LSE_T,i - LSE_S,i), and
+    dS_T[i,j] = g[i] * scale_T * P_T[i,j] * ((s_T - s_S)[i,j] - E_i) on J(i), else 0;
+    dQ_T = dS_T K_T, dK_T = dS_T^T Q_T.
+    """
+    B, H, n_q, d_t = q_t.shape
+    n_k = k_t.shape[2]
+    dq = torch.zeros(B, H, n_q, d_t, dtype=F64)
+    dk = torch.zeros(B, H, n_k, d_t, dtype=F64)
+    for b in range(B):
+        for h in range(H):
+            kt, ks = _f64(k_t[b, h]), _f64(k_s[b, h])
+            for r0 in range(0, n_q, row_block):
+                rows = torch.arange(r0, min(n_q, r0 + row_block))
+                qt = _f64(q_t[b, h, rows])
+                st, ss, mask, lt, ls = _row_block_stats(
+                    qt, kt, _f64(q_s[b, h, rows]), ks, rows, scale_t, scale_s, causal, n_q)
+                p_t, _ = _probs(st, lt, mask)
+                diff = torch.where(mask, st - ss, torch.zeros_like(st))
+                e = (p_t * diff).sum(dim=1)
+                gi = _f64(g[b, h, rows])
+                ds = gi[:, None] * scale_t * p_t * (diff - e[:, None])
+                ds = torch.where(mask, ds, torch.zeros_like(ds))
+                dq[b, h, rows] = ds @ kt
+                dk[b, h] += ds.T @ qt
+    return dq, dk

@@ -1,0 +1,62 @@
+"""autograd wrapper and loss reductions: values and gradients vs the fp64 oracle."""
+import math
+
+import pytest
+import torch
+
+from attention_kl_divergence_fwd_b200 import autograd as ska
+from workloads import WORKLOADS, make_inputs
+
+
+def test_unknown_reduction_rejected_before_any_launch():
+    with pytest.raises(ValueError):
+        ska.attention_kl_loss(None, None, None, None, reduction="avg")
+
+
+def test_reduce_kl_defines_g():
+    kl = torch.arange(24, dtype=torch.float32).reshape(2, 3, 4).requires_grad_(True)
+    for red, g in [("sum", 1.0), ("mean", 1.0 / 24), ("batchmean", 0.5)]:
+        kl.grad = None
+        ska.reduce_kl(kl, red).backward()
+        assert torch.allclose(kl.grad, torch.full_like(kl, g))
+    assert ska.reduce_kl(kl, "none") is kl
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("reduction", ["mean", "sum", "batchmean"])
+def test_loss_and_grads_match_oracle(reduction):
+    from oracle import oracle_bwd, oracle_fwd
+    w = WORKLOADS["b2h16_n4096_d128_causal"].with_sizes(B=2, H=2, N_Q=300, N_K=300)
+    x = make_inputs(w, seed=17)
+    d = {k: v.cuda() for k, v in x.items()}
+    q_s = d["q_s"].clone().requires_grad_(True)
+    k_s = d["k_s"].clone().requires_grad_(True)
+    loss = ska.attention_kl_loss(d["q_t"], d["k_t"], q_s, k_s, w.scale_T, w.scale_S, True,
+                                 reduction)
+    loss.backward()
+    args = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S, True)
+    kl, _, _ = oracle_fwd(*args)
+    n = kl.numel()
+    g = {"sum": 1.0, "mean": 1.0 / n, "batchmean": 1.0 / w.B}[reduction]
+    ref_loss = kl.sum() * g
+    assert abs(loss.item() - ref_loss.item()) <= 1e-4 * max(1.0, abs(ref_loss.item()))
+    dq, dk = oracle_bwd(*args, torch.full_like(x["g"], g))
+    rel = lambda a, b: ((a.double().cpu() - b).norm() / b.norm()).item()
+    assert q_s.grad.dtype == torch.bfloat16 and k_s.grad.dtype == torch.bfloat16
+    assert rel(q_s.grad, dq) < 1.5e-2
+    assert rel(k_s.grad, dk) < 1.5e-2
+
+
+@pytest.mark.gpu
+def test_default_scales_and_no_teacher_grad():
+    w = WORKLOADS["tiny_n256_d64"]
+    x = make_inputs(w)
+    d = {k: v.cuda() for k, v in x.items()}
+    q_t = d["q_t"].clone().requires_grad_(True)
+    q_s = d["q_s"].clone().requires_grad_(True)
+    kl = ska.attention_kl(q_t, d["k_t"], q_s, d["k_s"])  # scales default to 1/sqrt(64)
+    kl.sum().backward()
+    assert q_t.grad is None
+    kl2 = ska.attention_kl(d["q_t"], d["k_t"], d["q_s"], d["k_s"], 1 / math.sqrt(64),
+                           1 / math.sqrt(64))
+    assert torch.equal(kl.detach(), kl2)

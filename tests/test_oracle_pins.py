@@ -87,25 +87,33 @@ def test_brute_force_tiny(nq, nk, causal):
 
 # --------------------------------------------------------- library routine
 
+MASKED = -1.0e4  # finite stand-in for -inf: exp underflows to exactly 0 in fp64, no NaN grads
+
+
+def _masked_scores(s, nq, nk, causal):
+    if not causal:
+        return s
+    bad = torch.arange(nk)[None, :] > torch.arange(nq)[:, None] + nk - nq
+    return torch.where(bad, torch.full_like(s, MASKED), s)
+
+
 def library_kl(q_t, k_t, q_s, k_s, st, ss, causal, g):
-    """torch log_softmax + kl_div (log_target) in fp64, autograd for the gradients."""
+    """torch log_softmax + kl_div (log_target) in fp64, autograd for the student gradients.
+
+    Masked scores use a large finite value so that every gradient entry is finite and
+    compared; rows with no allowed key become uniform over masked keys (P_T = P_S, so KL
+    and gradients are 0 there, matching the empty-row reading) and are excluded from
+    the LSE comparison by the caller.
+    """
     qs = q_s.double().requires_grad_(True)
     ks = k_s.double().requires_grad_(True)
     nq, nk = q_t.shape[2], k_t.shape[2]
-    s_t = st * q_t.double() @ k_t.double().transpose(-1, -2)
-    s_s = ss * qs @ ks.transpose(-1, -2)
-    if causal:
-        i = torch.arange(nq)[:, None]
-        j = torch.arange(nk)[None, :]
-        bad = j > i + nk - nq
-        s_t = s_t.masked_fill(bad, float("-inf"))
-        s_s = s_s.masked_fill(bad, float("-inf"))
+    s_t = _masked_scores(st * q_t.double() @ k_t.double().transpose(-1, -2), nq, nk, causal)
+    s_s = _masked_scores(ss * qs @ ks.transpose(-1, -2), nq, nk, causal)
     lp_t = torch.log_softmax(s_t, -1)
     lp_s = torch.log_softmax(s_s, -1)
     # kl_div(input=log q, target=log p, log_target=True) = p * (log p - log q)
-    terms = torch.nn.functional.kl_div(lp_s, lp_t, reduction="none", log_target=True)
-    terms = torch.nan_to_num(terms, nan=0.0)
-    kl = terms.sum(-1)
+    kl = torch.nn.functional.kl_div(lp_s, lp_t, reduction="none", log_target=True).sum(-1)
     (kl * g.double()).sum().backward()
     return kl.detach(), torch.logsumexp(s_t, -1).detach(), torch.logsumexp(s_s, -1).detach(), qs.grad, ks.grad
 
@@ -119,12 +127,13 @@ def test_against_library(causal, dims):
     kl_r, lt_r, ls_r, dq_r, dk_r = library_kl(q_t, k_t, q_s, k_s, st, ss, causal, g)
     kl, lt, ls = O.oracle_fwd(q_t, k_t, q_s, k_s, st, ss, causal, row_block=5)
     dq, dk = O.oracle_bwd(q_t, k_t, q_s, k_s, st, ss, causal, g, row_block=5)
-    ok = torch.isfinite(lt_r)
-    torch.testing.assert_close(kl[ok], kl_r[ok], rtol=1e-12, atol=1e-12)
+    ok = torch.isfinite(lt)  # rows with at least one allowed key
+    torch.testing.assert_close(kl, kl_r, rtol=1e-12, atol=1e-12)
     torch.testing.assert_close(lt[ok], lt_r[ok], rtol=1e-12, atol=1e-12)
     torch.testing.assert_close(ls[ok], ls_r[ok], rtol=1e-12, atol=1e-12)
-    torch.testing.assert_close(dq, torch.nan_to_num(dq_r), rtol=1e-10, atol=1e-12)
-    torch.testing.assert_close(dk, torch.nan_to_num(dk_r), rtol=1e-10, atol=1e-12)
+    assert torch.all(torch.isfinite(dq_r)) and torch.all(torch.isfinite(dk_r))
+    torch.testing.assert_close(dq, dq_r, rtol=1e-10, atol=1e-12)
+    torch.testing.assert_close(dk, dk_r, rtol=1e-10, atol=1e-12)
 
 
 # ------------------------------------------------------------- closed forms
@@ -335,3 +344,45 @@ def test_planted_mistakes_are_caught(monkeypatch):
             same = all(torch.allclose(a, b, rtol=1e-9, atol=1e-12, equal_nan=True)
                        for a, b in zip((kl, lt, ls, dq, dk), ref))
             assert not same, f"planted mistake in {name} was not caught"
+
+
+# ------------------------------------------------- trainable-teacher gradient
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_teacher_grad_against_library_autograd(causal):
+    """dQ_T, dK_T from torch log_softmax/kl_div autograd w.r.t. the teacher inputs."""
+    q_t, k_t, q_s, k_s, g = rand_case(1, 2, 9, 11, 8, 4, seed=31 + causal)
+    st, ss = 0.45, 0.6
+    qt = q_t.double().requires_grad_(True)
+    kt = k_t.double().requires_grad_(True)
+    s_t = _masked_scores(st * qt @ kt.transpose(-1, -2), 9, 11, causal)
+    s_s = _masked_scores(ss * q_s.double() @ k_s.double().transpose(-1, -2), 9, 11, causal)
+    terms = torch.nn.functional.kl_div(torch.log_softmax(s_s, -1), torch.log_softmax(s_t, -1),
+                                       reduction="none", log_target=True)
+    (terms.sum(-1) * g.double()).sum().backward()
+    assert torch.all(torch.isfinite(qt.grad)) and torch.all(torch.isfinite(kt.grad))
+    dq, dk = O.oracle_bwd_teacher(q_t, k_t, q_s, k_s, st, ss, causal, g, row_block=4)
+    torch.testing.assert_close(dq, qt.grad, rtol=1e-10, atol=1e-12)
+    torch.testing.assert_close(dk, kt.grad, rtol=1e-10, atol=1e-12)
+
+
+def test_teacher_grad_finite_differences_and_invariants():
+    q_t, k_t, q_s, k_s, g = rand_case(1, 1, 5, 6, 3, 3, seed=41, bf16=False)
+    q_t, k_t, q_s, k_s, g = (x.double() for x in (q_t, k_t, q_s, k_s, g))
+    st, ss = 0.8, 0.7
+    dq, dk = O.oracle_bwd_teacher(q_t, k_t, q_s, k_s, st, ss, True, g)
+    loss = lambda qt, kt: float((O.oracle_fwd(qt, kt, q_s, k_s, st, ss, True)[0] * g).sum())
+    h = 1e-6
+    for (i, c) in [(1, 0), (4, 2)]:
+        e = torch.zeros_like(q_t); e[0, 0, i, c] = h
+        fd = (loss(q_t + e, k_t) - loss(q_t - e, k_t)) / (2 * h)
+        assert abs(fd - dq[0, 0, i, c].item()) <= 1e-6 * max(1.0, abs(fd))
+    for (j, c) in [(0, 1), (5, 0)]:
+        e = torch.zeros_like(k_t); e[0, 0, j, c] = h
+        fd = (loss(q_t, k_t + e) - loss(q_t, k_t - e)) / (2 * h)
+        assert abs(fd - dk[0, 0, j, c].item()) <= 1e-6 * max(1.0, abs(fd))
+    # sum_j dS_T[i, j] = 0 for every row, so the teacher key gradients sum to zero
+    assert dk.sum(dim=2).abs().max() < 1e-12
+    # identical teacher and student: zero gradient for the teacher as well
+    dq0, dk0 = O.oracle_bwd_teacher(q_t, k_t, q_t, k_t, st, st, True, g)
+    assert dq0.abs().max() < 1e-15 and dk0.abs().max() < 1e-15
