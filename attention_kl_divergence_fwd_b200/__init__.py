@@ -6,6 +6,8 @@ is no CPU fallback: if the library is missing, importing the functions raises.
 
     kl, lse_t, lse_s = streamkl_fwd(q_t, k_t, q_s, k_s, scale_T, scale_S, causal)
     dq_s, dk_s = streamkl_bwd(q_t, k_t, q_s, k_s, scale_T, scale_S, causal, lse_t, lse_s, g)
+    dq_t, dk_t = streamkl_bwd_teacher(q_t, k_t, q_s, k_s, scale_T, scale_S, causal,
+                                      kl, lse_t, lse_s, g)      # trainable teacher only
 
 Tensors: bf16 [B, H, N, d] contiguous on one CUDA device (d in {64, 128}); row
 statistics and g fp32 [B, H, N_Q]; gradients fp32.
@@ -20,8 +22,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "lib", "libstreamkl.so")
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "MISALIGNED", 4: "LAUNCH", 5: "TIMEOUT"}
-EXPORTS = ("streamkl_fwd", "streamkl_bwd", "streamkl_status_string", "streamkl_device_status",
-           "streamkl_version")
+EXPORTS = ("streamkl_fwd", "streamkl_bwd", "streamkl_bwd_teacher", "streamkl_status_string",
+           "streamkl_device_status", "streamkl_version")
 
 
 class StreamKLError(RuntimeError):
@@ -47,6 +49,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.streamkl_fwd.restype = i
     lib.streamkl_bwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, f, i, vp, vp, vp, vp, vp, vp]
     lib.streamkl_bwd.restype = i
+    lib.streamkl_bwd_teacher.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, f, i, vp, vp, vp,
+                                         vp, vp, vp, vp]
+    lib.streamkl_bwd_teacher.restype = i
     lib.streamkl_status_string.argtypes = [i]
     lib.streamkl_status_string.restype = ctypes.c_char_p
     lib.streamkl_device_status.argtypes = [vp]
@@ -104,6 +109,16 @@ def streamkl_bwd_raw(q_t: int, k_t: int, q_s: int, k_s: int, B: int, H: int, N_Q
                                        lse_t, lse_s, g, dq_s, dk_s, stream)
 
 
+def streamkl_bwd_teacher_raw(q_t: int, k_t: int, q_s: int, k_s: int, B: int, H: int, N_Q: int,
+                             N_K: int, d_T: int, d_S: int, scale_T: float, scale_S: float,
+                             causal: bool, kl: int, lse_t: int, lse_s: int, g: int, dq_t: int,
+                             dk_t: int, stream: int = 0) -> int:
+    return load_library().streamkl_bwd_teacher(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S,
+                                               float(scale_T), float(scale_S),
+                                               int(bool(causal)), kl, lse_t, lse_s, g, dq_t,
+                                               dk_t, stream)
+
+
 def streamkl_fwd(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
                  kl=None, lse_t=None, lse_s=None, stream=None):
     """Per-row KL(P_T || P_S), LSE_T, LSE_S (fp32 [B,H,N_Q]) on the current stream."""
@@ -137,6 +152,26 @@ def streamkl_bwd(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: boo
                           dq_s.data_ptr(), dk_s.data_ptr(), _stream_ptr(stream))
     _check(st, "streamkl_bwd")
     return dq_s, dk_s
+
+
+def streamkl_bwd_teacher(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
+                         kl, lse_t, lse_s, g, dq_t=None, dk_t=None, stream=None):
+    """dQ_T [B,H,N_Q,d_T] and dK_T [B,H,N_K,d_T] (fp32) of sum_i g_i KL_i (trainable teacher)."""
+    import torch
+    B, H, n_q, n_k, d_t, d_s = _shape(q_t, k_t, q_s, k_s)
+    dev = q_t.device
+    for name, t in (("kl", kl), ("lse_t", lse_t), ("lse_s", lse_s), ("g", g)):
+        if t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != (B, H, n_q):
+            raise ValueError(f"{name} must be contiguous fp32 [B,H,N_Q]")
+    dq_t = torch.empty(B, H, n_q, d_t, device=dev, dtype=torch.float32) if dq_t is None else dq_t
+    dk_t = torch.empty(B, H, n_k, d_t, device=dev, dtype=torch.float32) if dk_t is None else dk_t
+    st = streamkl_bwd_teacher_raw(q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(),
+                                  k_s.data_ptr(), B, H, n_q, n_k, d_t, d_s, scale_T, scale_S,
+                                  causal, kl.data_ptr(), lse_t.data_ptr(), lse_s.data_ptr(),
+                                  g.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(),
+                                  _stream_ptr(stream))
+    _check(st, "streamkl_bwd_teacher")
+    return dq_t, dk_t
 
 
 def device_status(stream=None) -> int:

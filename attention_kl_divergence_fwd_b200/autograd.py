@@ -1,7 +1,7 @@
 """PyTorch autograd wrapper over the StreamKL C ABI, with the usual loss reductions.
 
     loss = attention_kl_loss(q_t, k_t, q_s, k_s, causal=True, reduction="mean")
-    loss.backward()          # fills q_s.grad and k_s.grad (the teacher is frozen)
+    loss.backward()          # fills q_s.grad and k_s.grad; q_t/k_t too if they require grad
 
 The forward calls ``streamkl_fwd`` (per-row KL plus the two log-sum-exps it saves for
 backward); the backward calls ``streamkl_bwd`` with g = dLoss/dKL per row, which the
@@ -16,34 +16,48 @@ from typing import Optional
 
 import torch
 
-from . import streamkl_bwd, streamkl_fwd
+from . import streamkl_bwd, streamkl_bwd_teacher, streamkl_fwd
 
 REDUCTIONS = ("none", "sum", "mean", "batchmean")
 
 
 class StreamKLFunction(torch.autograd.Function):
-    """Row-wise KL(P_T || P_S) of two attention maps; gradients flow to Q_S and K_S only."""
+    """Row-wise KL(P_T || P_S) of two attention maps.
+
+    Gradients flow to Q_S and K_S (streamkl_bwd) and, when the teacher inputs require
+    grad, to Q_T and K_T as well (streamkl_bwd_teacher).
+    """
 
     @staticmethod
     def forward(ctx, q_t, k_t, q_s, k_s, scale_t: float, scale_s: float, causal: bool):
         kl, lse_t, lse_s = streamkl_fwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal)
-        ctx.save_for_backward(q_t, k_t, q_s, k_s, lse_t, lse_s)
+        ctx.save_for_backward(q_t, k_t, q_s, k_s, kl, lse_t, lse_s)
         ctx.params = (scale_t, scale_s, causal)
         ctx.mark_non_differentiable(lse_t, lse_s)
         return kl, lse_t, lse_s
 
     @staticmethod
     def backward(ctx, g_kl, _g_lse_t=None, _g_lse_s=None):
-        q_t, k_t, q_s, k_s, lse_t, lse_s = ctx.saved_tensors
+        q_t, k_t, q_s, k_s, kl, lse_t, lse_s = ctx.saved_tensors
         scale_t, scale_s, causal = ctx.params
         g = g_kl.detach().to(torch.float32).contiguous()
-        dq, dk = streamkl_bwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, lse_t, lse_s, g)
-        return None, None, dq.to(q_s.dtype), dk.to(k_s.dtype), None, None, None
+        need_t = ctx.needs_input_grad[0] or ctx.needs_input_grad[1]
+        need_s = ctx.needs_input_grad[2] or ctx.needs_input_grad[3]
+        dq_t = dk_t = dq_s = dk_s = None
+        if need_s:
+            dq_s, dk_s = streamkl_bwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, lse_t,
+                                      lse_s, g)
+            dq_s, dk_s = dq_s.to(q_s.dtype), dk_s.to(k_s.dtype)
+        if need_t:
+            dq_t, dk_t = streamkl_bwd_teacher(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, kl,
+                                              lse_t, lse_s, g)
+            dq_t, dk_t = dq_t.to(q_t.dtype), dk_t.to(k_t.dtype)
+        return dq_t, dk_t, dq_s, dk_s, None, None, None
 
 
 def attention_kl(q_t, k_t, q_s, k_s, scale_t: Optional[float] = None,
                  scale_s: Optional[float] = None, causal: bool = False):
-    """Per-row KL [B, H, N_Q] (fp32), differentiable w.r.t. q_s and k_s.
+    """Per-row KL [B, H, N_Q] (fp32), differentiable w.r.t. q_s, k_s (and q_t, k_t).
 
     Default scales are 1/sqrt(d) of each side. Tensors: bf16 [B, H, N, d] on one GPU.
     """

@@ -4,9 +4,14 @@
 // Boosting Attention Distillation" (abstract: the backward recomputes attention
 // probabilities tile by tile instead of storing quadratic intermediates).
 //
-// With the teacher frozen and g[i] = dLoss/dKL[i]:
-//     dS[i,j] = g[i] * scale_S * (P_S[i,j] - P_T[i,j]),   P_X = 2^(t_X - LSE_X*log2 e)
-//     dQ_S = dS K_S,   dK_S = dS^T Q_S.
+// With g[i] = dLoss/dKL[i] and P_X = 2^(t_X - LSE_X*log2 e):
+//   student (TEACHER = false): dS[i,j] = g[i] * scale_S * (P_S[i,j] - P_T[i,j]),
+//                              dQ_S = dS K_S,   dK_S = dS^T Q_S;
+//   trainable teacher (TEACHER = true):
+//                              dS[i,j] = g[i] * scale_T * P_T[i,j] * ((s_T - s_S)[i,j] - E_i),
+//                              E_i = KL_i + LSE_T,i - LSE_S,i,
+//                              dQ_T = dS K_T,   dK_T = dS^T Q_T.
+// Both recompute both score tiles; the teacher variant needs one exponential per pair.
 //
 // CTA = one tile of 128 keys of one (batch, head), resident in shared memory. It walks
 // the 64-row query tiles ("steps") that can see those keys. Per step s:
@@ -17,7 +22,7 @@
 //   3. tensor core: dK_S += dS^T Q_S (TMEM accumulator over all steps) and
 //      dQ^T_part = K_S^T dS^T into TMEM buffer s&1 (d_S on the lanes, queries on columns);
 //   4. the same warpgroup copies dQ^T_part from TMEM into a shared-memory staging tile
-//      laid out as dq_s rows, and one thread adds the tile into dq_s with a bulk tensor
+//      laid out as dQ rows, and one thread adds the tile into dQ with a bulk tensor
 //      reduce-add (the fp32 adds happen in L2).
 // Score tiles, dS tiles and dQ parts are double-buffered, so the two warpgroups work on
 // alternate steps while the tensor core computes the next ones.
@@ -37,17 +42,21 @@ struct BwdArgs {
   int causal;
   int off;          // N_K - N_Q
   float cT, cS;     // |scale| * log2(e)
-  float scale_S;    // signed student scale (folded into G = g * scale_S)
+  float aT, aS;     // |scale| (natural units, teacher gradient only)
+  float scale_G;    // signed scale of the side being differentiated (G = g * scale_G)
   int n_ktiles;     // ceil(N_K / 128)
   int n_qtiles;     // ceil(N_Q / 64)
   const float* lse_t;
   const float* lse_s;
   const float* g;
-  float* dq_s;
-  float* dk_s;
+  const float* kl;  // teacher gradient only: E = KL + LSE_T - LSE_S
+  float* dq;        // dQ of the differentiated side [BH, N_Q, d_G]
+  float* dk;        // dK of the differentiated side [BH, N_K, d_G]
 };
 
-template <int DT, int DS>
+// TEACHER = false: gradients of the student (dQ_S, dK_S), d_G = d_S.
+// TEACHER = true: gradients of a trainable teacher (dQ_T, dK_T), d_G = d_T.
+template <int DT, int DS, bool TEACHER = false>
 struct BwdCfg {
   static constexpr int BN = 128;  // keys per CTA (TMEM lanes)
   static constexpr int BM = 64;   // queries per step
@@ -59,23 +68,24 @@ struct BwdCfg {
   static constexpr int QS_TILE = BM * DS * 2;
   static constexpr int Q_STAGE = QT_TILE + QS_TILE;
   static constexpr int DS_TILE = BN * BM * 2;  // bf16 dS^T [128 keys][64 queries]
-  static constexpr int STATS = 3 * BM * 4;     // -LSE_T*log2e, -LSE_S*log2e, g*scale_S
+  static constexpr int DG = TEACHER ? DT : DS;  // head dim of the differentiated side
+  static constexpr int STATS = 4 * BM * 4;     // -LSE_T*log2e, -LSE_S*log2e, g*scale_G, E
   static constexpr int OFF_KT = 0;
   static constexpr int OFF_KS = OFF_KT + KT_TILE;
   static constexpr int OFF_Q = OFF_KS + KS_TILE;           // NQST stages {Q_T, Q_S}
   static constexpr int OFF_DS = OFF_Q + NQST * Q_STAGE;    // two dS tiles
-  static constexpr int STG_TILE = BM * DS * 4;             // fp32 dQ staging tile
+  static constexpr int STG_TILE = BM * DG * 4;             // fp32 dQ staging tile
   static constexpr int OFF_STG = OFF_DS + 2 * DS_TILE;
   static constexpr int OFF_ST = OFF_STG + STG_TILE;        // NSTS statistics slots
   static constexpr int OFF_BAR = OFF_ST + NSTS * STATS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES;  // the dynamic base is 1024-byte aligned
   static constexpr int THREADS = 384;
-  // TMEM columns: S_T^T / S_S^T per buffer, dK_S, dQ^T per buffer.
+  // TMEM columns: S_T^T / S_S^T per buffer, dK, dQ^T per buffer.
   static constexpr int TM_S = 0;          // buffer b: [128b, 128b+64) S_T, [+64, +128) S_S
-  static constexpr int TM_DK = 256;       // d_S columns
-  static constexpr int TM_DQ = 256 + DS;  // buffer b: + 64 b
-  static constexpr int DQ_M = DS;         // M of the dQ^T MMA (64 uses half the lanes)
+  static constexpr int TM_DK = 256;       // d_G columns
+  static constexpr int TM_DQ = 256 + DG;  // buffer b: + 64 b
+  static constexpr int DQ_M = DG;         // M of the dQ^T MMA (64 uses half the lanes)
   static_assert(TM_DQ + 2 * BM <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -98,7 +108,7 @@ __device__ __forceinline__ void skl_fail_b(volatile int* abort_flag) {
   *abort_flag = 1;
 }
 
-template <int DT, int DS>
+template <int DT, int DS, bool TEACHER>
 __global__ void __launch_bounds__(384, 1)
 streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                     const __grid_constant__ CUtensorMap map_kt,
@@ -107,7 +117,8 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                     const __grid_constant__ CUtensorMap map_dq, const BwdArgs args,
                     const uint32_t idesc_st, const uint32_t idesc_ss, const uint32_t idesc_dk,
                     const uint32_t idesc_dq) {
-  using C = BwdCfg<DT, DS>;
+  using C = BwdCfg<DT, DS, TEACHER>;
+  constexpr int DG = C::DG;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const uint32_t sb = smem_u32(smem);
@@ -210,28 +221,31 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     }
   } else if (warp == 10) {
     // ------------------------------------------------ row-statistics loader
-    // Each lane owns query rows lane and lane+32 of every step. Raw LSE_T, LSE_S and g
-    // are loaded kStatAhead steps before they are needed and kept in registers.
+    // Each lane owns query rows lane and lane+32 of every step. Raw LSE_T, LSE_S, g (and
+    // KL for the teacher gradient) are loaded kStatAhead steps before they are needed and
+    // kept in registers.
     constexpr int kStatAhead = 3;
     const float LOG2E = 1.4426950408889634f;
-    float r_lt[kStatAhead][2], r_ls[kStatAhead][2], r_g[kStatAhead][2];
-    auto load_step = [&](int s, float (&lt)[2], float (&ls)[2], float (&gg)[2]) {
+    float r_lt[kStatAhead][2], r_ls[kStatAhead][2], r_g[kStatAhead][2], r_kl[kStatAhead][2];
+    auto load_step = [&](int s, float (&lt)[2], float (&ls)[2], float (&gg)[2], float (&kv)[2]) {
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int row = (jq_begin + s) * C::BM + r * 32 + lane;
         lt[r] = -INFINITY;
         ls[r] = -INFINITY;
         gg[r] = 0.f;
+        kv[r] = 0.f;
         if (s < n_steps && row < args.N_Q) {
           const size_t o = (size_t)bh * args.N_Q + row;
           lt[r] = __ldg(args.lse_t + o);
           ls[r] = __ldg(args.lse_s + o);
           gg[r] = __ldg(args.g + o);
+          if (TEACHER) kv[r] = __ldg(args.kl + o);
         }
       }
     };
 #pragma unroll
-    for (int k = 0; k < kStatAhead; ++k) load_step(k, r_lt[k], r_ls[k], r_g[k]);
+    for (int k = 0; k < kStatAhead; ++k) load_step(k, r_lt[k], r_ls[k], r_g[k], r_kl[k]);
     bool ok = true;
     for (int s = 0; s < n_steps; ++s) {
       if (lane == 0 && !mbar_wait(smem_u32(&bars->st_empty[s & 1]), ((s >> 1) & 1) ^ 1)) {
@@ -240,15 +254,17 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      // Slot s&1: -LSE_T*log2e, -LSE_S*log2e, g*scale_S (rows without keys: -inf, -inf, 0).
-      float* sts = stats + (s & 1) * (3 * C::BM);
+      // Slot s&1: -LSE_T*log2e, -LSE_S*log2e, g*scale_G, E = KL + LSE_T - LSE_S
+      // (rows without keys: -inf, -inf, 0, 0).
+      float* sts = stats + (s & 1) * (4 * C::BM);
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const float lt = r_lt[0][r], ls = r_ls[0][r];
         const bool live = lt != -INFINITY && ls != -INFINITY;
         sts[r * 32 + lane] = live ? -lt * LOG2E : -INFINITY;
         sts[C::BM + r * 32 + lane] = live ? -ls * LOG2E : -INFINITY;
-        sts[2 * C::BM + r * 32 + lane] = live ? r_g[0][r] * args.scale_S : 0.f;
+        sts[2 * C::BM + r * 32 + lane] = live ? r_g[0][r] * args.scale_G : 0.f;
+        sts[3 * C::BM + r * 32 + lane] = live ? r_kl[0][r] + (lt - ls) : 0.f;
       }
       mbar_arrive(smem_u32(&bars->st_full[s & 1]));
 #pragma unroll
@@ -258,8 +274,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           r_lt[k][r] = r_lt[k + 1][r];
           r_ls[k][r] = r_ls[k + 1][r];
           r_g[k][r] = r_g[k + 1][r];
+          r_kl[k][r] = r_kl[k + 1][r];
         }
-      load_step(s + kStatAhead, r_lt[kStatAhead - 1], r_ls[kStatAhead - 1], r_g[kStatAhead - 1]);
+      load_step(s + kStatAhead, r_lt[kStatAhead - 1], r_ls[kStatAhead - 1], r_g[kStatAhead - 1],
+                r_kl[kStatAhead - 1]);
     }
   } else if (warp == 11) {
     // ------------------------------------------------------- dQ reduce issuer
@@ -272,7 +290,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         }
         const int i0 = (jq_begin + p) * C::BM;
 #pragma unroll
-        for (int db = 0; db < DS / 32; ++db)
+        for (int db = 0; db < DG / 32; ++db)
           tma_reduce_add_3d(&map_dq, sb + C::OFF_STG + db * (C::BM * 128), db * 32, i0, bh);
         bulk_commit_group();
         bulk_wait_group_read0();
@@ -326,22 +344,24 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         if (!mbar_wait(smem_u32(&bars->ds_full[pb]), (p >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s_ds = sb + C::OFF_DS + pb * C::DS_TILE;
-        const uint32_t s_qs = sb + C::OFF_Q + pst * C::Q_STAGE + C::QT_TILE;
-        // dK_S += dS^T Q_S : A = dS^T [keys][queries] K-major, B = Q_S [queries][d] MN-major.
+        // Q tile of the differentiated side (student Q_S, or teacher Q_T).
+        const uint32_t s_qg = sb + C::OFF_Q + pst * C::Q_STAGE + (TEACHER ? 0 : C::QT_TILE);
+        // dK += dS^T Q : A = dS^T [keys][queries] K-major, B = Q [queries][d] MN-major.
 #pragma unroll
         for (int kk = 0; kk < C::BM / 16; ++kk) {
           umma_bf16_ss(tmem + C::TM_DK, sdesc_sw128(s_ds + kk * 32, 16, 1024),
-                       sdesc_sw128(s_qs + kk * 2048, C::BM * 128, 1024), idesc_dk,
+                       sdesc_sw128(s_qg + kk * 2048, C::BM * 128, 1024), idesc_dk,
                        (p > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(smem_u32(&bars->q_empty[pst]));
         if (!mbar_wait(smem_u32(&bars->dq_free[pb]), ((p >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        // dQ^T = K_S^T dS^T : A = K_S [keys][d] MN-major, B = dS^T [keys][queries] MN-major.
+        // dQ^T = K^T dS^T : A = K [keys][d] MN-major, B = dS^T [keys][queries] MN-major.
+        const uint32_t s_kg = TEACHER ? s_kt : s_ks;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
           umma_bf16_ss(tmem + C::TM_DQ + pb * C::BM,
-                       sdesc_sw128(s_ks + kk * 2048, C::BN * 128, 1024),
+                       sdesc_sw128(s_kg + kk * 2048, C::BN * 128, 1024),
                        sdesc_sw128(s_ds + kk * 2048, C::BN * 128, 1024), idesc_dq, kk > 0 ? 1u : 0u);
         }
         umma_commit(smem_u32(&bars->ds_empty[pb]));
@@ -360,14 +380,14 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     const int kl = quarter * 32 + lane;  // key row within the tile = TMEM lane
     const int key = k0 + kl;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const float cT = args.cT, cS = args.cS;
+    const float cT = args.cT, cS = args.cS, aT = args.aT, aS = args.aS;
     const uint32_t s_ds_row = sb + C::OFF_DS + wg * C::DS_TILE + kl * 128;
     // dQ^T lanes are d: all 32 lanes of a quarter for d_S = 128; for d_S = 64 the M=64
     // layout puts rows 16w..16w+15 on lanes 32w..32w+15.
     const bool dq_lane_ok = (C::DQ_M == 128) || lane < 16;
     const int dq_d = (C::DQ_M == 128) ? kl : quarter * 16 + lane;
 
-    // dQ^T part of step p (TMEM) -> staging tile (dq_s row layout: 32-column boxes of
+    // dQ^T part of step p (TMEM) -> staging tile (dQ row layout: 32-column boxes of
     // 64 rows x 128 bytes, 128-byte swizzle) -> one bulk reduce-add by warp 11.
     auto drain_dq = [&](int p) -> bool {
       if (!mbar_wait(smem_u32(&bars->dq_full[wg]), (p >> 1) & 1)) return false;
@@ -413,7 +433,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[wg]));
       if (!mbar_wait(smem_u32(&bars->st_full[s & 1]), (s >> 1) & 1)) { ok = false; break; }
-      const float* sts = stats + (s & 1) * (3 * C::BM);
+      const float* sts = stats + (s & 1) * (4 * C::BM);
       // The dS buffer is free once the dK/dQ MMAs of step s-2 have read it (they were
       // issued before this step's scores, so this wait normally returns at once).
       if (!mbar_wait(smem_u32(&bars->ds_empty[wg]), ((s >> 1) & 1) ^ 1)) { ok = false; break; }
@@ -432,13 +452,29 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         const float nlt[8] = {nlt0.x, nlt0.y, nlt0.z, nlt0.w, nlt1.x, nlt1.y, nlt1.z, nlt1.w};
         const float nls[8] = {nls0.x, nls0.y, nls0.z, nls0.w, nls1.x, nls1.y, nls1.z, nls1.w};
         const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        float ee[8];
+        if (TEACHER) {
+          const float4 e0 = *reinterpret_cast<const float4*>(sts + 3 * C::BM + u * 8);
+          const float4 e1 = *reinterpret_cast<const float4*>(sts + 3 * C::BM + u * 8 + 4);
+          ee[0] = e0.x; ee[1] = e0.y; ee[2] = e0.z; ee[3] = e0.w;
+          ee[4] = e1.x; ee[5] = e1.y; ee[6] = e1.z; ee[7] = e1.w;
+        }
         float d[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int c = u * 8 + e;
           const float pT = ex2_approx(fmaf(__uint_as_float(vt[c]), cT, nlt[e]));
-          const float pS = ex2_approx(fmaf(__uint_as_float(vs[c]), cS, nls[e]));
-          float ds = gg[e] * (pS - pT);
+          float ds;
+          if (TEACHER) {
+            // g*scale_T * P_T * ((s_T - s_S) - E), scores in natural units; both products
+            // rounded alike so that identical teacher and student scores cancel exactly.
+            const float w = __fsub_rn(__fmul_rn(__uint_as_float(vt[c]), aT),
+                                      __fmul_rn(__uint_as_float(vs[c]), aS)) - ee[e];
+            ds = gg[e] * pT * w;
+          } else {
+            const float pS = ex2_approx(fmaf(__uint_as_float(vs[c]), cS, nls[e]));
+            ds = gg[e] * (pS - pT);
+          }
           if (need_mask && c < cmin) ds = 0.f;
           d[e] = ds;
         }
@@ -456,7 +492,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     if (ok && last >= 0 && !drain_dq(last)) ok = false;
 
     // dK_S rows of this key tile (TMEM lanes = keys); zero when no query sees them.
-    constexpr int DKH = DS / 2;  // dK columns handled by this warpgroup
+    constexpr int DKH = DG / 2;  // dK columns handled by this warpgroup
     if (ok) {
       uint32_t v[DKH];
       if (n_steps > 0) {
@@ -476,7 +512,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         for (int c = 0; c < DKH; ++c) v[c] = 0u;
       }
       if (ok && key < args.N_K) {
-        float4* dst = reinterpret_cast<float4*>(args.dk_s + ((size_t)bh * args.N_K + key) * DS +
+        float4* dst = reinterpret_cast<float4*>(args.dk + ((size_t)bh * args.N_K + key) * DG +
                                                 wg * DKH);
 #pragma unroll
         for (int c = 0; c < DKH; c += 4)

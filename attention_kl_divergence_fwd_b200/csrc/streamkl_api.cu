@@ -104,20 +104,68 @@ streamkl_status launch_fwd(const CUtensorMap* maps, const skl::FwdArgs& a, bool 
   return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
 }
 
-template <int DT, int DS>
+template <int DT, int DS, bool TEACHER>
 streamkl_status launch_bwd(const CUtensorMap* maps, const skl::BwdArgs& a, bool negT, bool negS,
                            cudaStream_t stream) {
-  using C = skl::BwdCfg<DT, DS>;
-  auto kern = skl::streamkl_bwd_kernel<DT, DS>;
+  using C = skl::BwdCfg<DT, DS, TEACHER>;
+  auto kern = skl::streamkl_bwd_kernel<DT, DS, TEACHER>;
   if (!set_smem(kern, C::SMEM)) return STREAMKL_ERR_LAUNCH;
   const uint32_t i_st = skl::idesc_bf16_f32(128, C::BM, false, false, negT);
   const uint32_t i_ss = skl::idesc_bf16_f32(128, C::BM, false, false, negS);
-  const uint32_t i_dk = skl::idesc_bf16_f32(128, DS, false, true);   // dS^T Q_S
-  const uint32_t i_dq = skl::idesc_bf16_f32(DS, C::BM, true, true);  // K_S^T dS^T
+  const uint32_t i_dk = skl::idesc_bf16_f32(128, C::DG, false, true);   // dS^T Q
+  const uint32_t i_dq = skl::idesc_bf16_f32(C::DG, C::BM, true, true);  // K^T dS^T
   const long long grid = (long long)a.n_ktiles * a.BH;
   kern<<<dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream>>>(
       maps[0], maps[1], maps[2], maps[3], maps[4], a, i_st, i_ss, i_dk, i_dq);
   return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
+}
+
+// Shared body of streamkl_bwd (student gradients) and streamkl_bwd_teacher.
+template <bool TEACHER>
+streamkl_status bwd_common(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
+                           int B, int H, int N_Q, int N_K, int d_T, int d_S, float scale_T,
+                           float scale_S, int causal, const float* kl, const float* lse_t,
+                           const float* lse_s, const float* g, float* dq, float* dk,
+                           cudaStream_t stream) {
+  streamkl_status st = check_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S);
+  if (st != STREAMKL_OK) return st;
+  if (!lse_t || !lse_s || !g || !dq || !dk || (TEACHER && !kl)) return STREAMKL_ERR_INVALID_ARG;
+  if (!aligned16(lse_t) || !aligned16(lse_s) || !aligned16(g) || !aligned16(dq) ||
+      !aligned16(dk) || (TEACHER && !aligned16(kl)))
+    return STREAMKL_ERR_MISALIGNED;
+  const int bh = B * H;
+  const int d_g = TEACHER ? d_T : d_S;
+  CUtensorMap maps[5];
+  if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 64) || !make_map(&maps[1], k_t, d_T, N_K, bh, 128) ||
+      !make_map(&maps[2], q_s, d_S, N_Q, bh, 64) || !make_map(&maps[3], k_s, d_S, N_K, bh, 128) ||
+      !make_map_f32(&maps[4], dq, d_g, N_Q, bh))
+    return STREAMKL_ERR_LAUNCH;
+  if (cudaMemsetAsync(dq, 0, (size_t)bh * N_Q * d_g * sizeof(float), stream) != cudaSuccess)
+    return STREAMKL_ERR_LAUNCH;
+  skl::BwdArgs a{};
+  a.BH = bh;
+  a.N_Q = N_Q;
+  a.N_K = N_K;
+  a.causal = causal ? 1 : 0;
+  a.off = N_K - N_Q;
+  a.cT = std::fabs(scale_T) * kLog2e;
+  a.cS = std::fabs(scale_S) * kLog2e;
+  a.aT = std::fabs(scale_T);
+  a.aS = std::fabs(scale_S);
+  a.scale_G = TEACHER ? scale_T : scale_S;
+  a.n_ktiles = (N_K + 127) / 128;
+  a.n_qtiles = (N_Q + 63) / 64;
+  a.lse_t = lse_t;
+  a.lse_s = lse_s;
+  a.g = g;
+  a.kl = kl;
+  a.dq = dq;
+  a.dk = dk;
+  const bool nT = scale_T < 0.f, nS = scale_S < 0.f;
+  if (d_T == 128 && d_S == 128) return launch_bwd<128, 128, TEACHER>(maps, a, nT, nS, stream);
+  if (d_T == 128 && d_S == 64) return launch_bwd<128, 64, TEACHER>(maps, a, nT, nS, stream);
+  if (d_T == 64 && d_S == 128) return launch_bwd<64, 128, TEACHER>(maps, a, nT, nS, stream);
+  return launch_bwd<64, 64, TEACHER>(maps, a, nT, nS, stream);
 }
 
 }  // namespace
@@ -160,41 +208,18 @@ streamkl_status streamkl_bwd(const void* q_t, const void* k_t, const void* q_s, 
                              int B, int H, int N_Q, int N_K, int d_T, int d_S, float scale_T,
                              float scale_S, int causal, const float* lse_t, const float* lse_s,
                              const float* g, float* dq_s, float* dk_s, cudaStream_t stream) {
-  streamkl_status st = check_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S);
-  if (st != STREAMKL_OK) return st;
-  if (!lse_t || !lse_s || !g || !dq_s || !dk_s) return STREAMKL_ERR_INVALID_ARG;
-  if (!aligned16(lse_t) || !aligned16(lse_s) || !aligned16(g) || !aligned16(dq_s) ||
-      !aligned16(dk_s))
-    return STREAMKL_ERR_MISALIGNED;
-  const int bh = B * H;
-  CUtensorMap maps[5];
-  if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 64) || !make_map(&maps[1], k_t, d_T, N_K, bh, 128) ||
-      !make_map(&maps[2], q_s, d_S, N_Q, bh, 64) || !make_map(&maps[3], k_s, d_S, N_K, bh, 128) ||
-      !make_map_f32(&maps[4], dq_s, d_S, N_Q, bh))
-    return STREAMKL_ERR_LAUNCH;
-  if (cudaMemsetAsync(dq_s, 0, (size_t)bh * N_Q * d_S * sizeof(float), stream) != cudaSuccess)
-    return STREAMKL_ERR_LAUNCH;
-  skl::BwdArgs a{};
-  a.BH = bh;
-  a.N_Q = N_Q;
-  a.N_K = N_K;
-  a.causal = causal ? 1 : 0;
-  a.off = N_K - N_Q;
-  a.cT = std::fabs(scale_T) * kLog2e;
-  a.cS = std::fabs(scale_S) * kLog2e;
-  a.scale_S = scale_S;
-  a.n_ktiles = (N_K + 127) / 128;
-  a.n_qtiles = (N_Q + 63) / 64;
-  a.lse_t = lse_t;
-  a.lse_s = lse_s;
-  a.g = g;
-  a.dq_s = dq_s;
-  a.dk_s = dk_s;
-  const bool nT = scale_T < 0.f, nS = scale_S < 0.f;
-  if (d_T == 128 && d_S == 128) return launch_bwd<128, 128>(maps, a, nT, nS, stream);
-  if (d_T == 128 && d_S == 64) return launch_bwd<128, 64>(maps, a, nT, nS, stream);
-  if (d_T == 64 && d_S == 128) return launch_bwd<64, 128>(maps, a, nT, nS, stream);
-  return launch_bwd<64, 64>(maps, a, nT, nS, stream);
+  return bwd_common<false>(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S, causal,
+                           nullptr, lse_t, lse_s, g, dq_s, dk_s, stream);
+}
+
+streamkl_status streamkl_bwd_teacher(const void* q_t, const void* k_t, const void* q_s,
+                                     const void* k_s, int B, int H, int N_Q, int N_K, int d_T,
+                                     int d_S, float scale_T, float scale_S, int causal,
+                                     const float* kl, const float* lse_t, const float* lse_s,
+                                     const float* g, float* dq_t, float* dk_t,
+                                     cudaStream_t stream) {
+  return bwd_common<true>(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S, causal,
+                          kl, lse_t, lse_s, g, dq_t, dk_t, stream);
 }
 
 const char* streamkl_status_string(streamkl_status s) {

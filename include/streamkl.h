@@ -14,7 +14,8 @@
  * "online formulation for the coupled two-distribution KL reduction" and "single
  * one-pass forward kernel"). The backward recomputes both probability tiles from the
  * saved log-sum-exps (the abstract's "recomputes attention probabilities
- * tile-by-tile"). The teacher is frozen: only the student gets gradients.
+ * tile-by-tile"). streamkl_bwd gives the student's gradients (teacher frozen, the
+ * abstract's setting); streamkl_bwd_teacher gives a trainable teacher's.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -79,14 +80,32 @@ streamkl_status streamkl_fwd(const void* q_t, const void* k_t, const void* q_s, 
  *   dS[i,j] = g[i] * scale_S * (P_S[i,j] - P_T[i,j])   on J(i), 0 elsewhere,
  *   dq_s = dS K_S   (fp32 [B,H,N_Q,d_S], fully overwritten: zeroed on `stream` first),
  *   dk_s = dS^T Q_S (fp32 [B,H,N_K,d_S], fully overwritten).
- * dq_s is accumulated with fp32 atomic reductions, so its low bits can differ between
- * runs; dk_s is deterministic.
+ * dq_s is accumulated with fp32 reductions in L2 (one partial per key tile), so its low
+ * bits can differ between runs; dk_s is deterministic.
  */
 streamkl_status streamkl_bwd(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
                              int B, int H, int N_Q, int N_K, int d_T, int d_S,
                              float scale_T, float scale_S, int causal,
                              const float* lse_t, const float* lse_s, const float* g,
                              float* dq_s, float* dk_s, cudaStream_t stream);
+
+/*
+ * Backward for a trainable teacher (the abstract's use of the primitive is one-sided,
+ * teacher frozen; this is the same recompute scheme for the other side). With the
+ * student fixed, dKL_i/ds_T[i,j] = P_T[i,j] * ((s_T - s_S)[i,j] - E_i) where
+ * E_i = sum_j P_T[i,j] (s_T - s_S)[i,j] = KL_i + LSE_T,i - LSE_S,i, so with g[i] = dLoss/dKL[i]:
+ *   dS_T[i,j] = g[i] * scale_T * P_T[i,j] * ((s_T - s_S)[i,j] - E_i)   on J(i), else 0,
+ *   dq_t = dS_T K_T (fp32 [B,H,N_Q,d_T], fully overwritten: zeroed on `stream` first),
+ *   dk_t = dS_T^T Q_T (fp32 [B,H,N_K,d_T], fully overwritten).
+ * kl, lse_t and lse_s are the forward's outputs (fp32 [B,H,N_Q]); everything else as in
+ * streamkl_bwd. Call both backward entry points to train teacher and student together.
+ */
+streamkl_status streamkl_bwd_teacher(const void* q_t, const void* k_t, const void* q_s,
+                                     const void* k_s, int B, int H, int N_Q, int N_K, int d_T,
+                                     int d_S, float scale_T, float scale_S, int causal,
+                                     const float* kl, const float* lse_t, const float* lse_s,
+                                     const float* g, float* dq_t, float* dk_t,
+                                     cudaStream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char* streamkl_status_string(streamkl_status status);

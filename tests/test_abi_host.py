@@ -66,7 +66,15 @@ def bwd(**kw):
     return skl.streamkl_bwd_raw(**a)
 
 
-@pytest.mark.parametrize("fn", [fwd, bwd])
+def bwd_teacher(**kw):
+    a = dict(q_t=P, k_t=P, q_s=P, k_s=P, B=1, H=1, N_Q=128, N_K=128, d_T=128, d_S=128,
+             scale_T=0.1, scale_S=0.1, causal=False, kl=P, lse_t=P, lse_s=P, g=P, dq_t=P,
+             dk_t=P, stream=0)
+    a.update(kw)
+    return skl.streamkl_bwd_teacher_raw(**a)
+
+
+@pytest.mark.parametrize("fn", [fwd, bwd, bwd_teacher])
 def test_host_validation(lib, fn):
     assert fn(q_t=0) == 1
     assert fn(k_s=0) == 1
@@ -90,3 +98,6 @@ def test_host_validation_outputs(lib):
     assert bwd(g=0) == 1
     assert bwd(dk_s=P + 12) == 3
     assert bwd(lse_t=0) == 1
+    assert bwd_teacher(kl=0) == 1
+    assert bwd_teacher(kl=P + 4) == 3
+    assert bwd_teacher(dk_t=P + 8) == 3

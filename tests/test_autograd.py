@@ -48,15 +48,30 @@ def test_loss_and_grads_match_oracle(reduction):
 
 
 @pytest.mark.gpu
-def test_default_scales_and_no_teacher_grad():
+def test_trainable_teacher_grads_match_oracle():
+    from oracle import oracle_bwd_teacher
+    w = WORKLOADS["b2h16_n4096_d128_causal"].with_sizes(B=1, H=2, N_Q=260, N_K=260)
+    x = make_inputs(w, seed=23)
+    d = {k: v.cuda() for k, v in x.items()}
+    q_t = d["q_t"].clone().requires_grad_(True)
+    k_t = d["k_t"].clone().requires_grad_(True)
+    ska.attention_kl_loss(q_t, k_t, d["q_s"], d["k_s"], w.scale_T, w.scale_S, True,
+                          "sum").backward()
+    dq, dk = oracle_bwd_teacher(x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S,
+                                True, torch.ones_like(x["g"]))
+    rel = lambda a, b: ((a.double().cpu() - b).norm() / b.norm()).item()
+    assert rel(q_t.grad, dq) < 1.5e-2 and rel(k_t.grad, dk) < 1.5e-2
+
+
+@pytest.mark.gpu
+def test_default_scales_and_frozen_teacher():
     w = WORKLOADS["tiny_n256_d64"]
     x = make_inputs(w)
     d = {k: v.cuda() for k, v in x.items()}
-    q_t = d["q_t"].clone().requires_grad_(True)
     q_s = d["q_s"].clone().requires_grad_(True)
-    kl = ska.attention_kl(q_t, d["k_t"], q_s, d["k_s"])  # scales default to 1/sqrt(64)
+    kl = ska.attention_kl(d["q_t"], d["k_t"], q_s, d["k_s"])  # scales default to 1/sqrt(64)
     kl.sum().backward()
-    assert q_t.grad is None
+    assert q_s.grad is not None and d["q_t"].grad is None
     kl2 = ska.attention_kl(d["q_t"], d["k_t"], d["q_s"], d["k_s"], 1 / math.sqrt(64),
                            1 / math.sqrt(64))
     assert torch.equal(kl.detach(), kl2)

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import attention_kl_divergence_fwd_b200 as skl
-from oracle import oracle_bwd, oracle_dk_rows, oracle_fwd, oracle_rows
+from oracle import oracle_bwd, oracle_bwd_teacher, oracle_dk_rows, oracle_fwd, oracle_rows
 from workloads import WORKLOADS, WORKLOAD_LIST, make_inputs, sample_keys, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -154,6 +154,42 @@ def test_repeatable_and_no_allocation():
     assert rel_fro(dq2.double(), dq.double()) < 1e-5
     # every buffer above existed before free0; the library adds nothing on the device
     assert free1 == free0
+
+
+# ------------------------------------------------- trainable-teacher gradient
+
+@pytest.mark.parametrize("nq,nk,dt,ds,causal", [
+    (300, 300, 128, 128, True),
+    (333, 517, 128, 64, False),
+    (517, 333, 64, 128, True),
+    (640, 640, 64, 64, True),
+])
+def test_teacher_grads_full(nq, nk, dt, ds, causal):
+    w = BASE.with_sizes(B=1, H=2, N_Q=nq, N_K=nk, d_T=dt, d_S=ds, causal=causal,
+                        scale_T=1 / math.sqrt(dt), scale_S=-0.7 / math.sqrt(ds),
+                        student="independent")
+    x = make_inputs(w, seed=nq + 3 * nk)
+    d = to_dev(x)
+    a = (d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal)
+    kl, lt, ls = skl.streamkl_fwd(*a)
+    dq, dk = skl.streamkl_bwd_teacher(*a, kl, lt, ls, d["g"])
+    assert skl.device_status() == 0
+    rq, rk = oracle_bwd_teacher(x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S,
+                                w.causal, x["g"])
+    assert rel_fro(dq.cpu().double(), rq) <= GRAD_REL, rel_fro(dq.cpu().double(), rq)
+    assert rel_fro(dk.cpu().double(), rk) <= GRAD_REL, rel_fro(dk.cpu().double(), rk)
+
+
+def test_teacher_grads_identical_inputs_zero():
+    w = BASE.with_sizes(B=1, H=2, N_Q=200, N_K=200, causal=True)
+    x = make_inputs(w, seed=9)
+    x["q_s"], x["k_s"] = x["q_t"].clone(), x["k_t"].clone()
+    d = to_dev(x)
+    a = (d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal)
+    kl, lt, ls = skl.streamkl_fwd(*a)
+    dq, dk = skl.streamkl_bwd_teacher(*a, kl, lt, ls, d["g"])
+    assert skl.device_status() == 0
+    assert dq.abs().max().item() == 0 and dk.abs().max().item() == 0
 
 
 # ----------------------------------------------------------- full-size workloads
