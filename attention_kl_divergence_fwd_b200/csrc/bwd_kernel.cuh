@@ -46,6 +46,7 @@ struct BwdArgs {
   float scale_G;    // signed scale of the side being differentiated (G = g * scale_G)
   int n_ktiles;     // ceil(N_K / 128)
   int n_qtiles;     // ceil(N_Q / 64)
+  int group;        // heads per scheduling group (grouped_order)
   const float* lse_t;
   const float* lse_s;
   const float* g;
@@ -132,9 +133,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x;
-  const int bh = t % args.BH;
-  const int kt = t / args.BH;  // causal: key tile 0 sees the most query tiles
+  // Key tile 0 sees the most query tiles (causal): heaviest first, heads in groups.
+  int bh, kt;
+  grouped_order(blockIdx.x, args.BH, args.n_ktiles, args.group, bh, kt);
   const int k0 = kt * C::BN;
 
   int jq_begin = 0;

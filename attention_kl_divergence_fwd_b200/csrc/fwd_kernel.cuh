@@ -32,6 +32,7 @@ struct FwdArgs {
   int off;            // N_K - N_Q (bottom-right causal alignment)
   float cT, cS;       // |scale| * log2(e); the MMA negates A when the scale is negative
   int n_ctas_per_bh;  // ceil(N_Q / 256)
+  int group;          // heads per scheduling group (grouped_order)
   float* kl;
   float* lse_t;
   float* lse_s;
@@ -208,10 +209,10 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Heaviest (last) query tiles first for causal load balance, all heads interleaved.
-  const int t = blockIdx.x;
-  const int bh = t % args.BH;
-  const int qpair = args.n_ctas_per_bh - 1 - t / args.BH;
+  // Heaviest (last) query tiles first for causal load balance, heads in groups.
+  int bh, unit;
+  grouped_order(blockIdx.x, args.BH, args.n_ctas_per_bh, args.group, bh, unit);
+  const int qpair = args.n_ctas_per_bh - 1 - unit;
   const int q0 = qpair * (C::NQ * C::BM);
   const int n_ktiles_all = (args.N_K + C::BN - 1) / C::BN;
 

@@ -242,6 +242,29 @@ __device__ __forceinline__ void tmem_ld_32_wait(uint32_t ta, uint32_t (&r)[32]) 
 
 #undef SKL_R8
 
+// ------------------------------------------------------- grid ordering
+
+// Maps a linear CTA index to (head, unit) with heads processed in groups of `group`
+// heads: inside a group the units are interleaved across its heads in the order given
+// (unit 0 first, the caller puts the heaviest causal unit first), and groups follow one
+// another. A group's working set (its heads' K/Q tiles and dQ rows) then stays in L2.
+__device__ __forceinline__ void grouped_order(int t, int bh_total, int units, int group,
+                                              int& bh, int& unit) {
+  const int full = bh_total / group;
+  const int per_group = group * units;
+  const int g = t / per_group;
+  if (g < full) {
+    const int r = t - g * per_group;
+    unit = r / group;
+    bh = g * group + r % group;
+  } else {
+    const int rest = bh_total - full * group;
+    const int r = t - full * per_group;
+    unit = r / rest;
+    bh = full * group + r % rest;
+  }
+}
+
 // ------------------------------------------------------------------ math
 
 __device__ __forceinline__ float ex2_approx(float x) {
