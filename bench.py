@@ -29,7 +29,7 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from workloads import WORKLOADS, flops_bwd, flops_fwd, make_inputs  # noqa: E402
+from workloads import WORKLOADS, flops_bwd, flops_bwd_teacher, flops_fwd, make_inputs  # noqa: E402
 
 METRIC = "fwd/bwd TFLOP/s and % of B200 bf16 peak at N=16K,d=128; ms per fwd+bwd"
 DEFAULT_WORKLOAD = "long_b1h32_n16384_d128_causal"
@@ -212,10 +212,12 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
 
-    world, rank, local = dist_setup()
     if args.impl == "reference":
-        run_reference(args, world, rank)
+        # The reference arm is the host-side oracle: rank 0 alone runs it, no process group.
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")),
+                      int(os.environ.get("RANK", "0")))
         return
+    world, rank, local = dist_setup()
 
     import attention_kl_divergence_fwd_b200 as skl
     skl.load_library()
@@ -289,6 +291,24 @@ def main():
             "traffic": traffic,
             "peak_kind": f"{peak_kind} bf16 dense, sustained (kernel timed inside a long loop)"}
 
+    # Trainable-teacher backward (streamkl_bwd_teacher), timed on its own: not part of the
+    # step (the teacher is frozen in the measured workload), reported beside it.
+    dq_t = torch.empty(B, H, nq, w.d_T, device=dev)
+    dk_t = torch.empty(B, H, nk, w.d_T, device=dev)
+    for _ in range(2):
+        skl.streamkl_bwd_teacher(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S,
+                                 w.causal, kl, lt, ls, d["g"], dq_t=dq_t, dk_t=dk_t)
+    torch.cuda.synchronize()
+    te0, te1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    te0.record(stream)
+    for _ in range(args.steps):
+        skl.streamkl_bwd_teacher(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S,
+                                 w.causal, kl, lt, ls, d["g"], dq_t=dq_t, dk_t=dk_t)
+    te1.record(stream)
+    torch.cuda.synchronize()
+    bwd_t_ms = max_over_ranks(te0.elapsed_time(te1) / args.steps, world)
+    del dq_t, dk_t
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(skl, w, x, dev, stream, args.steps, world)
@@ -307,6 +327,8 @@ def main():
                "fwd_frac_burst_peak": fwd_tf / peak_burst,
                "bwd_frac_burst_peak": bwd_tf / peak_burst,
                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+               "bwd_teacher_ms": bwd_t_ms,
+               "bwd_teacher_tflops": flops_bwd_teacher(w) / (bwd_t_ms * 1e-3) / 1e12,
                "gpu_launches": 2 * args.steps,
                "extra_hbm_bytes": 3 * 4 * w.bh * w.N_Q,
                "impl": "ours"}

@@ -161,6 +161,12 @@ def flops_bwd(w: Workload) -> float:
     return 2.0 * allowed_pairs(w) * (w.d_T + 3 * w.d_S) * w.bh
 
 
+def flops_bwd_teacher(w: Workload) -> float:
+    """Counted trainable-teacher backward FLOPs: 2*|J|*(3*d_T + d_S) per row
+    (S_T, S_S, dQ_T, dK_T)."""
+    return 2.0 * allowed_pairs(w) * (3 * w.d_T + w.d_S) * w.bh
+
+
 def allowed_pairs(w: Workload) -> float:
     """Number of (i, j) pairs per head that the method counts.
 
