@@ -47,6 +47,10 @@ struct BwdArgs {
   int n_ktiles;     // ceil(N_K / 128)
   int n_qtiles;     // ceil(N_Q / 64)
   int group;        // heads per scheduling group (grouped_order)
+  int H;            // query heads per batch entry
+  int gT, gS;       // query heads per teacher / student K head (GQA; 1 = one K head each)
+  int dk_reduce;    // 1: several query heads share the differentiated K head, so dK
+                    //    tiles are added into the zeroed dk (bulk reduce) instead of stored
   const float* lse_t;
   const float* lse_s;
   const float* g;
@@ -115,7 +119,8 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                     const __grid_constant__ CUtensorMap map_kt,
                     const __grid_constant__ CUtensorMap map_qs,
                     const __grid_constant__ CUtensorMap map_ks,
-                    const __grid_constant__ CUtensorMap map_dq, const BwdArgs args,
+                    const __grid_constant__ CUtensorMap map_dq,
+                    const __grid_constant__ CUtensorMap map_dk, const BwdArgs args,
                     const uint32_t idesc_st, const uint32_t idesc_ss, const uint32_t idesc_dk,
                     const uint32_t idesc_dq) {
   using C = BwdCfg<DT, DS, TEACHER>;
@@ -136,6 +141,11 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   // Key tile 0 sees the most query tiles (causal): heaviest first, heads in groups.
   int bh, kt;
   grouped_order(blockIdx.x, args.BH, args.n_ktiles, args.group, bh, kt);
+  // K heads of this query head (grouped-query attention: query head h reads K head h/g).
+  const int hq = bh % args.H, bq = bh / args.H;
+  const int bkt = bq * (args.H / args.gT) + hq / args.gT;
+  const int bks = bq * (args.H / args.gS) + hq / args.gS;
+  const int bkg = TEACHER ? bkt : bks;  // K head that receives this CTA's dK
   const int k0 = kt * C::BN;
 
   int jq_begin = 0;
@@ -144,6 +154,8 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     jq_begin = first_q <= 0 ? 0 : first_q / C::BM;
   }
   const int n_steps = max(0, args.n_qtiles - jq_begin);
+  // Staging rounds after the last step that add the dK tile (128 keys = 2 x 64 rows).
+  const int dk_rounds = (args.dk_reduce && n_steps > 0) ? 2 : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->k_full), 1);
@@ -193,9 +205,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       const uint32_t kb = smem_u32(&bars->k_full);
       mbar_arrive_expect_tx(kb, C::KT_TILE + C::KS_TILE);
       for (int blk = 0; blk < DT / 64; ++blk)
-        tma_load_3d(sb + C::OFF_KT + blk * (C::BN * 128), &map_kt, kb, blk * 64, k0, bh, keep);
+        tma_load_3d(sb + C::OFF_KT + blk * (C::BN * 128), &map_kt, kb, blk * 64, k0, bkt, keep);
       for (int blk = 0; blk < DS / 64; ++blk)
-        tma_load_3d(sb + C::OFF_KS + blk * (C::BN * 128), &map_ks, kb, blk * 64, k0, bh, keep);
+        tma_load_3d(sb + C::OFF_KS + blk * (C::BN * 128), &map_ks, kb, blk * 64, k0, bks, keep);
       for (int s = 0; s < n_steps; ++s) {
         const int st = s % C::NQST;
         const int i0 = (jq_begin + s) * C::BM;
@@ -281,18 +293,26 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                 r_kl[kStatAhead - 1]);
     }
   } else if (warp == 11) {
-    // ------------------------------------------------------- dQ reduce issuer
+    // ------------------------------------------- dQ (and shared-K dK) reduce issuer
     if (lane == 0) {
       tma_prefetch_desc(&map_dq);
-      for (int p = 0; p < n_steps; ++p) {
+      if (dk_rounds) tma_prefetch_desc(&map_dk);
+      for (int p = 0; p < n_steps + dk_rounds; ++p) {
         if (!mbar_wait(smem_u32(&bars->stg_full[p & 1]), (p >> 1) & 1)) {
           skl_fail_b(abort_flag);
           break;
         }
-        const int i0 = (jq_begin + p) * C::BM;
+        if (p < n_steps) {  // dQ part of step p: 64 query rows
+          const int i0 = (jq_begin + p) * C::BM;
 #pragma unroll
-        for (int db = 0; db < DG / 32; ++db)
-          tma_reduce_add_3d(&map_dq, sb + C::OFF_STG + db * (C::BM * 128), db * 32, i0, bh);
+          for (int db = 0; db < DG / 32; ++db)
+            tma_reduce_add_3d(&map_dq, sb + C::OFF_STG + db * (C::BM * 128), db * 32, i0, bh);
+        } else {  // dK tile of this CTA, 64 key rows per round
+          const int r0 = k0 + (p - n_steps) * 64;
+#pragma unroll
+          for (int db = 0; db < DG / 32; ++db)
+            tma_reduce_add_3d(&map_dk, sb + C::OFF_STG + db * (C::BM * 128), db * 32, r0, bkg);
+        }
         bulk_commit_group();
         bulk_wait_group_read0();
         mbar_arrive(smem_u32(&bars->stg_free[p & 1]));
@@ -492,33 +512,57 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     }
     if (ok && last >= 0 && !drain_dq(last)) ok = false;
 
-    // dK_S rows of this key tile (TMEM lanes = keys); zero when no query sees them.
+    // dK rows of this key tile (TMEM lanes = keys); zero when no query sees them. With a
+    // K head shared by several query heads (dk_reduce) the tile is added into the zeroed
+    // dk through the staging tile in two 64-row rounds, continuing the staging sequence.
     constexpr int DKH = DG / 2;  // dK columns handled by this warpgroup
-    if (ok) {
-      uint32_t v[DKH];
-      if (n_steps > 0) {
-        if (!mbar_wait(smem_u32(&bars->dk_full), 0)) {
-          ok = false;
-        } else {
-          tc_fence_after();
-          if constexpr (DKH == 64) {
-            tmem_ld_2x32_wait(tmem + lane_off + C::TM_DK + wg * DKH,
-                              tmem + lane_off + C::TM_DK + wg * DKH + 32, v);
-          } else {
-            tmem_ld_32_wait(tmem + lane_off + C::TM_DK + wg * DKH, v);
-          }
-        }
+    uint32_t v[DKH];
+#pragma unroll
+    for (int c = 0; c < DKH; ++c) v[c] = 0u;
+    if (ok && n_steps > 0) {
+      if (!mbar_wait(smem_u32(&bars->dk_full), 0)) {
+        ok = false;
       } else {
-#pragma unroll
-        for (int c = 0; c < DKH; ++c) v[c] = 0u;
+        tc_fence_after();
+        if constexpr (DKH == 64) {
+          tmem_ld_2x32_wait(tmem + lane_off + C::TM_DK + wg * DKH,
+                            tmem + lane_off + C::TM_DK + wg * DKH + 32, v);
+        } else {
+          tmem_ld_32_wait(tmem + lane_off + C::TM_DK + wg * DKH, v);
+        }
       }
-      if (ok && key < args.N_K) {
-        float4* dst = reinterpret_cast<float4*>(args.dk + ((size_t)bh * args.N_K + key) * DG +
-                                                wg * DKH);
+    }
+    if (ok && !dk_rounds && key < args.N_K) {
+      float4* dst = reinterpret_cast<float4*>(args.dk + ((size_t)bkg * args.N_K + key) * DG +
+                                              wg * DKH);
 #pragma unroll
-        for (int c = 0; c < DKH; c += 4)
-          dst[c / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                   __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+      for (int c = 0; c < DKH; c += 4)
+        dst[c / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                 __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+    }
+    if (dk_rounds) {
+      // Every dS warp reaches this barrier (dk_rounds is uniform over the CTA), after its
+      // last dQ drain, so each staging wait below is at most one phase ahead of its barrier.
+      named_bar_sync(1, 256);
+      ok = __all_sync(0xffffffffu, ok);
+      for (int r = 0; ok && r < 2; ++r) {
+        const int p = n_steps + r;
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(smem_u32(&bars->stg_free[(p - 1) & 1]), ((p - 1) >> 1) & 1));
+        if (!ok) break;
+        if ((quarter >> 1) == r) {  // this warp's lanes are rows 64r .. 64r+63 of the tile
+          const int row = kl - 64 * r;
+#pragma unroll
+          for (int c = 0; c < DKH; c += 4) {
+            const int dcol = wg * DKH + c;
+            const uint32_t addr = sb + C::OFF_STG + (dcol >> 5) * (C::BM * 128) + row * 128 +
+                                  ((((dcol & 31) >> 2) ^ (row & 7)) << 4);
+            st_shared_v4(addr, v[c], v[c + 1], v[c + 2], v[c + 3]);
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bars->stg_full[p & 1]));
+        }
       }
     }
     if (!ok) skl_fail_b(abort_flag);

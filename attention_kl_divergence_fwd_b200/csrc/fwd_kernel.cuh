@@ -33,6 +33,8 @@ struct FwdArgs {
   float cT, cS;       // |scale| * log2(e); the MMA negates A when the scale is negative
   int n_ctas_per_bh;  // ceil(N_Q / 256)
   int group;          // heads per scheduling group (grouped_order)
+  int H;              // query heads per batch entry
+  int gT, gS;         // query heads per teacher / student K head (GQA; 1 = one K head each)
   float* kl;
   float* lse_t;
   float* lse_s;
@@ -213,6 +215,10 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   int bh, unit;
   grouped_order(blockIdx.x, args.BH, args.n_ctas_per_bh, args.group, bh, unit);
   const int qpair = args.n_ctas_per_bh - 1 - unit;
+  // K heads of this query head (grouped-query attention: query head h reads K head h/g).
+  const int hq = bh % args.H, bq = bh / args.H;
+  const int bkt = bq * (args.H / args.gT) + hq / args.gT;
+  const int bks = bq * (args.H / args.gS) + hq / args.gS;
   const int q0 = qpair * (C::NQ * C::BM);
   const int n_ktiles_all = (args.N_K + C::BN - 1) / C::BN;
 
@@ -342,10 +348,10 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           mbar_arrive_expect_tx(fb, C::STAGE);
           const uint32_t st = s_k + s * C::STAGE;
           for (int blk = 0; blk < DT / 64; ++blk)
-            tma_load_3d(st + blk * (C::BN * 128), &map_kt, fb, blk * 64, j * C::BN, bh, keep);
+            tma_load_3d(st + blk * (C::BN * 128), &map_kt, fb, blk * 64, j * C::BN, bkt, keep);
           for (int blk = 0; blk < DS / 64; ++blk)
             tma_load_3d(st + C::KT_TILE + blk * (C::BN * 128), &map_ks, fb, blk * 64, j * C::BN,
-                        bh, keep);
+                        bks, keep);
           issued = j + 1;
         }
         if (*abort_flag) {

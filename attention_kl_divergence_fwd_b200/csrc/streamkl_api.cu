@@ -129,31 +129,88 @@ streamkl_status launch_bwd(const CUtensorMap* maps, const skl::BwdArgs& a, bool 
   const uint32_t i_dq = skl::idesc_bf16_f32(C::DG, C::BM, true, true);  // K^T dS^T
   const long long grid = (long long)a.n_ktiles * a.BH;
   kern<<<dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream>>>(
-      maps[0], maps[1], maps[2], maps[3], maps[4], a, i_st, i_ss, i_dk, i_dq);
+      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], a, i_st, i_ss, i_dk, i_dq);
   return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
 }
 
-// Shared body of streamkl_bwd (student gradients) and streamkl_bwd_teacher.
+// Query heads per K head; UNSUPPORTED unless it divides H.
+bool kv_groups(int H, int H_kv_T, int H_kv_S, int& gT, int& gS) {
+  if (H_kv_T < 1 || H_kv_S < 1 || H % H_kv_T != 0 || H % H_kv_S != 0) return false;
+  gT = H / H_kv_T;
+  gS = H / H_kv_S;
+  return true;
+}
+
+streamkl_status fwd_common(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
+                           int B, int H, int H_kv_T, int H_kv_S, int N_Q, int N_K, int d_T,
+                           int d_S, float scale_T, float scale_S, int causal, float* kl,
+                           float* lse_t, float* lse_s, cudaStream_t stream) {
+  streamkl_status st = check_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S);
+  if (st != STREAMKL_OK) return st;
+  if (!kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
+  int gT, gS;
+  if (!kv_groups(H, H_kv_T, H_kv_S, gT, gS)) return STREAMKL_ERR_UNSUPPORTED;
+  if (!aligned16(kl) || !aligned16(lse_t) || !aligned16(lse_s)) return STREAMKL_ERR_MISALIGNED;
+  const int bh = B * H;
+  CUtensorMap maps[4];
+  if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 128) ||
+      !make_map(&maps[1], k_t, d_T, N_K, B * H_kv_T, 64) ||
+      !make_map(&maps[2], q_s, d_S, N_Q, bh, 128) ||
+      !make_map(&maps[3], k_s, d_S, N_K, B * H_kv_S, 64))
+    return STREAMKL_ERR_LAUNCH;
+  skl::FwdArgs a{};
+  a.BH = bh;
+  a.N_Q = N_Q;
+  a.N_K = N_K;
+  a.causal = causal ? 1 : 0;
+  a.off = N_K - N_Q;
+  a.cT = std::fabs(scale_T) * kLog2e;
+  a.cS = std::fabs(scale_S) * kLog2e;
+  a.n_ctas_per_bh = (N_Q + 255) / 256;
+  a.group = head_group("STREAMKL_FWD_GROUP", 4, bh);
+  a.H = H;
+  a.gT = gT;
+  a.gS = gS;
+  a.kl = kl;
+  a.lse_t = lse_t;
+  a.lse_s = lse_s;
+  const bool nT = scale_T < 0.f, nS = scale_S < 0.f;
+  if (d_T == 128 && d_S == 128) return launch_fwd<128, 128>(maps, a, nT, nS, stream);
+  if (d_T == 128 && d_S == 64) return launch_fwd<128, 64>(maps, a, nT, nS, stream);
+  if (d_T == 64 && d_S == 128) return launch_fwd<64, 128>(maps, a, nT, nS, stream);
+  return launch_fwd<64, 64>(maps, a, nT, nS, stream);
+}
+
+// Shared body of the student and trainable-teacher backward entry points.
 template <bool TEACHER>
 streamkl_status bwd_common(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
-                           int B, int H, int N_Q, int N_K, int d_T, int d_S, float scale_T,
-                           float scale_S, int causal, const float* kl, const float* lse_t,
-                           const float* lse_s, const float* g, float* dq, float* dk,
-                           cudaStream_t stream) {
+                           int B, int H, int H_kv_T, int H_kv_S, int N_Q, int N_K, int d_T,
+                           int d_S, float scale_T, float scale_S, int causal, const float* kl,
+                           const float* lse_t, const float* lse_s, const float* g, float* dq,
+                           float* dk, cudaStream_t stream) {
   streamkl_status st = check_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S);
   if (st != STREAMKL_OK) return st;
   if (!lse_t || !lse_s || !g || !dq || !dk || (TEACHER && !kl)) return STREAMKL_ERR_INVALID_ARG;
+  int gT, gS;
+  if (!kv_groups(H, H_kv_T, H_kv_S, gT, gS)) return STREAMKL_ERR_UNSUPPORTED;
   if (!aligned16(lse_t) || !aligned16(lse_s) || !aligned16(g) || !aligned16(dq) ||
       !aligned16(dk) || (TEACHER && !aligned16(kl)))
     return STREAMKL_ERR_MISALIGNED;
   const int bh = B * H;
   const int d_g = TEACHER ? d_T : d_S;
-  CUtensorMap maps[5];
-  if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 64) || !make_map(&maps[1], k_t, d_T, N_K, bh, 128) ||
-      !make_map(&maps[2], q_s, d_S, N_Q, bh, 64) || !make_map(&maps[3], k_s, d_S, N_K, bh, 128) ||
-      !make_map_f32(&maps[4], dq, d_g, N_Q, bh))
+  const int g_g = TEACHER ? gT : gS;       // query heads per differentiated K head
+  const int bkv_g = B * (H / g_g);         // K heads of the differentiated side
+  CUtensorMap maps[6];
+  if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 64) ||
+      !make_map(&maps[1], k_t, d_T, N_K, B * H_kv_T, 128) ||
+      !make_map(&maps[2], q_s, d_S, N_Q, bh, 64) ||
+      !make_map(&maps[3], k_s, d_S, N_K, B * H_kv_S, 128) ||
+      !make_map_f32(&maps[4], dq, d_g, N_Q, bh) || !make_map_f32(&maps[5], dk, d_g, N_K, bkv_g))
     return STREAMKL_ERR_LAUNCH;
   if (cudaMemsetAsync(dq, 0, (size_t)bh * N_Q * d_g * sizeof(float), stream) != cudaSuccess)
+    return STREAMKL_ERR_LAUNCH;
+  if (g_g > 1 &&
+      cudaMemsetAsync(dk, 0, (size_t)bkv_g * N_K * d_g * sizeof(float), stream) != cudaSuccess)
     return STREAMKL_ERR_LAUNCH;
   skl::BwdArgs a{};
   a.BH = bh;
@@ -169,6 +226,10 @@ streamkl_status bwd_common(const void* q_t, const void* k_t, const void* q_s, co
   a.n_ktiles = (N_K + 127) / 128;
   a.n_qtiles = (N_Q + 63) / 64;
   a.group = head_group("STREAMKL_BWD_GROUP", 2, bh);
+  a.H = H;
+  a.gT = gT;
+  a.gS = gS;
+  a.dk_reduce = g_g > 1 ? 1 : 0;
   a.lse_t = lse_t;
   a.lse_s = lse_s;
   a.g = g;
@@ -190,41 +251,34 @@ streamkl_status streamkl_fwd(const void* q_t, const void* k_t, const void* q_s, 
                              int B, int H, int N_Q, int N_K, int d_T, int d_S, float scale_T,
                              float scale_S, int causal, float* kl, float* lse_t, float* lse_s,
                              cudaStream_t stream) {
-  streamkl_status st = check_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S);
-  if (st != STREAMKL_OK) return st;
-  if (!kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
-  if (!aligned16(kl) || !aligned16(lse_t) || !aligned16(lse_s)) return STREAMKL_ERR_MISALIGNED;
-  const int bh = B * H;
-  CUtensorMap maps[4];
-  if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 128) || !make_map(&maps[1], k_t, d_T, N_K, bh, 64) ||
-      !make_map(&maps[2], q_s, d_S, N_Q, bh, 128) || !make_map(&maps[3], k_s, d_S, N_K, bh, 64))
-    return STREAMKL_ERR_LAUNCH;
-  skl::FwdArgs a{};
-  a.BH = bh;
-  a.N_Q = N_Q;
-  a.N_K = N_K;
-  a.causal = causal ? 1 : 0;
-  a.off = N_K - N_Q;
-  a.cT = std::fabs(scale_T) * kLog2e;
-  a.cS = std::fabs(scale_S) * kLog2e;
-  a.n_ctas_per_bh = (N_Q + 255) / 256;
-  a.group = head_group("STREAMKL_FWD_GROUP", 4, bh);
-  a.kl = kl;
-  a.lse_t = lse_t;
-  a.lse_s = lse_s;
-  const bool nT = scale_T < 0.f, nS = scale_S < 0.f;
-  if (d_T == 128 && d_S == 128) return launch_fwd<128, 128>(maps, a, nT, nS, stream);
-  if (d_T == 128 && d_S == 64) return launch_fwd<128, 64>(maps, a, nT, nS, stream);
-  if (d_T == 64 && d_S == 128) return launch_fwd<64, 128>(maps, a, nT, nS, stream);
-  return launch_fwd<64, 64>(maps, a, nT, nS, stream);
+  return fwd_common(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_T, d_S, scale_T, scale_S, causal,
+                    kl, lse_t, lse_s, stream);
+}
+
+streamkl_status streamkl_fwd_gqa(const void* q_t, const void* k_t, const void* q_s,
+                                 const void* k_s, int B, int H, int H_kv_T, int H_kv_S, int N_Q,
+                                 int N_K, int d_T, int d_S, float scale_T, float scale_S,
+                                 int causal, float* kl, float* lse_t, float* lse_s,
+                                 cudaStream_t stream) {
+  return fwd_common(q_t, k_t, q_s, k_s, B, H, H_kv_T, H_kv_S, N_Q, N_K, d_T, d_S, scale_T,
+                    scale_S, causal, kl, lse_t, lse_s, stream);
 }
 
 streamkl_status streamkl_bwd(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
                              int B, int H, int N_Q, int N_K, int d_T, int d_S, float scale_T,
                              float scale_S, int causal, const float* lse_t, const float* lse_s,
                              const float* g, float* dq_s, float* dk_s, cudaStream_t stream) {
-  return bwd_common<false>(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S, causal,
-                           nullptr, lse_t, lse_s, g, dq_s, dk_s, stream);
+  return bwd_common<false>(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_T, d_S, scale_T, scale_S,
+                           causal, nullptr, lse_t, lse_s, g, dq_s, dk_s, stream);
+}
+
+streamkl_status streamkl_bwd_gqa(const void* q_t, const void* k_t, const void* q_s,
+                                 const void* k_s, int B, int H, int H_kv_T, int H_kv_S, int N_Q,
+                                 int N_K, int d_T, int d_S, float scale_T, float scale_S,
+                                 int causal, const float* lse_t, const float* lse_s,
+                                 const float* g, float* dq_s, float* dk_s, cudaStream_t stream) {
+  return bwd_common<false>(q_t, k_t, q_s, k_s, B, H, H_kv_T, H_kv_S, N_Q, N_K, d_T, d_S, scale_T,
+                           scale_S, causal, nullptr, lse_t, lse_s, g, dq_s, dk_s, stream);
 }
 
 streamkl_status streamkl_bwd_teacher(const void* q_t, const void* k_t, const void* q_s,
@@ -233,8 +287,18 @@ streamkl_status streamkl_bwd_teacher(const void* q_t, const void* k_t, const voi
                                      const float* kl, const float* lse_t, const float* lse_s,
                                      const float* g, float* dq_t, float* dk_t,
                                      cudaStream_t stream) {
-  return bwd_common<true>(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S, causal,
-                          kl, lse_t, lse_s, g, dq_t, dk_t, stream);
+  return bwd_common<true>(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_T, d_S, scale_T, scale_S,
+                          causal, kl, lse_t, lse_s, g, dq_t, dk_t, stream);
+}
+
+streamkl_status streamkl_bwd_teacher_gqa(const void* q_t, const void* k_t, const void* q_s,
+                                         const void* k_s, int B, int H, int H_kv_T, int H_kv_S,
+                                         int N_Q, int N_K, int d_T, int d_S, float scale_T,
+                                         float scale_S, int causal, const float* kl,
+                                         const float* lse_t, const float* lse_s, const float* g,
+                                         float* dq_t, float* dk_t, cudaStream_t stream) {
+  return bwd_common<true>(q_t, k_t, q_s, k_s, B, H, H_kv_T, H_kv_S, N_Q, N_K, d_T, d_S, scale_T,
+                          scale_S, causal, kl, lse_t, lse_s, g, dq_t, dk_t, stream);
 }
 
 const char* streamkl_status_string(streamkl_status s) {

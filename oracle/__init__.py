@@ -2,9 +2,12 @@
 from .streamkl_oracle import (  # noqa: F401
     allowed,
     oracle_bwd,
+    oracle_bwd_gqa,
     oracle_bwd_teacher,
+    oracle_bwd_teacher_gqa,
     oracle_dk_rows,
     oracle_fwd,
+    oracle_fwd_gqa,
     oracle_row_work,
     oracle_rows,
     row_pair_count,

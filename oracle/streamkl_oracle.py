@@ -276,3 +276,43 @@ def oracle_bwd_teacher(q_t, k_t, q_s, k_s, scale_t: float, scale_s: float, causa
                 dq[b, h, rows] = ds @ kt
                 dk[b, h] += ds.T @ qt
     return dq, dk
+
+
+# ------------------------------------------------ grouped-query attention (GQA)
+#
+# Query head h of H reads K head h // (H / H_kv) (teacher and student may group their
+# K heads differently). The KL of a query head is unchanged; the gradient of a shared K
+# head is the sum over the query heads of its group.
+
+def expand_kv(k, h_q: int):
+    """[B, H_kv, N, d] -> [B, H_q, N, d], query head h reading K head h // (H_q / H_kv)."""
+    return k.repeat_interleave(h_q // k.shape[1], dim=1)
+
+
+def group_sum_kv(dk, h_kv: int):
+    """[B, H_q, N, d] -> [B, H_kv, N, d]: sum over the query heads sharing a K head."""
+    B, H, N, d = dk.shape
+    return dk.reshape(B, h_kv, H // h_kv, N, d).sum(dim=2)
+
+
+def oracle_fwd_gqa(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, row_block: int = 1024):
+    H = q_t.shape[1]
+    return oracle_fwd(q_t, expand_kv(k_t, H), q_s, expand_kv(k_s, H), scale_t, scale_s, causal,
+                      row_block)
+
+
+def oracle_bwd_gqa(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g, row_block: int = 1024):
+    """dQ_S [B,H,N_Q,d_S], dK_S [B,H_kv_S,N_K,d_S] with grouped K heads."""
+    H = q_t.shape[1]
+    dq, dk = oracle_bwd(q_t, expand_kv(k_t, H), q_s, expand_kv(k_s, H), scale_t, scale_s,
+                        causal, g, row_block)
+    return dq, group_sum_kv(dk, k_s.shape[1])
+
+
+def oracle_bwd_teacher_gqa(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g,
+                           row_block: int = 1024):
+    """dQ_T [B,H,N_Q,d_T], dK_T [B,H_kv_T,N_K,d_T] with grouped K heads."""
+    H = q_t.shape[1]
+    dq, dk = oracle_bwd_teacher(q_t, expand_kv(k_t, H), q_s, expand_kv(k_s, H), scale_t,
+                                scale_s, causal, g, row_block)
+    return dq, group_sum_kv(dk, k_t.shape[1])

@@ -386,3 +386,73 @@ def test_teacher_grad_finite_differences_and_invariants():
     # identical teacher and student: zero gradient for the teacher as well
     dq0, dk0 = O.oracle_bwd_teacher(q_t, k_t, q_t, k_t, st, st, True, g)
     assert dq0.abs().max() < 1e-15 and dk0.abs().max() < 1e-15
+
+
+# ------------------------------------------------ grouped-query attention (GQA)
+
+def brute_force_gqa(q_t, k_t, q_s, k_s, st, ss, causal, g):
+    """Pure-Python loops with explicit K-head indices: query head h reads teacher K head
+    h // (H / H_kv_T) and student K head h // (H / H_kv_S); dK of a K head sums over the
+    query heads that read it."""
+    B, H, nq, dt = q_t.shape
+    hkt, hks = k_t.shape[1], k_s.shape[1]
+    nk, ds_ = k_t.shape[2], q_s.shape[3]
+    L = lambda t: t.double().tolist()
+    QT, KT, QS, KS, G = L(q_t), L(k_t), L(q_s), L(k_s), L(g)
+    kl = [[[0.0] * nq for _ in range(H)] for _ in range(B)]
+    dk = [[[[0.0] * ds_ for _ in range(nk)] for _ in range(hks)] for _ in range(B)]
+    for b in range(B):
+        for h in range(H):
+            ht, hs = h // (H // hkt), h // (H // hks)
+            for i in range(nq):
+                js = [j for j in range(nk) if (not causal) or j <= i + nk - nq]
+                if not js:
+                    continue
+                sT = {j: st * sum(QT[b][h][i][c] * KT[b][ht][j][c] for c in range(dt)) for j in js}
+                sS = {j: ss * sum(QS[b][h][i][c] * KS[b][hs][j][c] for c in range(ds_)) for j in js}
+                zT = sum(math.exp(v) for v in sT.values())
+                zS = sum(math.exp(v) for v in sS.values())
+                pT = {j: math.exp(sT[j]) / zT for j in js}
+                pS = {j: math.exp(sS[j]) / zS for j in js}
+                kl[b][h][i] = sum(pT[j] * math.log(pT[j] / pS[j]) for j in js)
+                for j in js:
+                    dsij = G[b][h][i] * ss * (pS[j] - pT[j])
+                    for c in range(ds_):
+                        dk[b][hs][j][c] += dsij * QS[b][h][i][c]
+    return torch.tensor(kl, dtype=F64), torch.tensor(dk, dtype=F64)
+
+
+@pytest.mark.parametrize("hkt,hks", [(2, 1), (1, 2), (4, 4), (4, 2)])
+def test_gqa_against_brute_force(hkt, hks):
+    g = torch.Generator().manual_seed(7 * hkt + hks)
+    mk = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16)
+    q_t, k_t = mk(1, 4, 5, 3), mk(1, hkt, 6, 3)
+    q_s, k_s = mk(1, 4, 5, 2), mk(1, hks, 6, 2)
+    gg = torch.rand(1, 4, 5, generator=g) + 0.5
+    kl_r, dk_r = brute_force_gqa(q_t, k_t, q_s, k_s, 0.8, 1.2, True, gg)
+    kl, _, _ = O.oracle_fwd_gqa(q_t, k_t, q_s, k_s, 0.8, 1.2, True)
+    dq, dk = O.oracle_bwd_gqa(q_t, k_t, q_s, k_s, 0.8, 1.2, True, gg)
+    torch.testing.assert_close(kl, kl_r, rtol=1e-12, atol=1e-13)
+    torch.testing.assert_close(dk, dk_r, rtol=1e-11, atol=1e-13)
+    assert dq.shape == q_s.shape and dk.shape == k_s.shape
+
+
+def test_gqa_shared_key_finite_differences():
+    """Both query heads of a group move with a shared K entry: dK sums their parts."""
+    g = torch.Generator().manual_seed(3)
+    q_t, k_t = torch.randn(1, 4, 5, 3, generator=g, dtype=F64), torch.randn(1, 4, 6, 3, generator=g, dtype=F64)
+    q_s, k_s = torch.randn(1, 4, 5, 3, generator=g, dtype=F64), torch.randn(1, 2, 6, 3, generator=g, dtype=F64)
+    gg = torch.rand(1, 4, 5, generator=g, dtype=F64)
+    dq, dk = O.oracle_bwd_gqa(q_t, k_t, q_s, k_s, 0.5, 0.9, False, gg)
+    dqt, dkt = O.oracle_bwd_teacher_gqa(q_t, k_t[:, :1], q_s, k_s, 0.5, 0.9, False, gg)
+    loss = lambda kt, ks: float((O.oracle_fwd_gqa(q_t, kt, q_s, ks, 0.5, 0.9, False)[0] * gg).sum())
+    h = 1e-6
+    for (hk, j, c) in [(0, 1, 0), (1, 5, 2)]:
+        e = torch.zeros_like(k_s); e[0, hk, j, c] = h
+        fd = (loss(k_t, k_s + e) - loss(k_t, k_s - e)) / (2 * h)
+        assert abs(fd - dk[0, hk, j, c].item()) <= 1e-6 * max(1.0, abs(fd))
+    kt1 = k_t[:, :1]
+    for (j, c) in [(0, 2), (4, 1)]:
+        e = torch.zeros_like(kt1); e[0, 0, j, c] = h
+        fd = (loss(kt1 + e, k_s) - loss(kt1 - e, k_s)) / (2 * h)
+        assert abs(fd - dkt[0, 0, j, c].item()) <= 1e-6 * max(1.0, abs(fd))
