@@ -22,7 +22,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "lib", "libstreamkl.so")
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "MISALIGNED", 4: "LAUNCH", 5: "TIMEOUT"}
-EXPORTS = ("streamkl_fwd", "streamkl_bwd", "streamkl_bwd_teacher", "streamkl_status_string",
+EXPORTS = ("streamkl_fwd", "streamkl_bwd", "streamkl_bwd_teacher", "streamkl_fwd_gqa",
+           "streamkl_bwd_gqa", "streamkl_bwd_teacher_gqa", "streamkl_status_string",
            "streamkl_device_status", "streamkl_version")
 
 
@@ -52,6 +53,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.streamkl_bwd_teacher.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, f, i, vp, vp, vp,
                                          vp, vp, vp, vp]
     lib.streamkl_bwd_teacher.restype = i
+    lib.streamkl_fwd_gqa.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, f, i, vp, vp, vp,
+                                     vp]
+    lib.streamkl_fwd_gqa.restype = i
+    lib.streamkl_bwd_gqa.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, f, i, vp, vp, vp,
+                                     vp, vp, vp]
+    lib.streamkl_bwd_gqa.restype = i
+    lib.streamkl_bwd_teacher_gqa.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, f, i, vp,
+                                             vp, vp, vp, vp, vp, vp]
+    lib.streamkl_bwd_teacher_gqa.restype = i
     lib.streamkl_status_string.argtypes = [i]
     lib.streamkl_status_string.restype = ctypes.c_char_p
     lib.streamkl_device_status.argtypes = [vp]
@@ -171,6 +181,71 @@ def streamkl_bwd_teacher(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, cau
                                   g.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(),
                                   _stream_ptr(stream))
     _check(st, "streamkl_bwd_teacher")
+    return dq_t, dk_t
+
+
+def _shape_gqa(q_t, k_t, q_s, k_s):
+    """Shapes with grouped K heads: k_t [B,H_kv_T,N_K,d_T], k_s [B,H_kv_S,N_K,d_S]."""
+    import torch
+    for name, t in (("q_t", q_t), ("k_t", k_t), ("q_s", q_s), ("k_s", k_s)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor [B,H,N,d]")
+    B, H, n_q, d_t = q_t.shape
+    h_kt, n_k = k_t.shape[1], k_t.shape[2]
+    h_ks, d_s = k_s.shape[1], q_s.shape[3]
+    if tuple(k_t.shape) != (B, h_kt, n_k, d_t) or tuple(q_s.shape) != (B, H, n_q, d_s) or \
+            tuple(k_s.shape) != (B, h_ks, n_k, d_s):
+        raise ValueError("inconsistent shapes")
+    return B, H, h_kt, h_ks, n_q, n_k, d_t, d_s
+
+
+def streamkl_fwd_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
+                     kl=None, lse_t=None, lse_s=None, stream=None):
+    """streamkl_fwd with grouped K heads (k_* may have fewer heads than q_*)."""
+    import torch
+    B, H, h_kt, h_ks, n_q, n_k, d_t, d_s = _shape_gqa(q_t, k_t, q_s, k_s)
+    dev = q_t.device
+    kl = torch.empty(B, H, n_q, device=dev, dtype=torch.float32) if kl is None else kl
+    lse_t = torch.empty_like(kl) if lse_t is None else lse_t
+    lse_s = torch.empty_like(kl) if lse_s is None else lse_s
+    st = load_library().streamkl_fwd_gqa(
+        q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), B, H, h_kt, h_ks, n_q,
+        n_k, d_t, d_s, float(scale_T), float(scale_S), int(bool(causal)), kl.data_ptr(),
+        lse_t.data_ptr(), lse_s.data_ptr(), _stream_ptr(stream))
+    _check(st, "streamkl_fwd_gqa")
+    return kl, lse_t, lse_s
+
+
+def streamkl_bwd_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
+                     lse_t, lse_s, g, dq_s=None, dk_s=None, stream=None):
+    """streamkl_bwd with grouped K heads; dk_s has the student's K-head count."""
+    import torch
+    B, H, h_kt, h_ks, n_q, n_k, d_t, d_s = _shape_gqa(q_t, k_t, q_s, k_s)
+    dev = q_t.device
+    dq_s = torch.empty(B, H, n_q, d_s, device=dev, dtype=torch.float32) if dq_s is None else dq_s
+    dk_s = torch.empty(B, h_ks, n_k, d_s, device=dev, dtype=torch.float32) if dk_s is None else dk_s
+    st = load_library().streamkl_bwd_gqa(
+        q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), B, H, h_kt, h_ks, n_q,
+        n_k, d_t, d_s, float(scale_T), float(scale_S), int(bool(causal)), lse_t.data_ptr(),
+        lse_s.data_ptr(), g.data_ptr(), dq_s.data_ptr(), dk_s.data_ptr(), _stream_ptr(stream))
+    _check(st, "streamkl_bwd_gqa")
+    return dq_s, dk_s
+
+
+def streamkl_bwd_teacher_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
+                             kl, lse_t, lse_s, g, dq_t=None, dk_t=None, stream=None):
+    """streamkl_bwd_teacher with grouped K heads; dk_t has the teacher's K-head count."""
+    import torch
+    B, H, h_kt, h_ks, n_q, n_k, d_t, d_s = _shape_gqa(q_t, k_t, q_s, k_s)
+    dev = q_t.device
+    dq_t = torch.empty(B, H, n_q, d_t, device=dev, dtype=torch.float32) if dq_t is None else dq_t
+    dk_t = torch.empty(B, h_kt, n_k, d_t, device=dev, dtype=torch.float32) if dk_t is None else dk_t
+    st = load_library().streamkl_bwd_teacher_gqa(
+        q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), B, H, h_kt, h_ks, n_q,
+        n_k, d_t, d_s, float(scale_T), float(scale_S), int(bool(causal)), kl.data_ptr(),
+        lse_t.data_ptr(), lse_s.data_ptr(), g.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(),
+        _stream_ptr(stream))
+    _check(st, "streamkl_bwd_teacher_gqa")
     return dq_t, dk_t
 
 

@@ -16,7 +16,8 @@ from typing import Optional
 
 import torch
 
-from . import streamkl_bwd, streamkl_bwd_teacher, streamkl_fwd
+from . import (streamkl_bwd, streamkl_bwd_gqa, streamkl_bwd_teacher, streamkl_bwd_teacher_gqa,
+               streamkl_fwd, streamkl_fwd_gqa)
 
 REDUCTIONS = ("none", "sum", "mean", "batchmean")
 
@@ -25,32 +26,35 @@ class StreamKLFunction(torch.autograd.Function):
     """Row-wise KL(P_T || P_S) of two attention maps.
 
     Gradients flow to Q_S and K_S (streamkl_bwd) and, when the teacher inputs require
-    grad, to Q_T and K_T as well (streamkl_bwd_teacher).
+    grad, to Q_T and K_T as well (streamkl_bwd_teacher). K tensors with fewer heads than
+    the queries select the grouped-query (GQA) entry points.
     """
 
     @staticmethod
     def forward(ctx, q_t, k_t, q_s, k_s, scale_t: float, scale_s: float, causal: bool):
-        kl, lse_t, lse_s = streamkl_fwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal)
+        gqa = k_t.shape[1] != q_t.shape[1] or k_s.shape[1] != q_s.shape[1]
+        fwd = streamkl_fwd_gqa if gqa else streamkl_fwd
+        kl, lse_t, lse_s = fwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal)
         ctx.save_for_backward(q_t, k_t, q_s, k_s, kl, lse_t, lse_s)
-        ctx.params = (scale_t, scale_s, causal)
+        ctx.params = (scale_t, scale_s, causal, gqa)
         ctx.mark_non_differentiable(lse_t, lse_s)
         return kl, lse_t, lse_s
 
     @staticmethod
     def backward(ctx, g_kl, _g_lse_t=None, _g_lse_s=None):
         q_t, k_t, q_s, k_s, kl, lse_t, lse_s = ctx.saved_tensors
-        scale_t, scale_s, causal = ctx.params
+        scale_t, scale_s, causal, gqa = ctx.params
         g = g_kl.detach().to(torch.float32).contiguous()
         need_t = ctx.needs_input_grad[0] or ctx.needs_input_grad[1]
         need_s = ctx.needs_input_grad[2] or ctx.needs_input_grad[3]
         dq_t = dk_t = dq_s = dk_s = None
         if need_s:
-            dq_s, dk_s = streamkl_bwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, lse_t,
-                                      lse_s, g)
+            bwd = streamkl_bwd_gqa if gqa else streamkl_bwd
+            dq_s, dk_s = bwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, lse_t, lse_s, g)
             dq_s, dk_s = dq_s.to(q_s.dtype), dk_s.to(k_s.dtype)
         if need_t:
-            dq_t, dk_t = streamkl_bwd_teacher(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, kl,
-                                              lse_t, lse_s, g)
+            bwd_t = streamkl_bwd_teacher_gqa if gqa else streamkl_bwd_teacher
+            dq_t, dk_t = bwd_t(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, kl, lse_t, lse_s, g)
             dq_t, dk_t = dq_t.to(q_t.dtype), dk_t.to(k_t.dtype)
         return dq_t, dk_t, dq_s, dk_s, None, None, None
 

@@ -26,7 +26,7 @@
  * - Layout: q_t [B,H,N_Q,d_T], k_t [B,H,N_K,d_T], q_s [B,H,N_Q,d_S], k_s [B,H,N_K,d_S],
  *   contiguous row-major bf16 (d innermost). Row statistics and g are contiguous fp32
  *   [B,H,N_Q]. Gradients are contiguous fp32.
- * - Supported: d_T, d_S in {64, 128}; B, H, N_Q, N_K >= 1; B*H*max(N_Q,N_K) < 2^31;
+ * - Supported: d_T, d_S in {64, 128}; B, H, N_Q, N_K >= 1; B*H*max(N_Q,N_K) < 2^31, B*H < 2^24;
  *   any finite scale_T, scale_S. N_Q and N_K need not be multiples of any tile size.
  * - Every input/output pointer must be 16-byte aligned.
  * - Calls are asynchronous on `stream`: argument checks happen on the host before any
@@ -106,6 +106,37 @@ streamkl_status streamkl_bwd_teacher(const void* q_t, const void* k_t, const voi
                                      const float* kl, const float* lse_t, const float* lse_s,
                                      const float* g, float* dq_t, float* dk_t,
                                      cudaStream_t stream);
+
+/*
+ * Grouped-query attention variants (several query heads share one K head; teacher and
+ * student may group differently). Same operations and conventions as above, with
+ *   k_t [B,H_kv_T,N_K,d_T], k_s [B,H_kv_S,N_K,d_S]; query head h reads teacher K head
+ *   h / (H / H_kv_T) and student K head h / (H / H_kv_S); H_kv_T and H_kv_S must divide H
+ *   (else STREAMKL_ERR_UNSUPPORTED).
+ * Gradients of a shared K head are summed over the query heads of its group:
+ *   dk_s [B,H_kv_S,N_K,d_S] (streamkl_bwd_gqa), dk_t [B,H_kv_T,N_K,d_T]
+ *   (streamkl_bwd_teacher_gqa); when a group has more than one query head, dk is zeroed on
+ *   `stream` and accumulated with fp32 reductions in L2 (low bits can vary between runs).
+ * The entry points without the suffix are these with H_kv_T = H_kv_S = H.
+ */
+streamkl_status streamkl_fwd_gqa(const void* q_t, const void* k_t, const void* q_s,
+                                 const void* k_s, int B, int H, int H_kv_T, int H_kv_S, int N_Q,
+                                 int N_K, int d_T, int d_S, float scale_T, float scale_S,
+                                 int causal, float* kl, float* lse_t, float* lse_s,
+                                 cudaStream_t stream);
+
+streamkl_status streamkl_bwd_gqa(const void* q_t, const void* k_t, const void* q_s,
+                                 const void* k_s, int B, int H, int H_kv_T, int H_kv_S, int N_Q,
+                                 int N_K, int d_T, int d_S, float scale_T, float scale_S,
+                                 int causal, const float* lse_t, const float* lse_s,
+                                 const float* g, float* dq_s, float* dk_s, cudaStream_t stream);
+
+streamkl_status streamkl_bwd_teacher_gqa(const void* q_t, const void* k_t, const void* q_s,
+                                         const void* k_s, int B, int H, int H_kv_T, int H_kv_S,
+                                         int N_Q, int N_K, int d_T, int d_S, float scale_T,
+                                         float scale_S, int causal, const float* kl,
+                                         const float* lse_t, const float* lse_s, const float* g,
+                                         float* dq_t, float* dk_t, cudaStream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char* streamkl_status_string(streamkl_status status);

@@ -92,6 +92,21 @@ def test_host_validation(lib, fn):
     assert fn(k_s=P + 2) == 3
 
 
+def test_gqa_head_groups_validated(lib):
+    def fwd_gqa(H, hkt, hks):
+        return lib.streamkl_fwd_gqa(P, P, P, P, 1, H, hkt, hks, 128, 128, 128, 128, 0.1, 0.1, 0,
+                                    P, P, P, 0)
+    assert fwd_gqa(8, 3, 8) == 2     # 3 does not divide 8
+    assert fwd_gqa(8, 8, 0) == 2     # no K heads
+    assert fwd_gqa(8, 4, 16) == 2    # more K heads than query heads
+    assert lib.streamkl_bwd_gqa(P, P, P, P, 1, 6, 4, 2, 128, 128, 128, 128, 0.1, 0.1, 0,
+                                P, P, P, P, P, 0) == 2
+    assert lib.streamkl_bwd_teacher_gqa(P, P, P, P, 1, 6, 3, 5, 128, 128, 128, 128, 0.1, 0.1,
+                                        0, P, P, P, P, P, P, 0) == 2
+    assert lib.streamkl_fwd_gqa(0, P, P, P, 1, 8, 4, 2, 128, 128, 128, 128, 0.1, 0.1, 0,
+                                P, P, P, 0) == 1
+
+
 def test_host_validation_outputs(lib):
     assert fwd(kl=0) == 1
     assert fwd(lse_s=P + 4) == 3

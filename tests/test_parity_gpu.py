@@ -14,7 +14,8 @@ import pytest
 import torch
 
 import attention_kl_divergence_fwd_b200 as skl
-from oracle import oracle_bwd, oracle_bwd_teacher, oracle_dk_rows, oracle_fwd, oracle_rows
+from oracle import (oracle_bwd, oracle_bwd_gqa, oracle_bwd_teacher, oracle_bwd_teacher_gqa,
+                    oracle_dk_rows, oracle_fwd, oracle_fwd_gqa, oracle_rows)
 from workloads import WORKLOADS, WORKLOAD_LIST, make_inputs, sample_keys, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -190,6 +191,54 @@ def test_teacher_grads_identical_inputs_zero():
     dq, dk = skl.streamkl_bwd_teacher(*a, kl, lt, ls, d["g"])
     assert skl.device_status() == 0
     assert dq.abs().max().item() == 0 and dk.abs().max().item() == 0
+
+
+# ------------------------------------------------ grouped-query attention (GQA)
+
+@pytest.mark.parametrize("H,hkt,hks,nq,nk,dt,ds,causal", [
+    (4, 2, 1, 300, 300, 128, 128, True),
+    (4, 4, 2, 333, 517, 128, 64, False),
+    (6, 3, 2, 517, 333, 64, 128, True),
+    (8, 1, 8, 200, 260, 64, 64, True),
+])
+def test_gqa_full(H, hkt, hks, nq, nk, dt, ds, causal):
+    gen = torch.Generator().manual_seed(H * 100 + hkt * 10 + hks)
+    mk = lambda *s: torch.randn(*s, generator=gen).to(torch.bfloat16)
+    x = {"q_t": mk(1, H, nq, dt), "k_t": mk(1, hkt, nk, dt), "q_s": mk(1, H, nq, ds),
+         "k_s": mk(1, hks, nk, ds), "g": torch.rand(1, H, nq, generator=gen)}
+    st, ss = 1 / math.sqrt(dt), 1 / math.sqrt(ds)
+    d = to_dev(x)
+    a = (d["q_t"], d["k_t"], d["q_s"], d["k_s"], st, ss, causal)
+    kl, lt, ls = skl.streamkl_fwd_gqa(*a)
+    dq, dk = skl.streamkl_bwd_gqa(*a, lt, ls, d["g"])
+    dqt, dkt = skl.streamkl_bwd_teacher_gqa(*a, kl, lt, ls, d["g"])
+    assert skl.device_status() == 0
+    r = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], st, ss, causal)
+    kl_r, lt_r, ls_r = oracle_fwd_gqa(*r)
+    check_kl(kl.cpu().double(), kl_r)
+    check_lse(lt.cpu().double(), lt_r)
+    check_lse(ls.cpu().double(), ls_r)
+    dq_r, dk_r = oracle_bwd_gqa(*r, x["g"])
+    assert dk.shape == x["k_s"].shape
+    assert rel_fro(dq.cpu().double(), dq_r) <= GRAD_REL
+    assert rel_fro(dk.cpu().double(), dk_r) <= GRAD_REL
+    dqt_r, dkt_r = oracle_bwd_teacher_gqa(*r, x["g"])
+    assert dkt.shape == x["k_t"].shape
+    assert rel_fro(dqt.cpu().double(), dqt_r) <= GRAD_REL
+    assert rel_fro(dkt.cpu().double(), dkt_r) <= GRAD_REL
+
+
+def test_gqa_with_one_group_equals_mha():
+    w = BASE.with_sizes(B=2, H=2, N_Q=300, N_K=300)
+    d = to_dev(make_inputs(w, seed=12))
+    a = (d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal)
+    kl, lt, ls = skl.streamkl_fwd(*a)
+    kl2, lt2, ls2 = skl.streamkl_fwd_gqa(*a)
+    dq, dk = skl.streamkl_bwd(*a, lt, ls, d["g"])
+    dq2, dk2 = skl.streamkl_bwd_gqa(*a, lt, ls, d["g"])
+    assert skl.device_status() == 0
+    assert torch.equal(kl, kl2) and torch.equal(lt, lt2) and torch.equal(dk, dk2)
+    assert rel_fro(dq2.double(), dq.double()) < 1e-5
 
 
 # ----------------------------------------------------------- full-size workloads
