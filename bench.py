@@ -309,6 +309,32 @@ def main():
     bwd_t_ms = max_over_ranks(te0.elapsed_time(te1) / args.steps, world)
     del dq_t, dk_t
 
+    # Grouped-query variant of the same workload (student K heads shared by 4 query heads),
+    # timed on its own and reported beside the step.
+    gqa = None
+    if w.H % 4 == 0:
+        k_s4 = d["k_s"][:, : w.H // 4].contiguous()
+        dk4 = torch.empty(B, w.H // 4, nk, w.d_S, device=dev)
+        ga = (d["q_t"], d["k_t"], d["q_s"], k_s4, w.scale_T, w.scale_S, w.causal)
+        for _ in range(2):
+            skl.streamkl_fwd_gqa(*ga, kl=kl, lse_t=lt, lse_s=ls)
+            skl.streamkl_bwd_gqa(*ga, lt, ls, d["g"], dq_s=dq, dk_s=dk4)
+        torch.cuda.synchronize()
+        ge = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ge[0].record(stream)
+        for _ in range(args.steps):
+            skl.streamkl_fwd_gqa(*ga, kl=kl, lse_t=lt, lse_s=ls)
+        ge[1].record(stream)
+        for _ in range(args.steps):
+            skl.streamkl_bwd_gqa(*ga, lt, ls, d["g"], dq_s=dq, dk_s=dk4)
+        ge[2].record(stream)
+        torch.cuda.synchronize()
+        gf = max_over_ranks(ge[0].elapsed_time(ge[1]) / args.steps, world)
+        gb = max_over_ranks(ge[1].elapsed_time(ge[2]) / args.steps, world)
+        gqa = {"student_kv_heads": w.H // 4, "fwd_ms": gf, "bwd_ms": gb,
+               "fwd_tflops": ff / (gf * 1e-3) / 1e12, "bwd_tflops": fb / (gb * 1e-3) / 1e12}
+        del k_s4, dk4
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(skl, w, x, dev, stream, args.steps, world)
@@ -327,6 +353,7 @@ def main():
                "fwd_frac_burst_peak": fwd_tf / peak_burst,
                "bwd_frac_burst_peak": bwd_tf / peak_burst,
                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+               "gqa": gqa,
                "bwd_teacher_ms": bwd_t_ms,
                "bwd_teacher_tflops": flops_bwd_teacher(w) / (bwd_t_ms * 1e-3) / 1e12,
                "gpu_launches": 2 * args.steps,

@@ -28,7 +28,7 @@ Backward (teacher frozen; g[i] = dLoss/dKL[i]):
     dS[i, j]  = g[i] * scale_S * (P_S[i, j] - P_T[i, j])   (gradient w.r.t. <q_S[i], k_S[j]>)
     dQ_S      = dS @ K_S            dK_S = dS^T @ Q_S
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent (the plainest reading the rest supports):
 * causal alignment for N_Q != N_K is bottom-right (j <= i + N_K - N_Q);
 * a row with an empty J(i) has KL = 0, LSE = -inf and zero gradient;
 * KL is reported raw (no clamp at 0); LSE is the natural-log value.
@@ -316,3 +316,75 @@ def oracle_bwd_teacher_gqa(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g,
     dq, dk = oracle_bwd_teacher(q_t, expand_kv(k_t, H), q_s, expand_kv(k_s, H), scale_t,
                                 scale_s, causal, g, row_block)
     return dq, group_sum_kv(dk, k_t.shape[1])
+
+
+# ------------------------------------------------ packed variable-length sequences
+#
+# B sequences of different lengths share one packed tensor: sequence b owns query rows
+# cu_q[b] .. cu_q[b+1]-1 and key rows cu_k[b] .. cu_k[b+1]-1 (token-major, [total, heads,
+# d]). Each sequence is an independent problem with its own causal alignment (bottom-right
+# within the sequence: j <= i + n_k(b) - n_q(b)); no query attends to another sequence's
+# keys. Row outputs and g are [H, total_q]. Query heads read K heads as in GQA.
+
+def _seq_bounds(cu):
+    cu = [int(c) for c in cu]
+    if len(cu) < 2 or cu[0] != 0 or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("cu_seqlens must start at 0 and be non-decreasing")
+    return list(zip(cu[:-1], cu[1:]))
+
+
+def _seq_heads_first(x, lo, hi):
+    """Rows lo..hi-1 of a packed [total, heads, d] tensor as a [1, heads, n, d] problem."""
+    return x[lo:hi].permute(1, 0, 2).unsqueeze(0)
+
+
+def oracle_fwd_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, scale_t, scale_s, causal,
+                      row_block: int = 1024):
+    """KL, LSE_T, LSE_S as float64 [H, total_q] for packed sequences."""
+    H, total_q = q_t.shape[1], q_t.shape[0]
+    kl = torch.zeros(H, total_q, dtype=F64)
+    lse_t = torch.full((H, total_q), NEG_INF, dtype=F64)
+    lse_s = torch.full((H, total_q), NEG_INF, dtype=F64)
+    seq_q, seq_k = _seq_bounds(cu_q), _seq_bounds(cu_k)
+    if len(seq_q) != len(seq_k):
+        raise ValueError("cu_q and cu_k must describe the same number of sequences")
+    for (q0, q1), (k0, k1) in zip(seq_q, seq_k):
+        if q1 == q0 or k1 == k0:
+            continue  # no rows, or rows with no keys: KL 0, LSE -inf (already set)
+        out = oracle_fwd_gqa(_seq_heads_first(q_t, q0, q1), _seq_heads_first(k_t, k0, k1),
+                             _seq_heads_first(q_s, q0, q1), _seq_heads_first(k_s, k0, k1),
+                             scale_t, scale_s, causal, row_block)
+        for dst, src in zip((kl, lse_t, lse_s), out):
+            dst[:, q0:q1] = src[0]
+    return kl, lse_t, lse_s
+
+
+def _bwd_varlen(fn, q_t, k_t, q_s, k_s, cu_q, cu_k, scale_t, scale_s, causal, g, side,
+                row_block):
+    q_g, k_g = (q_t, k_t) if side == "teacher" else (q_s, k_s)
+    dq = torch.zeros(q_g.shape, dtype=F64)
+    dk = torch.zeros(k_g.shape, dtype=F64)
+    for (q0, q1), (k0, k1) in zip(_seq_bounds(cu_q), _seq_bounds(cu_k)):
+        if q1 == q0 or k1 == k0:
+            continue
+        gb = g[:, q0:q1].unsqueeze(0)
+        dq_b, dk_b = fn(_seq_heads_first(q_t, q0, q1), _seq_heads_first(k_t, k0, k1),
+                        _seq_heads_first(q_s, q0, q1), _seq_heads_first(k_s, k0, k1),
+                        scale_t, scale_s, causal, gb, row_block)
+        dq[q0:q1] = dq_b[0].permute(1, 0, 2)
+        dk[k0:k1] = dk_b[0].permute(1, 0, 2)
+    return dq, dk
+
+
+def oracle_bwd_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, scale_t, scale_s, causal, g,
+                      row_block: int = 1024):
+    """dQ_S [total_q, H, d_S], dK_S [total_k, H_kv_S, d_S] (float64); g is [H, total_q]."""
+    return _bwd_varlen(oracle_bwd_gqa, q_t, k_t, q_s, k_s, cu_q, cu_k, scale_t, scale_s,
+                       causal, g, "student", row_block)
+
+
+def oracle_bwd_teacher_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, scale_t, scale_s, causal, g,
+                              row_block: int = 1024):
+    """dQ_T [total_q, H, d_T], dK_T [total_k, H_kv_T, d_T] (float64); g is [H, total_q]."""
+    return _bwd_varlen(oracle_bwd_teacher_gqa, q_t, k_t, q_s, k_s, cu_q, cu_k, scale_t,
+                       scale_s, causal, g, "teacher", row_block)

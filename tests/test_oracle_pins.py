@@ -456,3 +456,133 @@ def test_gqa_shared_key_finite_differences():
         e = torch.zeros_like(kt1); e[0, 0, j, c] = h
         fd = (loss(kt1 + e, k_s) - loss(kt1 - e, k_s)) / (2 * h)
         assert abs(fd - dkt[0, 0, j, c].item()) <= 1e-6 * max(1.0, abs(fd))
+
+
+# ------------------------------------------------ packed variable-length sequences
+
+def brute_force_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, st, ss, causal, g):
+    """Pure-Python loops over packed [total, heads, d] rows with explicit token indices.
+
+    Query token i of sequence b (rows cu_q[b] <= i < cu_q[b+1]) sees key token j of the
+    same sequence iff not causal or (j - cu_k[b]) <= (i - cu_q[b]) + n_k(b) - n_q(b).
+    Returns KL and LSE_T as [H, total_q], dQ_S [total_q, H, d_S], dK_S [total_k, H_kv_S, d_S].
+    """
+    tq, H, dt = q_t.shape
+    tk, hkt, _ = k_t.shape
+    hks, ds_ = k_s.shape[1], k_s.shape[2]
+    L = lambda t: t.double().tolist()
+    QT, KT, QS, KS, G = L(q_t), L(k_t), L(q_s), L(k_s), L(g)
+    kl = [[0.0] * tq for _ in range(H)]
+    lt = [[float("-inf")] * tq for _ in range(H)]
+    dq = [[[0.0] * ds_ for _ in range(H)] for _ in range(tq)]
+    dk = [[[0.0] * ds_ for _ in range(hks)] for _ in range(tk)]
+    for b in range(len(cu_q) - 1):
+        nq, nk = cu_q[b + 1] - cu_q[b], cu_k[b + 1] - cu_k[b]
+        for h in range(H):
+            ht, hs = h // (H // hkt), h // (H // hks)
+            for i in range(cu_q[b], cu_q[b + 1]):
+                js = [j for j in range(cu_k[b], cu_k[b + 1])
+                      if (not causal) or (j - cu_k[b]) <= (i - cu_q[b]) + nk - nq]
+                if not js:
+                    continue
+                sT = {j: st * sum(QT[i][h][c] * KT[j][ht][c] for c in range(dt)) for j in js}
+                sS = {j: ss * sum(QS[i][h][c] * KS[j][hs][c] for c in range(ds_)) for j in js}
+                zT = sum(math.exp(v) for v in sT.values())
+                zS = sum(math.exp(v) for v in sS.values())
+                pT = {j: math.exp(sT[j]) / zT for j in js}
+                pS = {j: math.exp(sS[j]) / zS for j in js}
+                kl[h][i] = sum(pT[j] * math.log(pT[j] / pS[j]) for j in js)
+                lt[h][i] = math.log(zT)
+                for j in js:
+                    dsij = G[h][i] * ss * (pS[j] - pT[j])
+                    for c in range(ds_):
+                        dq[i][h][c] += dsij * KS[j][hs][c]
+                        dk[j][hs][c] += dsij * QS[i][h][c]
+    T = lambda x: torch.tensor(x, dtype=F64)
+    return T(kl), T(lt), T(dq), T(dk)
+
+
+def varlen_case(lq, lk, H, hkt, hks, dt, ds, seed):
+    g = torch.Generator().manual_seed(seed)
+    mk = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16)
+    tq, tk = sum(lq), sum(lk)
+    cu_q = [0] + list(torch.tensor(lq).cumsum(0).tolist())
+    cu_k = [0] + list(torch.tensor(lk).cumsum(0).tolist())
+    return (mk(tq, H, dt), mk(tk, hkt, dt), mk(tq, H, ds), mk(tk, hks, ds), cu_q, cu_k,
+            torch.rand(H, tq, generator=g) + 0.5)
+
+
+# sequences with: equal lengths, n_q > n_k (empty causal rows), n_q < n_k, no queries,
+# no keys, a single token
+VARLEN_LENS = [([3, 5, 0, 4, 1, 2], [3, 2, 4, 6, 1, 0])]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("hkt,hks", [(2, 2), (1, 2)])
+def test_varlen_against_brute_force(causal, hkt, hks):
+    lq, lk = VARLEN_LENS[0]
+    q_t, k_t, q_s, k_s, cu_q, cu_k, gg = varlen_case(lq, lk, 2, hkt, hks, 3, 2, 11 + hkt)
+    kl_r, lt_r, dq_r, dk_r = brute_force_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, 0.7, 1.1,
+                                                causal, gg)
+    kl, lt, _ = O.oracle_fwd_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, 0.7, 1.1, causal)
+    dq, dk = O.oracle_bwd_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, 0.7, 1.1, causal, gg)
+    torch.testing.assert_close(kl, kl_r, rtol=1e-12, atol=1e-13)
+    torch.testing.assert_close(lt, lt_r, rtol=1e-12, atol=1e-13)
+    torch.testing.assert_close(dq, dq_r, rtol=1e-11, atol=1e-13)
+    torch.testing.assert_close(dk, dk_r, rtol=1e-11, atol=1e-13)
+    assert dq.shape == q_s.shape and dk.shape == k_s.shape
+
+
+def test_varlen_sequences_are_independent_and_match_padded_runs():
+    """A sequence's outputs equal those of the same tokens run alone in the [B, H, N, d]
+    layout, and do not move when another sequence's tokens change."""
+    lq, lk = [4, 6], [5, 6]
+    q_t, k_t, q_s, k_s, cu_q, cu_k, gg = varlen_case(lq, lk, 2, 2, 2, 3, 3, 5)
+    kl, _, _ = O.oracle_fwd_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, 0.9, 0.6, True)
+    alone = lambda x, lo, hi: x[lo:hi].permute(1, 0, 2).unsqueeze(0)
+    kl1, _, _ = O.oracle_fwd(alone(q_t, 4, 10), alone(k_t, 5, 11), alone(q_s, 4, 10),
+                             alone(k_s, 5, 11), 0.9, 0.6, True)
+    torch.testing.assert_close(kl[:, 4:10], kl1[0], rtol=0, atol=0)
+    k_s2 = k_s.clone()
+    k_s2[:5] = torch.randn(5, 2, 3).to(torch.bfloat16)
+    kl2, _, _ = O.oracle_fwd_varlen(q_t, k_t, q_s, k_s2, cu_q, cu_k, 0.9, 0.6, True)
+    assert torch.equal(kl2[:, 4:], kl[:, 4:]) and not torch.equal(kl2[:, :4], kl[:, :4])
+
+
+def test_varlen_teacher_finite_differences():
+    lq, lk = [3, 4], [5, 4]
+    g = torch.Generator().manual_seed(9)
+    mk = lambda *s: torch.randn(*s, generator=g, dtype=F64)
+    q_t, k_t, q_s, k_s = mk(7, 2, 3), mk(9, 1, 3), mk(7, 2, 2), mk(9, 2, 2)
+    cu_q, cu_k = [0, 3, 7], [0, 5, 9]
+    gg = torch.rand(2, 7, generator=g, dtype=F64)
+    dq, dk = O.oracle_bwd_teacher_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, 0.8, 1.3, True, gg)
+    loss = lambda qt, kt: float((O.oracle_fwd_varlen(qt, kt, q_s, k_s, cu_q, cu_k, 0.8, 1.3,
+                                                     True)[0] * gg).sum())
+    h = 1e-6
+    for (i, hh, c) in [(1, 0, 2), (6, 1, 0)]:
+        e = torch.zeros_like(q_t); e[i, hh, c] = h
+        fd = (loss(q_t + e, k_t) - loss(q_t - e, k_t)) / (2 * h)
+        assert abs(fd - dq[i, hh, c].item()) <= 1e-6 * max(1.0, abs(fd))
+    for (j, c) in [(0, 1), (4, 2), (8, 0)]:
+        e = torch.zeros_like(k_t); e[j, 0, c] = h
+        fd = (loss(q_t, k_t + e) - loss(q_t, k_t - e)) / (2 * h)
+        assert abs(fd - dk[j, 0, c].item()) <= 1e-6 * max(1.0, abs(fd))
+
+
+def test_varlen_one_sequence_mistake_is_caught(monkeypatch):
+    """Treating the packed tensor as one sequence (no boundaries) fails the brute force."""
+    lq, lk = [3, 4], [4, 3]
+    q_t, k_t, q_s, k_s, cu_q, cu_k, gg = varlen_case(lq, lk, 2, 2, 2, 3, 2, 21)
+    kl_r, _, _, _ = brute_force_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, 0.7, 1.1, True, gg)
+    monkeypatch.setattr(O, "_seq_bounds", lambda cu: [(0, int(cu[-1]))])
+    kl, _, _ = O.oracle_fwd_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, 0.7, 1.1, True)
+    assert not torch.allclose(kl, kl_r, rtol=1e-6, atol=1e-8)
+
+
+def test_varlen_rejects_bad_offsets():
+    q = torch.zeros(4, 1, 2)
+    with pytest.raises(ValueError):
+        O.oracle_fwd_varlen(q, q, q, q, [0, 3, 2, 4], [0, 1, 2, 4], 1.0, 1.0, False)
+    with pytest.raises(ValueError):
+        O.oracle_fwd_varlen(q, q, q, q, [1, 4], [0, 4], 1.0, 1.0, False)

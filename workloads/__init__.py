@@ -8,7 +8,7 @@ The five workloads follow the synthetic attention shapes the method is measured
 on ("StreamKL: Fast and Memory-Efficient KL Divergence for Boosting Attention
 Distillation", abstract: long-context attention distillation between a teacher
 and a student attention map). The pages print no workload table, so the shapes,
-value distributions and seeds here are the plain reading stated in the design doc:
+value distributions and seeds here are a plain reading of those workloads:
 
 * teacher Q and K are standard normal, rounded to bf16;
 * the student is either the teacher plus sigma * N(0, 1) noise (added in fp32 to
