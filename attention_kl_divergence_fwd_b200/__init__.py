@@ -11,6 +11,11 @@ is no CPU fallback: if the library is missing, importing the functions raises.
 
 Tensors: bf16 [B, H, N, d] contiguous on one CUDA device (d in {64, 128}); row
 statistics and g fp32 [B, H, N_Q]; gradients fp32.
+
+The ``*_gqa`` variants take K tensors with fewer heads than Q (grouped-query attention).
+The ``*_varlen`` variants take packed sequences: q_* [total_q, H, d], k_* [total_k, H_kv, d],
+int32 offsets cu_seqlens_q / cu_seqlens_k [B+1] on the device, row statistics and g
+[H, total_q]; gradients keep the packed shapes of Q and K.
 """
 from __future__ import annotations
 
@@ -23,7 +28,8 @@ LIB_PATH = os.path.join(_PKG, "lib", "libstreamkl.so")
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "MISALIGNED", 4: "LAUNCH", 5: "TIMEOUT"}
 EXPORTS = ("streamkl_fwd", "streamkl_bwd", "streamkl_bwd_teacher", "streamkl_fwd_gqa",
-           "streamkl_bwd_gqa", "streamkl_bwd_teacher_gqa", "streamkl_status_string",
+           "streamkl_bwd_gqa", "streamkl_bwd_teacher_gqa", "streamkl_fwd_varlen",
+           "streamkl_bwd_varlen", "streamkl_bwd_teacher_varlen", "streamkl_status_string",
            "streamkl_device_status", "streamkl_version")
 
 
@@ -62,6 +68,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.streamkl_bwd_teacher_gqa.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, f, i, vp,
                                              vp, vp, vp, vp, vp, vp]
     lib.streamkl_bwd_teacher_gqa.restype = i
+    # varlen: q_t, k_t, q_s, k_s, cu_q, cu_k, B, H, H_kv_T, H_kv_S, total_q, total_k,
+    # max_q, max_k, d_T, d_S, scale_T, scale_S, causal, then the outputs / row inputs.
+    head = [vp] * 6 + [i] * 10 + [f, f, i]
+    lib.streamkl_fwd_varlen.argtypes = head + [vp, vp, vp, vp]
+    lib.streamkl_fwd_varlen.restype = i
+    lib.streamkl_bwd_varlen.argtypes = head + [vp, vp, vp, vp, vp, vp]
+    lib.streamkl_bwd_varlen.restype = i
+    lib.streamkl_bwd_teacher_varlen.argtypes = head + [vp, vp, vp, vp, vp, vp, vp]
+    lib.streamkl_bwd_teacher_varlen.restype = i
     lib.streamkl_status_string.argtypes = [i]
     lib.streamkl_status_string.restype = ctypes.c_char_p
     lib.streamkl_device_status.argtypes = [vp]
@@ -135,9 +150,10 @@ def streamkl_fwd(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: boo
     import torch
     B, H, n_q, n_k, d_t, d_s = _shape(q_t, k_t, q_s, k_s)
     dev = q_t.device
-    kl = torch.empty(B, H, n_q, device=dev, dtype=torch.float32) if kl is None else kl
-    lse_t = torch.empty_like(kl) if lse_t is None else lse_t
-    lse_s = torch.empty_like(kl) if lse_s is None else lse_s
+    mk = lambda: torch.empty(B, H, n_q, device=dev, dtype=torch.float32)
+    kl = mk() if kl is None else _check_out(kl, (B, H, n_q), "kl")
+    lse_t = mk() if lse_t is None else _check_out(lse_t, (B, H, n_q), "lse_t")
+    lse_s = mk() if lse_s is None else _check_out(lse_s, (B, H, n_q), "lse_s")
     st = streamkl_fwd_raw(q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(),
                           B, H, n_q, n_k, d_t, d_s, scale_T, scale_S, causal,
                           kl.data_ptr(), lse_t.data_ptr(), lse_s.data_ptr(), _stream_ptr(stream))
@@ -154,8 +170,10 @@ def streamkl_bwd(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: boo
     for name, t in (("lse_t", lse_t), ("lse_s", lse_s), ("g", g)):
         if t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != (B, H, n_q):
             raise ValueError(f"{name} must be contiguous fp32 [B,H,N_Q]")
-    dq_s = torch.empty(B, H, n_q, d_s, device=dev, dtype=torch.float32) if dq_s is None else dq_s
-    dk_s = torch.empty(B, H, n_k, d_s, device=dev, dtype=torch.float32) if dk_s is None else dk_s
+    dq_s = (torch.empty(B, H, n_q, d_s, device=dev, dtype=torch.float32) if dq_s is None
+            else _check_out(dq_s, (B, H, n_q, d_s), "dq_s"))
+    dk_s = (torch.empty(B, H, n_k, d_s, device=dev, dtype=torch.float32) if dk_s is None
+            else _check_out(dk_s, (B, H, n_k, d_s), "dk_s"))
     st = streamkl_bwd_raw(q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(),
                           B, H, n_q, n_k, d_t, d_s, scale_T, scale_S, causal,
                           lse_t.data_ptr(), lse_s.data_ptr(), g.data_ptr(),
@@ -173,8 +191,10 @@ def streamkl_bwd_teacher(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, cau
     for name, t in (("kl", kl), ("lse_t", lse_t), ("lse_s", lse_s), ("g", g)):
         if t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != (B, H, n_q):
             raise ValueError(f"{name} must be contiguous fp32 [B,H,N_Q]")
-    dq_t = torch.empty(B, H, n_q, d_t, device=dev, dtype=torch.float32) if dq_t is None else dq_t
-    dk_t = torch.empty(B, H, n_k, d_t, device=dev, dtype=torch.float32) if dk_t is None else dk_t
+    dq_t = (torch.empty(B, H, n_q, d_t, device=dev, dtype=torch.float32) if dq_t is None
+            else _check_out(dq_t, (B, H, n_q, d_t), "dq_t"))
+    dk_t = (torch.empty(B, H, n_k, d_t, device=dev, dtype=torch.float32) if dk_t is None
+            else _check_out(dk_t, (B, H, n_k, d_t), "dk_t"))
     st = streamkl_bwd_teacher_raw(q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(),
                                   k_s.data_ptr(), B, H, n_q, n_k, d_t, d_s, scale_T, scale_S,
                                   causal, kl.data_ptr(), lse_t.data_ptr(), lse_s.data_ptr(),
@@ -205,9 +225,10 @@ def streamkl_fwd_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal:
     import torch
     B, H, h_kt, h_ks, n_q, n_k, d_t, d_s = _shape_gqa(q_t, k_t, q_s, k_s)
     dev = q_t.device
-    kl = torch.empty(B, H, n_q, device=dev, dtype=torch.float32) if kl is None else kl
-    lse_t = torch.empty_like(kl) if lse_t is None else lse_t
-    lse_s = torch.empty_like(kl) if lse_s is None else lse_s
+    mk = lambda: torch.empty(B, H, n_q, device=dev, dtype=torch.float32)
+    kl = mk() if kl is None else _check_out(kl, (B, H, n_q), "kl")
+    lse_t = mk() if lse_t is None else _check_out(lse_t, (B, H, n_q), "lse_t")
+    lse_s = mk() if lse_s is None else _check_out(lse_s, (B, H, n_q), "lse_s")
     st = load_library().streamkl_fwd_gqa(
         q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), B, H, h_kt, h_ks, n_q,
         n_k, d_t, d_s, float(scale_T), float(scale_S), int(bool(causal)), kl.data_ptr(),
@@ -221,9 +242,12 @@ def streamkl_bwd_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal:
     """streamkl_bwd with grouped K heads; dk_s has the student's K-head count."""
     import torch
     B, H, h_kt, h_ks, n_q, n_k, d_t, d_s = _shape_gqa(q_t, k_t, q_s, k_s)
+    _check_rows((("lse_t", lse_t), ("lse_s", lse_s), ("g", g)), (B, H, n_q))
     dev = q_t.device
-    dq_s = torch.empty(B, H, n_q, d_s, device=dev, dtype=torch.float32) if dq_s is None else dq_s
-    dk_s = torch.empty(B, h_ks, n_k, d_s, device=dev, dtype=torch.float32) if dk_s is None else dk_s
+    dq_s = (torch.empty(B, H, n_q, d_s, device=dev, dtype=torch.float32) if dq_s is None
+            else _check_out(dq_s, (B, H, n_q, d_s), "dq_s"))
+    dk_s = (torch.empty(B, h_ks, n_k, d_s, device=dev, dtype=torch.float32) if dk_s is None
+            else _check_out(dk_s, (B, h_ks, n_k, d_s), "dk_s"))
     st = load_library().streamkl_bwd_gqa(
         q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), B, H, h_kt, h_ks, n_q,
         n_k, d_t, d_s, float(scale_T), float(scale_S), int(bool(causal)), lse_t.data_ptr(),
@@ -237,15 +261,123 @@ def streamkl_bwd_teacher_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float,
     """streamkl_bwd_teacher with grouped K heads; dk_t has the teacher's K-head count."""
     import torch
     B, H, h_kt, h_ks, n_q, n_k, d_t, d_s = _shape_gqa(q_t, k_t, q_s, k_s)
+    _check_rows((("kl", kl), ("lse_t", lse_t), ("lse_s", lse_s), ("g", g)), (B, H, n_q))
     dev = q_t.device
-    dq_t = torch.empty(B, H, n_q, d_t, device=dev, dtype=torch.float32) if dq_t is None else dq_t
-    dk_t = torch.empty(B, h_kt, n_k, d_t, device=dev, dtype=torch.float32) if dk_t is None else dk_t
+    dq_t = (torch.empty(B, H, n_q, d_t, device=dev, dtype=torch.float32) if dq_t is None
+            else _check_out(dq_t, (B, H, n_q, d_t), "dq_t"))
+    dk_t = (torch.empty(B, h_kt, n_k, d_t, device=dev, dtype=torch.float32) if dk_t is None
+            else _check_out(dk_t, (B, h_kt, n_k, d_t), "dk_t"))
     st = load_library().streamkl_bwd_teacher_gqa(
         q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), B, H, h_kt, h_ks, n_q,
         n_k, d_t, d_s, float(scale_T), float(scale_S), int(bool(causal)), kl.data_ptr(),
         lse_t.data_ptr(), lse_s.data_ptr(), g.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(),
         _stream_ptr(stream))
     _check(st, "streamkl_bwd_teacher_gqa")
+    return dq_t, dk_t
+
+
+def _check_rows(named, shape) -> None:
+    import torch
+    for name, t in named:
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or \
+                tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor of shape {tuple(shape)}")
+
+
+def _check_out(t, shape, name):
+    import torch
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or \
+            tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor of shape {tuple(shape)}")
+    return t
+
+
+def _shape_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k):
+    """Packed shapes: q_* [total_q, H, d], k_* [total_k, H_kv, d], cu_* int32 [B+1]."""
+    import torch
+    for name, t in (("q_t", q_t), ("k_t", k_t), ("q_s", q_s), ("k_s", k_s)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 3-D bf16 CUDA tensor [total, heads, d]")
+    for name, t in (("cu_seqlens_q", cu_q), ("cu_seqlens_k", cu_k)):
+        if t.dtype != torch.int32 or not t.is_cuda or t.dim() != 1 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 1-D int32 CUDA tensor [B+1]")
+    if cu_q.numel() != cu_k.numel() or cu_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B+1 >= 2 entries")
+    total_q, H, d_t = q_t.shape
+    total_k, h_kt = k_t.shape[0], k_t.shape[1]
+    h_ks, d_s = k_s.shape[1], q_s.shape[2]
+    if tuple(k_t.shape) != (total_k, h_kt, d_t) or tuple(q_s.shape) != (total_q, H, d_s) or \
+            tuple(k_s.shape) != (total_k, h_ks, d_s):
+        raise ValueError("inconsistent shapes")
+    return cu_q.numel() - 1, H, h_kt, h_ks, total_q, total_k, d_t, d_s
+
+
+def streamkl_fwd_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                        max_seqlen_k: int, scale_T: float, scale_S: float, causal: bool,
+                        kl=None, lse_t=None, lse_s=None, stream=None):
+    """streamkl_fwd over packed sequences: KL, LSE_T, LSE_S fp32 [H, total_q]. Rows that
+    belong to no sequence are not written."""
+    import torch
+    B, H, h_kt, h_ks, tq, tk, d_t, d_s = _shape_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q,
+                                                        cu_seqlens_k)
+    dev = q_t.device
+    mk = lambda: torch.empty(H, tq, device=dev, dtype=torch.float32)
+    kl = mk() if kl is None else _check_out(kl, (H, tq), "kl")
+    lse_t = mk() if lse_t is None else _check_out(lse_t, (H, tq), "lse_t")
+    lse_s = mk() if lse_s is None else _check_out(lse_s, (H, tq), "lse_s")
+    st = load_library().streamkl_fwd_varlen(
+        q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), cu_seqlens_q.data_ptr(),
+        cu_seqlens_k.data_ptr(), B, H, h_kt, h_ks, tq, tk, int(max_seqlen_q), int(max_seqlen_k),
+        d_t, d_s, float(scale_T), float(scale_S), int(bool(causal)), kl.data_ptr(),
+        lse_t.data_ptr(), lse_s.data_ptr(), _stream_ptr(stream))
+    _check(st, "streamkl_fwd_varlen")
+    return kl, lse_t, lse_s
+
+
+def streamkl_bwd_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                        max_seqlen_k: int, scale_T: float, scale_S: float, causal: bool,
+                        lse_t, lse_s, g, dq_s=None, dk_s=None, stream=None):
+    """streamkl_bwd over packed sequences: dQ_S [total_q, H, d_S], dK_S [total_k, H_kv_S, d_S]."""
+    import torch
+    B, H, h_kt, h_ks, tq, tk, d_t, d_s = _shape_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q,
+                                                        cu_seqlens_k)
+    _check_rows((("lse_t", lse_t), ("lse_s", lse_s), ("g", g)), (H, tq))
+    dev = q_t.device
+    dq_s = (torch.empty(tq, H, d_s, device=dev, dtype=torch.float32) if dq_s is None
+            else _check_out(dq_s, (tq, H, d_s), "dq_s"))
+    dk_s = (torch.empty(tk, h_ks, d_s, device=dev, dtype=torch.float32) if dk_s is None
+            else _check_out(dk_s, (tk, h_ks, d_s), "dk_s"))
+    st = load_library().streamkl_bwd_varlen(
+        q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), cu_seqlens_q.data_ptr(),
+        cu_seqlens_k.data_ptr(), B, H, h_kt, h_ks, tq, tk, int(max_seqlen_q), int(max_seqlen_k),
+        d_t, d_s, float(scale_T), float(scale_S), int(bool(causal)), lse_t.data_ptr(),
+        lse_s.data_ptr(), g.data_ptr(), dq_s.data_ptr(), dk_s.data_ptr(), _stream_ptr(stream))
+    _check(st, "streamkl_bwd_varlen")
+    return dq_s, dk_s
+
+
+def streamkl_bwd_teacher_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k,
+                                max_seqlen_q: int, max_seqlen_k: int, scale_T: float,
+                                scale_S: float, causal: bool, kl, lse_t, lse_s, g, dq_t=None,
+                                dk_t=None, stream=None):
+    """streamkl_bwd_teacher over packed sequences: dQ_T [total_q, H, d_T], dK_T
+    [total_k, H_kv_T, d_T]."""
+    import torch
+    B, H, h_kt, h_ks, tq, tk, d_t, d_s = _shape_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q,
+                                                        cu_seqlens_k)
+    _check_rows((("kl", kl), ("lse_t", lse_t), ("lse_s", lse_s), ("g", g)), (H, tq))
+    dev = q_t.device
+    dq_t = (torch.empty(tq, H, d_t, device=dev, dtype=torch.float32) if dq_t is None
+            else _check_out(dq_t, (tq, H, d_t), "dq_t"))
+    dk_t = (torch.empty(tk, h_kt, d_t, device=dev, dtype=torch.float32) if dk_t is None
+            else _check_out(dk_t, (tk, h_kt, d_t), "dk_t"))
+    st = load_library().streamkl_bwd_teacher_varlen(
+        q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), cu_seqlens_q.data_ptr(),
+        cu_seqlens_k.data_ptr(), B, H, h_kt, h_ks, tq, tk, int(max_seqlen_q), int(max_seqlen_k),
+        d_t, d_s, float(scale_T), float(scale_S), int(bool(causal)), kl.data_ptr(),
+        lse_t.data_ptr(), lse_s.data_ptr(), g.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(),
+        _stream_ptr(stream))
+    _check(st, "streamkl_bwd_teacher_varlen")
     return dq_t, dk_t
 
 

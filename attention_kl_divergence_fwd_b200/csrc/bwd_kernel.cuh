@@ -38,25 +38,27 @@
 namespace skl {
 
 struct BwdArgs {
-  int BH, N_Q, N_K;
+  int BH, N_Q, N_K;  // B*H; queries / keys per sequence (packed: the longest sequence)
   int causal;
-  int off;          // N_K - N_Q
   float cT, cS;     // |scale| * log2(e)
   float aT, aS;     // |scale| (natural units, teacher gradient only)
   float scale_G;    // signed scale of the side being differentiated (G = g * scale_G)
   int n_ktiles;     // ceil(N_K / 128)
-  int n_qtiles;     // ceil(N_Q / 64)
   int group;        // heads per scheduling group (grouped_order)
   int H;            // query heads per batch entry
   int gT, gS;       // query heads per teacher / student K head (GQA; 1 = one K head each)
   int dk_reduce;    // 1: several query heads share the differentiated K head, so dK
                     //    tiles are added into the zeroed dk (bulk reduce) instead of stored
+  const int* cu_q;  // packed layout: [B+1] sequence offsets (null: dense [B, H, N, d])
+  const int* cu_k;
+  int total_q, total_k;    // packed layout: rows of the packed Q / K tensors
+  long long dk_hs, dk_rs;  // dk element strides of a K head and of a key row
   const float* lse_t;
   const float* lse_s;
   const float* g;
   const float* kl;  // teacher gradient only: E = KL + LSE_T - LSE_S
-  float* dq;        // dQ of the differentiated side [BH, N_Q, d_G]
-  float* dk;        // dK of the differentiated side [BH, N_K, d_G]
+  float* dq;        // dQ of the differentiated side (fp32, the layout of Q)
+  float* dk;        // dK of the differentiated side (fp32, the layout of K)
 };
 
 // TEACHER = false: gradients of the student (dQ_S, dK_S), d_G = d_S.
@@ -141,19 +143,22 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   // Key tile 0 sees the most query tiles (causal): heaviest first, heads in groups.
   int bh, kt;
   grouped_order(blockIdx.x, args.BH, args.n_ktiles, args.group, bh, kt);
-  // K heads of this query head (grouped-query attention: query head h reads K head h/g).
-  const int hq = bh % args.H, bq = bh / args.H;
-  const int bkt = bq * (args.H / args.gT) + hq / args.gT;
-  const int bks = bq * (args.H / args.gS) + hq / args.gS;
-  const int bkg = TEACHER ? bkt : bks;  // K head that receives this CTA's dK
+  SeqView seq;
+  if (!seq_view(args.cu_q, args.cu_k, bh, args.H, args.gT, args.gS, args.N_Q, args.N_K,
+                args.total_q, args.total_k, seq)) {
+    if (threadIdx.x == 0) atomicOr(&g_skl_error, kErrBadOffsets);
+    return;
+  }
   const int k0 = kt * C::BN;
+  if (k0 >= seq.nk) return;  // packed layout: this sequence is shorter than the longest
+  const int bkg = TEACHER ? seq.zkt : seq.zks;  // K head that receives this CTA's dK
 
   int jq_begin = 0;
   if (args.causal) {
-    const int first_q = k0 - args.off;  // first query row that sees key k0
+    const int first_q = k0 - seq.off;  // first query row that sees key k0
     jq_begin = first_q <= 0 ? 0 : first_q / C::BM;
   }
-  const int n_steps = max(0, args.n_qtiles - jq_begin);
+  const int n_steps = max(0, (seq.nq + C::BM - 1) / C::BM - jq_begin);
   // Staging rounds after the last step that add the dK tile (128 keys = 2 x 64 rows).
   const int dk_rounds = (args.dk_reduce && n_steps > 0) ? 2 : 0;
 
@@ -205,12 +210,14 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       const uint32_t kb = smem_u32(&bars->k_full);
       mbar_arrive_expect_tx(kb, C::KT_TILE + C::KS_TILE);
       for (int blk = 0; blk < DT / 64; ++blk)
-        tma_load_3d(sb + C::OFF_KT + blk * (C::BN * 128), &map_kt, kb, blk * 64, k0, bkt, keep);
+        tma_load_3d(sb + C::OFF_KT + blk * (C::BN * 128), &map_kt, kb, blk * 64, seq.kr + k0,
+                    seq.zkt, keep);
       for (int blk = 0; blk < DS / 64; ++blk)
-        tma_load_3d(sb + C::OFF_KS + blk * (C::BN * 128), &map_ks, kb, blk * 64, k0, bks, keep);
+        tma_load_3d(sb + C::OFF_KS + blk * (C::BN * 128), &map_ks, kb, blk * 64, seq.kr + k0,
+                    seq.zks, keep);
       for (int s = 0; s < n_steps; ++s) {
         const int st = s % C::NQST;
-        const int i0 = (jq_begin + s) * C::BM;
+        const int i0 = seq.qr + (jq_begin + s) * C::BM;
         if (!mbar_wait(smem_u32(&bars->q_empty[st]), ((s / C::NQST) & 1) ^ 1)) {
           skl_fail_b(abort_flag);
           break;
@@ -219,10 +226,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
         mbar_arrive_expect_tx(fb, C::Q_STAGE);
         for (int blk = 0; blk < DT / 64; ++blk)
-          tma_load_3d(q_base + blk * (C::BM * 128), &map_qt, fb, blk * 64, i0, bh, keep);
+          tma_load_3d(q_base + blk * (C::BM * 128), &map_qt, fb, blk * 64, i0, seq.zq, keep);
         for (int blk = 0; blk < DS / 64; ++blk)
-          tma_load_3d(q_base + C::QT_TILE + blk * (C::BM * 128), &map_qs, fb, blk * 64, i0, bh,
-                      keep);
+          tma_load_3d(q_base + C::QT_TILE + blk * (C::BM * 128), &map_qs, fb, blk * 64, i0,
+                      seq.zq, keep);
         issued = s + 1;
       }
       if (*abort_flag) {
@@ -248,8 +255,8 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         ls[r] = -INFINITY;
         gg[r] = 0.f;
         kv[r] = 0.f;
-        if (s < n_steps && row < args.N_Q) {
-          const size_t o = (size_t)bh * args.N_Q + row;
+        if (s < n_steps && row < seq.nq) {
+          const size_t o = (size_t)(seq.ob + row);
           lt[r] = __ldg(args.lse_t + o);
           ls[r] = __ldg(args.lse_s + o);
           gg[r] = __ldg(args.g + o);
@@ -303,12 +310,12 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           break;
         }
         if (p < n_steps) {  // dQ part of step p: 64 query rows
-          const int i0 = (jq_begin + p) * C::BM;
+          const int i0 = seq.qr + (jq_begin + p) * C::BM;
 #pragma unroll
           for (int db = 0; db < DG / 32; ++db)
-            tma_reduce_add_3d(&map_dq, sb + C::OFF_STG + db * (C::BM * 128), db * 32, i0, bh);
+            tma_reduce_add_3d(&map_dq, sb + C::OFF_STG + db * (C::BM * 128), db * 32, i0, seq.zq);
         } else {  // dK tile of this CTA, 64 key rows per round
-          const int r0 = k0 + (p - n_steps) * 64;
+          const int r0 = seq.kr + k0 + (p - n_steps) * 64;
 #pragma unroll
           for (int db = 0; db < DG / 32; ++db)
             tma_reduce_add_3d(&map_dk, sb + C::OFF_STG + db * (C::BM * 128), db * 32, r0, bkg);
@@ -459,9 +466,12 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       // issued before this step's scores, so this wait normally returns at once).
       if (!mbar_wait(smem_u32(&bars->ds_empty[wg]), ((s >> 1) & 1) ^ 1)) { ok = false; break; }
 
-      // Query column c is allowed for this key iff i0 + c >= key - off.
-      const bool need_mask = args.causal && (i0 + args.off < k0 + C::BN - 1);
-      const int cmin = need_mask ? (key - args.off - i0) : -1;
+      // Query column c is allowed for this key iff i0 + c >= key - off; keys past the end
+      // of the sequence (the next sequence's keys in the packed layout, zero fill in the
+      // dense one) get dS = 0 for every column.
+      const bool causal_mask = args.causal && (i0 + seq.off < k0 + C::BN - 1);
+      const bool need_mask = causal_mask || (k0 + C::BN > seq.nk);
+      const int cmin = key >= seq.nk ? C::BM : (causal_mask ? (key - seq.off - i0) : -1);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {  // 8 query columns = one 16-byte chunk of dS^T
         const float4 nlt0 = *reinterpret_cast<const float4*>(sts + u * 8);
@@ -532,9 +542,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         }
       }
     }
-    if (ok && !dk_rounds && key < args.N_K) {
-      float4* dst = reinterpret_cast<float4*>(args.dk + ((size_t)bkg * args.N_K + key) * DG +
-                                              wg * DKH);
+    if (ok && !dk_rounds && key < seq.nk) {
+      float4* dst = reinterpret_cast<float4*>(args.dk + bkg * args.dk_hs +
+                                              (long long)(seq.kr + key) * args.dk_rs + wg * DKH);
 #pragma unroll
       for (int c = 0; c < DKH; c += 4)
         dst[c / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),

@@ -27,14 +27,16 @@
 namespace skl {
 
 struct FwdArgs {
-  int BH, N_Q, N_K;
+  int BH, N_Q, N_K;   // B*H; queries / keys per sequence (packed: the longest sequence)
   int causal;
-  int off;            // N_K - N_Q (bottom-right causal alignment)
   float cT, cS;       // |scale| * log2(e); the MMA negates A when the scale is negative
   int n_ctas_per_bh;  // ceil(N_Q / 256)
   int group;          // heads per scheduling group (grouped_order)
   int H;              // query heads per batch entry
   int gT, gS;         // query heads per teacher / student K head (GQA; 1 = one K head each)
+  const int* cu_q;    // packed layout: [B+1] sequence offsets (null: dense [B, H, N, d])
+  const int* cu_k;
+  int total_q, total_k;  // packed layout: rows of the packed Q / K tensors
   float* kl;
   float* lse_t;
   float* lse_s;
@@ -215,25 +217,28 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   int bh, unit;
   grouped_order(blockIdx.x, args.BH, args.n_ctas_per_bh, args.group, bh, unit);
   const int qpair = args.n_ctas_per_bh - 1 - unit;
-  // K heads of this query head (grouped-query attention: query head h reads K head h/g).
-  const int hq = bh % args.H, bq = bh / args.H;
-  const int bkt = bq * (args.H / args.gT) + hq / args.gT;
-  const int bks = bq * (args.H / args.gS) + hq / args.gS;
+  SeqView seq;
+  if (!seq_view(args.cu_q, args.cu_k, bh, args.H, args.gT, args.gS, args.N_Q, args.N_K,
+                args.total_q, args.total_k, seq)) {
+    if (threadIdx.x == 0) atomicOr(&g_skl_error, kErrBadOffsets);
+    return;
+  }
   const int q0 = qpair * (C::NQ * C::BM);
-  const int n_ktiles_all = (args.N_K + C::BN - 1) / C::BN;
+  if (q0 >= seq.nq) return;  // packed layout: this sequence is shorter than the longest
+  const int n_ktiles_all = (seq.nk + C::BN - 1) / C::BN;
 
   // Key tiles needed by each query tile.
   int nk[C::NQ];
 #pragma unroll
   for (int q = 0; q < C::NQ; ++q) {
     const int first = q0 + q * C::BM;
-    if (first >= args.N_Q) {
+    if (first >= seq.nq) {
       nk[q] = 0;
     } else if (!args.causal) {
       nk[q] = n_ktiles_all;
     } else {
-      const int last_row = min(first + C::BM, args.N_Q) - 1;
-      const int last_key = last_row + args.off;
+      const int last_row = min(first + C::BM, seq.nq) - 1;
+      const int last_key = last_row + seq.off;
       nk[q] = last_key < 0 ? 0 : min(n_ktiles_all, last_key / C::BN + 1);
     }
   }
@@ -285,19 +290,19 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       tc_fence_after();
       const int k0 = j * C::BN;
       const bool need_mask =
-          (k0 + C::BN > args.N_K) || (args.causal && k0 + C::BN - 1 > first_row + args.off);
+          (k0 + C::BN > seq.nk) || (args.causal && k0 + C::BN - 1 > first_row + seq.off);
       const uint32_t ta = tmem + lane_off + q * 256 + b * 128;
       const uint32_t fr = smem_u32(&bars->s_free[q][b]);
       if (need_mask) {
-        int last = args.N_K - 1;
-        if (args.causal) last = min(last, row + args.off);
+        int last = seq.nk - 1;
+        if (args.causal) last = min(last, row + seq.off);
         fold_tile<true>(st, ta, cT, cS, last - k0, fr, lane);
       } else {
         fold_tile<false>(st, ta, cT, cS, C::BN - 1, fr, lane);
       }
     }
 
-    if (ok && row < args.N_Q) {
+    if (ok && row < seq.nq) {
       const float LN2 = 0.69314718055994530942f;
       float kl, lse_t, lse_s;
       if (st.lT > 0.f) {
@@ -311,7 +316,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         lse_t = -INFINITY;
         lse_s = -INFINITY;
       }
-      const size_t o = (size_t)bh * args.N_Q + row;
+      const size_t o = (size_t)(seq.ob + row);
       args.kl[o] = kl;
       args.lse_t[o] = lse_t;
       args.lse_s[o] = lse_s;
@@ -332,10 +337,10 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         for (int q = 0; q < C::NQ; ++q) {
           for (int blk = 0; blk < DT / 64; ++blk)
             tma_load_3d(s_qt + q * C::QT_TILE + blk * (C::BM * 128), &map_qt, qb, blk * 64,
-                        q0 + q * C::BM, bh, once);
+                        seq.qr + q0 + q * C::BM, seq.zq, once);
           for (int blk = 0; blk < DS / 64; ++blk)
             tma_load_3d(s_qs + q * C::QS_TILE + blk * (C::BM * 128), &map_qs, qb, blk * 64,
-                        q0 + q * C::BM, bh, once);
+                        seq.qr + q0 + q * C::BM, seq.zq, once);
         }
         int issued = 0;
         for (int j = 0; j < nk_max; ++j) {
@@ -348,10 +353,11 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           mbar_arrive_expect_tx(fb, C::STAGE);
           const uint32_t st = s_k + s * C::STAGE;
           for (int blk = 0; blk < DT / 64; ++blk)
-            tma_load_3d(st + blk * (C::BN * 128), &map_kt, fb, blk * 64, j * C::BN, bkt, keep);
+            tma_load_3d(st + blk * (C::BN * 128), &map_kt, fb, blk * 64, seq.kr + j * C::BN,
+                        seq.zkt, keep);
           for (int blk = 0; blk < DS / 64; ++blk)
-            tma_load_3d(st + C::KT_TILE + blk * (C::BN * 128), &map_ks, fb, blk * 64, j * C::BN,
-                        bks, keep);
+            tma_load_3d(st + C::KT_TILE + blk * (C::BN * 128), &map_ks, fb, blk * 64,
+                        seq.kr + j * C::BN, seq.zks, keep);
           issued = j + 1;
         }
         if (*abort_flag) {

@@ -265,6 +265,59 @@ __device__ __forceinline__ void grouped_order(int t, int bh_total, int units, in
   }
 }
 
+// ------------------------------------------------------------ sequence view
+//
+// One CTA works on one (sequence, query head) problem. Two tensor layouts:
+//  * dense  [B, H, N, d]: every sequence has N_Q queries and N_K keys; the TMA maps are
+//    {d, N, B*heads} and the row arrays (KL, LSE, g) are [B*H, N_Q];
+//  * packed [total, heads, d] with cu_q / cu_k offsets ([B+1] int32 in device memory):
+//    sequence b owns rows cu[b] .. cu[b+1]-1; the TMA maps are {d, total, heads} and the
+//    row arrays are [H, total_q]. N_Q / N_K are then the longest sequence lengths.
+// Query head h reads teacher K head h/gT and student K head h/gS (grouped-query attention).
+struct SeqView {
+  int nq, nk;         // queries and keys of this sequence
+  int off;            // nk - nq (bottom-right causal alignment within the sequence)
+  int qr, kr;         // row of the sequence's first query / key in the tensor maps
+  int zq, zkt, zks;   // head coordinate of Q, K_T, K_S in the tensor maps
+  long long ob;       // index of the sequence's query row 0 in the row arrays
+};
+
+// Returns false when the packed offsets of this sequence are malformed (not
+// 0 <= cu[b] <= cu[b+1] <= total, or longer than the longest length given).
+__device__ __forceinline__ bool seq_view(const int* cu_q, const int* cu_k, int bh, int H,
+                                         int gT, int gS, int N_Q, int N_K, int total_q,
+                                         int total_k, SeqView& v) {
+  const int b = bh / H, h = bh - b * H;
+  if (cu_q == nullptr) {
+    v.nq = N_Q;
+    v.nk = N_K;
+    v.qr = 0;
+    v.kr = 0;
+    v.zq = bh;
+    v.zkt = b * (H / gT) + h / gT;
+    v.zks = b * (H / gS) + h / gS;
+    v.ob = (long long)bh * N_Q;
+  } else {
+    const int q_lo = __ldg(cu_q + b), q_hi = __ldg(cu_q + b + 1);
+    const int k_lo = __ldg(cu_k + b), k_hi = __ldg(cu_k + b + 1);
+    if (q_lo < 0 || q_hi < q_lo || q_hi > total_q || q_hi - q_lo > N_Q) return false;
+    if (k_lo < 0 || k_hi < k_lo || k_hi > total_k || k_hi - k_lo > N_K) return false;
+    v.nq = q_hi - q_lo;
+    v.nk = k_hi - k_lo;
+    v.qr = q_lo;
+    v.kr = k_lo;
+    v.zq = h;
+    v.zkt = h / gT;
+    v.zks = h / gS;
+    v.ob = (long long)h * total_q + q_lo;
+  }
+  v.off = v.nk - v.nq;
+  return true;
+}
+
+// Error word bit for malformed packed-sequence offsets (found on the device).
+constexpr unsigned int kErrBadOffsets = 8u;
+
 // ------------------------------------------------------------------ math
 
 __device__ __forceinline__ float ex2_approx(float x) {

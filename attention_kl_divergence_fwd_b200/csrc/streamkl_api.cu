@@ -1,9 +1,9 @@
 // streamkl_api.cu - C ABI, argument checks and launch planner of the StreamKL library.
 //
 // The planner picks the kernel instantiation from (d_T, d_S), encodes the TMA tensor
-// maps ([B*H, N, d] bf16, 128-byte swizzle, zero fill out of bounds so ragged N needs
-// no padding), orders the grid so causal work is scheduled heaviest-first, and
-// launches on the caller's stream. See include/streamkl.h for the contract.
+// maps (dense [B*H, N, d] or packed [total, heads, d] bf16, 128-byte swizzle, zero fill
+// out of bounds so ragged N needs no padding), orders the grid so causal work is
+// scheduled heaviest-first, and launches on the caller's stream. See include/streamkl.h for the contract.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -38,12 +38,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over a [BH, N, d] bf16 tensor: box of 64 columns (128 bytes) x rows x 1.
-bool make_map(CUtensorMap* m, const void* base, int d, int n, int bh, int box_rows) {
+// 3-D bf16 map {d, rows, heads}: box of 64 columns (128 bytes) x box_rows x 1 head.
+// Dense [BH, N, d]: rows = N with stride d, heads = BH with stride N*d. Packed
+// [total, heads, d]: rows = total with stride heads*d, heads with stride d.
+bool make_map(CUtensorMap* m, const void* base, int d, long long rows, long long heads,
+              long long row_stride, long long head_stride, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)bh};
-  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)head_stride * 2};
   const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
@@ -52,12 +55,13 @@ bool make_map(CUtensorMap* m, const void* base, int d, int n, int bh, int box_ro
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D map over the fp32 [BH, N_Q, d] dQ accumulator: box of 32 columns x 64 rows x 1.
-bool make_map_f32(CUtensorMap* m, void* base, int d, int n, int bh) {
+// The same over an fp32 dQ / dK accumulator: box of 32 columns x 64 rows x 1 head.
+bool make_map_f32(CUtensorMap* m, void* base, int d, long long rows, long long heads,
+                  long long row_stride, long long head_stride) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)bh};
-  const cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)n * d * 4};
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_stride * 4, (cuuint64_t)head_stride * 4};
   const cuuint32_t box[3] = {32, 64, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
@@ -66,19 +70,71 @@ bool make_map_f32(CUtensorMap* m, void* base, int d, int n, int bh) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// One call's problem: dense [B, H, N, d] tensors (cu_q == nullptr) or packed sequences.
+struct Problem {
+  const int* cu_q = nullptr;  // packed: [B+1] query / key offsets in device memory
+  const int* cu_k = nullptr;
+  int B = 0, H = 0, H_kv_T = 0, H_kv_S = 0;
+  int N_Q = 0, N_K = 0;          // dense sizes; packed: longest query / key sequence
+  int total_q = 0, total_k = 0;  // packed: rows of the packed Q / K tensors
+  bool packed() const { return cu_q != nullptr; }
+  long long q_rows() const { return packed() ? total_q : (long long)B * H * N_Q; }
+  long long k_rows(int h_kv) const { return packed() ? total_k : (long long)B * h_kv * N_K; }
+};
+
+// Map over a Q (h_kv = 0: H heads) or K tensor of the problem.
+bool map_of(CUtensorMap* m, const void* base, const Problem& P, int d, bool is_k, int h_kv,
+            int box_rows) {
+  const int heads = is_k ? h_kv : P.H;
+  if (P.packed()) {
+    const long long rows = is_k ? P.total_k : P.total_q;
+    // A packed K with no rows is never read (every sequence has no keys); the caller then
+    // passes Q's base, and the map covers one row of it (Q has at least as many heads).
+    if (rows == 0) return make_map(m, base, d, 1, heads, (long long)P.H * d, d, box_rows);
+    return make_map(m, base, d, rows, heads, (long long)heads * d, d, box_rows);
+  }
+  const int n = is_k ? P.N_K : P.N_Q;
+  return make_map(m, base, d, n, (long long)P.B * heads, d, (long long)n * d, box_rows);
+}
+
+bool map_of_f32(CUtensorMap* m, void* base, const Problem& P, int d, bool is_k, int h_kv) {
+  const int heads = is_k ? h_kv : P.H;
+  if (P.packed()) {
+    const long long rows = is_k ? P.total_k : P.total_q;
+    return make_map_f32(m, base, d, rows < 1 ? 1 : rows, heads, (long long)heads * d, d);
+  }
+  const int n = is_k ? P.N_K : P.N_Q;
+  return make_map_f32(m, base, d, n, (long long)P.B * heads, d, (long long)n * d);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 streamkl_status check_common(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
-                             int B, int H, int N_Q, int N_K, int d_T, int d_S, float scale_T,
-                             float scale_S) {
-  if (!q_t || !k_t || !q_s || !k_s) return STREAMKL_ERR_INVALID_ARG;
-  if (B < 1 || H < 1 || N_Q < 1 || N_K < 1) return STREAMKL_ERR_INVALID_ARG;
+                             const Problem& P, int d_T, int d_S, float scale_T, float scale_S) {
+  if (P.B < 1 || P.H < 1) return STREAMKL_ERR_INVALID_ARG;
   if (!std::isfinite(scale_T) || !std::isfinite(scale_S)) return STREAMKL_ERR_INVALID_ARG;
   if ((d_T != 64 && d_T != 128) || (d_S != 64 && d_S != 128)) return STREAMKL_ERR_UNSUPPORTED;
-  const long long bh = (long long)B * H;
-  const long long nmax = N_Q > N_K ? N_Q : N_K;
-  if (bh * nmax >= (1ll << 31) || bh >= (1ll << 24)) return STREAMKL_ERR_UNSUPPORTED;
-  if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(q_s) || !aligned16(k_s))
+  if (P.H_kv_T < 1 || P.H_kv_S < 1 || P.H % P.H_kv_T != 0 || P.H % P.H_kv_S != 0)
+    return STREAMKL_ERR_UNSUPPORTED;
+  const long long bh = (long long)P.B * P.H;
+  if (bh >= (1ll << 24)) return STREAMKL_ERR_UNSUPPORTED;
+  if (P.packed()) {
+    if (!P.cu_k || P.N_Q < 0 || P.N_K < 0 || P.total_q < 0 || P.total_k < 0)
+      return STREAMKL_ERR_INVALID_ARG;
+    if ((long long)P.H * P.total_q >= (1ll << 31) || (long long)P.H * P.total_k >= (1ll << 31))
+      return STREAMKL_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(P.cu_q) & 3u) || (reinterpret_cast<uintptr_t>(P.cu_k) & 3u))
+      return STREAMKL_ERR_MISALIGNED;
+    if (P.total_q > 0 && (!q_t || !q_s)) return STREAMKL_ERR_INVALID_ARG;
+    if (P.total_k > 0 && (!k_t || !k_s)) return STREAMKL_ERR_INVALID_ARG;
+  } else {
+    if (!q_t || !k_t || !q_s || !k_s) return STREAMKL_ERR_INVALID_ARG;
+    if (P.N_Q < 1 || P.N_K < 1) return STREAMKL_ERR_INVALID_ARG;
+    const long long nmax = P.N_Q > P.N_K ? P.N_Q : P.N_K;
+    if (bh * nmax >= (1ll << 31)) return STREAMKL_ERR_UNSUPPORTED;
+  }
+  if ((q_t && !aligned16(q_t)) || (k_t && !aligned16(k_t)) || (q_s && !aligned16(q_s)) ||
+      (k_s && !aligned16(k_s)))
     return STREAMKL_ERR_MISALIGNED;
   return STREAMKL_OK;
 }
@@ -133,47 +189,43 @@ streamkl_status launch_bwd(const CUtensorMap* maps, const skl::BwdArgs& a, bool 
   return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
 }
 
-// Query heads per K head; UNSUPPORTED unless it divides H.
-bool kv_groups(int H, int H_kv_T, int H_kv_S, int& gT, int& gS) {
-  if (H_kv_T < 1 || H_kv_S < 1 || H % H_kv_T != 0 || H % H_kv_S != 0) return false;
-  gT = H / H_kv_T;
-  gS = H / H_kv_S;
-  return true;
-}
-
 streamkl_status fwd_common(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
-                           int B, int H, int H_kv_T, int H_kv_S, int N_Q, int N_K, int d_T,
-                           int d_S, float scale_T, float scale_S, int causal, float* kl,
-                           float* lse_t, float* lse_s, cudaStream_t stream) {
-  streamkl_status st = check_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S);
+                           const Problem& P, int d_T, int d_S, float scale_T, float scale_S,
+                           int causal, float* kl, float* lse_t, float* lse_s,
+                           cudaStream_t stream) {
+  streamkl_status st = check_common(q_t, k_t, q_s, k_s, P, d_T, d_S, scale_T, scale_S);
   if (st != STREAMKL_OK) return st;
+  if (P.q_rows() == 0) return STREAMKL_OK;  // packed, no query rows: nothing to write
   if (!kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
-  int gT, gS;
-  if (!kv_groups(H, H_kv_T, H_kv_S, gT, gS)) return STREAMKL_ERR_UNSUPPORTED;
   if (!aligned16(kl) || !aligned16(lse_t) || !aligned16(lse_s)) return STREAMKL_ERR_MISALIGNED;
-  const int bh = B * H;
+  const bool no_keys = P.packed() && P.total_k == 0;
   CUtensorMap maps[4];
-  if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 128) ||
-      !make_map(&maps[1], k_t, d_T, N_K, B * H_kv_T, 64) ||
-      !make_map(&maps[2], q_s, d_S, N_Q, bh, 128) ||
-      !make_map(&maps[3], k_s, d_S, N_K, B * H_kv_S, 64))
+  if (!map_of(&maps[0], q_t, P, d_T, false, 0, 128) ||
+      !map_of(&maps[1], no_keys ? q_t : k_t, P, d_T, true, P.H_kv_T, 64) ||
+      !map_of(&maps[2], q_s, P, d_S, false, 0, 128) ||
+      !map_of(&maps[3], no_keys ? q_s : k_s, P, d_S, true, P.H_kv_S, 64))
     return STREAMKL_ERR_LAUNCH;
+  const int bh = P.B * P.H;
   skl::FwdArgs a{};
   a.BH = bh;
-  a.N_Q = N_Q;
-  a.N_K = N_K;
+  a.N_Q = P.N_Q;
+  a.N_K = P.N_K;
   a.causal = causal ? 1 : 0;
-  a.off = N_K - N_Q;
   a.cT = std::fabs(scale_T) * kLog2e;
   a.cS = std::fabs(scale_S) * kLog2e;
-  a.n_ctas_per_bh = (N_Q + 255) / 256;
+  a.n_ctas_per_bh = (P.N_Q + 255) / 256;
   a.group = head_group("STREAMKL_FWD_GROUP", 4, bh);
-  a.H = H;
-  a.gT = gT;
-  a.gS = gS;
+  a.H = P.H;
+  a.gT = P.H / P.H_kv_T;
+  a.gS = P.H / P.H_kv_S;
+  a.cu_q = P.cu_q;
+  a.cu_k = P.cu_k;
+  a.total_q = P.total_q;
+  a.total_k = P.total_k;
   a.kl = kl;
   a.lse_t = lse_t;
   a.lse_s = lse_s;
+  if (a.n_ctas_per_bh == 0) return STREAMKL_OK;  // packed, every sequence empty
   const bool nT = scale_T < 0.f, nS = scale_S < 0.f;
   if (d_T == 128 && d_S == 128) return launch_fwd<128, 128>(maps, a, nT, nS, stream);
   if (d_T == 128 && d_S == 64) return launch_fwd<128, 64>(maps, a, nT, nS, stream);
@@ -184,63 +236,96 @@ streamkl_status fwd_common(const void* q_t, const void* k_t, const void* q_s, co
 // Shared body of the student and trainable-teacher backward entry points.
 template <bool TEACHER>
 streamkl_status bwd_common(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
-                           int B, int H, int H_kv_T, int H_kv_S, int N_Q, int N_K, int d_T,
-                           int d_S, float scale_T, float scale_S, int causal, const float* kl,
-                           const float* lse_t, const float* lse_s, const float* g, float* dq,
-                           float* dk, cudaStream_t stream) {
-  streamkl_status st = check_common(q_t, k_t, q_s, k_s, B, H, N_Q, N_K, d_T, d_S, scale_T, scale_S);
+                           const Problem& P, int d_T, int d_S, float scale_T, float scale_S,
+                           int causal, const float* kl, const float* lse_t, const float* lse_s,
+                           const float* g, float* dq, float* dk, cudaStream_t stream) {
+  streamkl_status st = check_common(q_t, k_t, q_s, k_s, P, d_T, d_S, scale_T, scale_S);
   if (st != STREAMKL_OK) return st;
-  if (!lse_t || !lse_s || !g || !dq || !dk || (TEACHER && !kl)) return STREAMKL_ERR_INVALID_ARG;
-  int gT, gS;
-  if (!kv_groups(H, H_kv_T, H_kv_S, gT, gS)) return STREAMKL_ERR_UNSUPPORTED;
-  if (!aligned16(lse_t) || !aligned16(lse_s) || !aligned16(g) || !aligned16(dq) ||
-      !aligned16(dk) || (TEACHER && !aligned16(kl)))
-    return STREAMKL_ERR_MISALIGNED;
-  const int bh = B * H;
   const int d_g = TEACHER ? d_T : d_S;
-  const int g_g = TEACHER ? gT : gS;       // query heads per differentiated K head
-  const int bkv_g = B * (H / g_g);         // K heads of the differentiated side
+  const int h_kv_g = TEACHER ? P.H_kv_T : P.H_kv_S;  // K heads of the differentiated side
+  const long long dq_elems = P.q_rows() * (P.packed() ? (long long)P.H * d_g : d_g);
+  const long long dk_elems = P.k_rows(h_kv_g) * (P.packed() ? (long long)h_kv_g * d_g : d_g);
+  if ((dq_elems > 0 && !dq) || (dk_elems > 0 && !dk)) return STREAMKL_ERR_INVALID_ARG;
+  if ((dq && !aligned16(dq)) || (dk && !aligned16(dk))) return STREAMKL_ERR_MISALIGNED;
+  const bool launch = dq_elems > 0 && dk_elems > 0;  // packed: some rows and some keys
+  if (launch) {
+    if (!lse_t || !lse_s || !g || (TEACHER && !kl)) return STREAMKL_ERR_INVALID_ARG;
+    if (!aligned16(lse_t) || !aligned16(lse_s) || !aligned16(g) || (TEACHER && !aligned16(kl)))
+      return STREAMKL_ERR_MISALIGNED;
+  }
+  // dQ is accumulated with reduce-adds; dK too when K heads are shared, and packed dK rows
+  // outside every sequence are never written, so those outputs start from zero.
+  const bool dk_reduce = P.H / h_kv_g > 1;
+  if (dq_elems > 0 && cudaMemsetAsync(dq, 0, dq_elems * sizeof(float), stream) != cudaSuccess)
+    return STREAMKL_ERR_LAUNCH;
+  if (dk_elems > 0 && (dk_reduce || P.packed() || !launch) &&
+      cudaMemsetAsync(dk, 0, dk_elems * sizeof(float), stream) != cudaSuccess)
+    return STREAMKL_ERR_LAUNCH;
+  if (!launch) return STREAMKL_OK;
   CUtensorMap maps[6];
-  if (!make_map(&maps[0], q_t, d_T, N_Q, bh, 64) ||
-      !make_map(&maps[1], k_t, d_T, N_K, B * H_kv_T, 128) ||
-      !make_map(&maps[2], q_s, d_S, N_Q, bh, 64) ||
-      !make_map(&maps[3], k_s, d_S, N_K, B * H_kv_S, 128) ||
-      !make_map_f32(&maps[4], dq, d_g, N_Q, bh) || !make_map_f32(&maps[5], dk, d_g, N_K, bkv_g))
+  if (!map_of(&maps[0], q_t, P, d_T, false, 0, 64) ||
+      !map_of(&maps[1], k_t, P, d_T, true, P.H_kv_T, 128) ||
+      !map_of(&maps[2], q_s, P, d_S, false, 0, 64) ||
+      !map_of(&maps[3], k_s, P, d_S, true, P.H_kv_S, 128) ||
+      !map_of_f32(&maps[4], dq, P, d_g, false, 0) ||
+      !map_of_f32(&maps[5], dk, P, d_g, true, h_kv_g))
     return STREAMKL_ERR_LAUNCH;
-  if (cudaMemsetAsync(dq, 0, (size_t)bh * N_Q * d_g * sizeof(float), stream) != cudaSuccess)
-    return STREAMKL_ERR_LAUNCH;
-  if (g_g > 1 &&
-      cudaMemsetAsync(dk, 0, (size_t)bkv_g * N_K * d_g * sizeof(float), stream) != cudaSuccess)
-    return STREAMKL_ERR_LAUNCH;
+  const int bh = P.B * P.H;
   skl::BwdArgs a{};
   a.BH = bh;
-  a.N_Q = N_Q;
-  a.N_K = N_K;
+  a.N_Q = P.N_Q;
+  a.N_K = P.N_K;
   a.causal = causal ? 1 : 0;
-  a.off = N_K - N_Q;
   a.cT = std::fabs(scale_T) * kLog2e;
   a.cS = std::fabs(scale_S) * kLog2e;
   a.aT = std::fabs(scale_T);
   a.aS = std::fabs(scale_S);
   a.scale_G = TEACHER ? scale_T : scale_S;
-  a.n_ktiles = (N_K + 127) / 128;
-  a.n_qtiles = (N_Q + 63) / 64;
+  a.n_ktiles = (P.N_K + 127) / 128;
   a.group = head_group("STREAMKL_BWD_GROUP", 2, bh);
-  a.H = H;
-  a.gT = gT;
-  a.gS = gS;
-  a.dk_reduce = g_g > 1 ? 1 : 0;
+  a.H = P.H;
+  a.gT = P.H / P.H_kv_T;
+  a.gS = P.H / P.H_kv_S;
+  a.dk_reduce = dk_reduce ? 1 : 0;
+  a.cu_q = P.cu_q;
+  a.cu_k = P.cu_k;
+  a.total_q = P.total_q;
+  a.total_k = P.total_k;
+  a.dk_hs = P.packed() ? d_g : (long long)P.N_K * d_g;
+  a.dk_rs = P.packed() ? (long long)h_kv_g * d_g : d_g;
   a.lse_t = lse_t;
   a.lse_s = lse_s;
   a.g = g;
   a.kl = kl;
   a.dq = dq;
   a.dk = dk;
+  if (a.n_ktiles == 0) return STREAMKL_OK;  // packed, every sequence without keys
   const bool nT = scale_T < 0.f, nS = scale_S < 0.f;
   if (d_T == 128 && d_S == 128) return launch_bwd<128, 128, TEACHER>(maps, a, nT, nS, stream);
   if (d_T == 128 && d_S == 64) return launch_bwd<128, 64, TEACHER>(maps, a, nT, nS, stream);
   if (d_T == 64 && d_S == 128) return launch_bwd<64, 128, TEACHER>(maps, a, nT, nS, stream);
   return launch_bwd<64, 64, TEACHER>(maps, a, nT, nS, stream);
+}
+
+Problem dense(int B, int H, int H_kv_T, int H_kv_S, int N_Q, int N_K) {
+  Problem P;
+  P.B = B;
+  P.H = H;
+  P.H_kv_T = H_kv_T;
+  P.H_kv_S = H_kv_S;
+  P.N_Q = N_Q;
+  P.N_K = N_K;
+  return P;
+}
+
+Problem packed(const int* cu_q, const int* cu_k, int B, int H, int H_kv_T, int H_kv_S,
+               int total_q, int total_k, int max_q, int max_k) {
+  Problem P = dense(B, H, H_kv_T, H_kv_S, max_q, max_k);
+  P.total_q = total_q;
+  P.total_k = total_k;
+  P.cu_q = cu_q;  // non-null: the entry points reject null offsets before this
+  P.cu_k = cu_k;
+  return P;
 }
 
 }  // namespace
@@ -251,8 +336,8 @@ streamkl_status streamkl_fwd(const void* q_t, const void* k_t, const void* q_s, 
                              int B, int H, int N_Q, int N_K, int d_T, int d_S, float scale_T,
                              float scale_S, int causal, float* kl, float* lse_t, float* lse_s,
                              cudaStream_t stream) {
-  return fwd_common(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_T, d_S, scale_T, scale_S, causal,
-                    kl, lse_t, lse_s, stream);
+  return fwd_common(q_t, k_t, q_s, k_s, dense(B, H, H, H, N_Q, N_K), d_T, d_S, scale_T, scale_S,
+                    causal, kl, lse_t, lse_s, stream);
 }
 
 streamkl_status streamkl_fwd_gqa(const void* q_t, const void* k_t, const void* q_s,
@@ -260,16 +345,30 @@ streamkl_status streamkl_fwd_gqa(const void* q_t, const void* k_t, const void* q
                                  int N_K, int d_T, int d_S, float scale_T, float scale_S,
                                  int causal, float* kl, float* lse_t, float* lse_s,
                                  cudaStream_t stream) {
-  return fwd_common(q_t, k_t, q_s, k_s, B, H, H_kv_T, H_kv_S, N_Q, N_K, d_T, d_S, scale_T,
-                    scale_S, causal, kl, lse_t, lse_s, stream);
+  return fwd_common(q_t, k_t, q_s, k_s, dense(B, H, H_kv_T, H_kv_S, N_Q, N_K), d_T, d_S,
+                    scale_T, scale_S, causal, kl, lse_t, lse_s, stream);
+}
+
+streamkl_status streamkl_fwd_varlen(const void* q_t, const void* k_t, const void* q_s,
+                                    const void* k_s, const int* cu_seqlens_q,
+                                    const int* cu_seqlens_k, int B, int H, int H_kv_T,
+                                    int H_kv_S, int total_q, int total_k, int max_seqlen_q,
+                                    int max_seqlen_k, int d_T, int d_S, float scale_T,
+                                    float scale_S, int causal, float* kl, float* lse_t,
+                                    float* lse_s, cudaStream_t stream) {
+  if (!cu_seqlens_q || !cu_seqlens_k) return STREAMKL_ERR_INVALID_ARG;
+  return fwd_common(q_t, k_t, q_s, k_s,
+                    packed(cu_seqlens_q, cu_seqlens_k, B, H, H_kv_T, H_kv_S, total_q, total_k,
+                           max_seqlen_q, max_seqlen_k),
+                    d_T, d_S, scale_T, scale_S, causal, kl, lse_t, lse_s, stream);
 }
 
 streamkl_status streamkl_bwd(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
                              int B, int H, int N_Q, int N_K, int d_T, int d_S, float scale_T,
                              float scale_S, int causal, const float* lse_t, const float* lse_s,
                              const float* g, float* dq_s, float* dk_s, cudaStream_t stream) {
-  return bwd_common<false>(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_T, d_S, scale_T, scale_S,
-                           causal, nullptr, lse_t, lse_s, g, dq_s, dk_s, stream);
+  return bwd_common<false>(q_t, k_t, q_s, k_s, dense(B, H, H, H, N_Q, N_K), d_T, d_S, scale_T,
+                           scale_S, causal, nullptr, lse_t, lse_s, g, dq_s, dk_s, stream);
 }
 
 streamkl_status streamkl_bwd_gqa(const void* q_t, const void* k_t, const void* q_s,
@@ -277,8 +376,25 @@ streamkl_status streamkl_bwd_gqa(const void* q_t, const void* k_t, const void* q
                                  int N_K, int d_T, int d_S, float scale_T, float scale_S,
                                  int causal, const float* lse_t, const float* lse_s,
                                  const float* g, float* dq_s, float* dk_s, cudaStream_t stream) {
-  return bwd_common<false>(q_t, k_t, q_s, k_s, B, H, H_kv_T, H_kv_S, N_Q, N_K, d_T, d_S, scale_T,
-                           scale_S, causal, nullptr, lse_t, lse_s, g, dq_s, dk_s, stream);
+  return bwd_common<false>(q_t, k_t, q_s, k_s, dense(B, H, H_kv_T, H_kv_S, N_Q, N_K), d_T, d_S,
+                           scale_T, scale_S, causal, nullptr, lse_t, lse_s, g, dq_s, dk_s,
+                           stream);
+}
+
+streamkl_status streamkl_bwd_varlen(const void* q_t, const void* k_t, const void* q_s,
+                                    const void* k_s, const int* cu_seqlens_q,
+                                    const int* cu_seqlens_k, int B, int H, int H_kv_T,
+                                    int H_kv_S, int total_q, int total_k, int max_seqlen_q,
+                                    int max_seqlen_k, int d_T, int d_S, float scale_T,
+                                    float scale_S, int causal, const float* lse_t,
+                                    const float* lse_s, const float* g, float* dq_s,
+                                    float* dk_s, cudaStream_t stream) {
+  if (!cu_seqlens_q || !cu_seqlens_k) return STREAMKL_ERR_INVALID_ARG;
+  return bwd_common<false>(q_t, k_t, q_s, k_s,
+                           packed(cu_seqlens_q, cu_seqlens_k, B, H, H_kv_T, H_kv_S, total_q,
+                                  total_k, max_seqlen_q, max_seqlen_k),
+                           d_T, d_S, scale_T, scale_S, causal, nullptr, lse_t, lse_s, g, dq_s,
+                           dk_s, stream);
 }
 
 streamkl_status streamkl_bwd_teacher(const void* q_t, const void* k_t, const void* q_s,
@@ -287,8 +403,8 @@ streamkl_status streamkl_bwd_teacher(const void* q_t, const void* k_t, const voi
                                      const float* kl, const float* lse_t, const float* lse_s,
                                      const float* g, float* dq_t, float* dk_t,
                                      cudaStream_t stream) {
-  return bwd_common<true>(q_t, k_t, q_s, k_s, B, H, H, H, N_Q, N_K, d_T, d_S, scale_T, scale_S,
-                          causal, kl, lse_t, lse_s, g, dq_t, dk_t, stream);
+  return bwd_common<true>(q_t, k_t, q_s, k_s, dense(B, H, H, H, N_Q, N_K), d_T, d_S, scale_T,
+                          scale_S, causal, kl, lse_t, lse_s, g, dq_t, dk_t, stream);
 }
 
 streamkl_status streamkl_bwd_teacher_gqa(const void* q_t, const void* k_t, const void* q_s,
@@ -297,14 +413,28 @@ streamkl_status streamkl_bwd_teacher_gqa(const void* q_t, const void* k_t, const
                                          float scale_S, int causal, const float* kl,
                                          const float* lse_t, const float* lse_s, const float* g,
                                          float* dq_t, float* dk_t, cudaStream_t stream) {
-  return bwd_common<true>(q_t, k_t, q_s, k_s, B, H, H_kv_T, H_kv_S, N_Q, N_K, d_T, d_S, scale_T,
-                          scale_S, causal, kl, lse_t, lse_s, g, dq_t, dk_t, stream);
+  return bwd_common<true>(q_t, k_t, q_s, k_s, dense(B, H, H_kv_T, H_kv_S, N_Q, N_K), d_T, d_S,
+                          scale_T, scale_S, causal, kl, lse_t, lse_s, g, dq_t, dk_t, stream);
+}
+
+streamkl_status streamkl_bwd_teacher_varlen(
+    const void* q_t, const void* k_t, const void* q_s, const void* k_s, const int* cu_seqlens_q,
+    const int* cu_seqlens_k, int B, int H, int H_kv_T, int H_kv_S, int total_q, int total_k,
+    int max_seqlen_q, int max_seqlen_k, int d_T, int d_S, float scale_T, float scale_S,
+    int causal, const float* kl, const float* lse_t, const float* lse_s, const float* g,
+    float* dq_t, float* dk_t, cudaStream_t stream) {
+  if (!cu_seqlens_q || !cu_seqlens_k) return STREAMKL_ERR_INVALID_ARG;
+  return bwd_common<true>(q_t, k_t, q_s, k_s,
+                          packed(cu_seqlens_q, cu_seqlens_k, B, H, H_kv_T, H_kv_S, total_q,
+                                 total_k, max_seqlen_q, max_seqlen_k),
+                          d_T, d_S, scale_T, scale_S, causal, kl, lse_t, lse_s, g, dq_t, dk_t,
+                          stream);
 }
 
 const char* streamkl_status_string(streamkl_status s) {
   switch (s) {
     case STREAMKL_OK: return "ok";
-    case STREAMKL_ERR_INVALID_ARG: return "invalid argument (null pointer, size < 1 or non-finite scale)";
+    case STREAMKL_ERR_INVALID_ARG: return "invalid argument (null pointer, size out of range, non-finite scale or malformed packed-sequence offsets)";
     case STREAMKL_ERR_UNSUPPORTED: return "unsupported shape (head dims must be 64 or 128; sizes beyond limits)";
     case STREAMKL_ERR_MISALIGNED: return "pointer not 16-byte aligned";
     case STREAMKL_ERR_LAUNCH: return "CUDA runtime error during set-up or launch";
@@ -322,11 +452,13 @@ streamkl_status streamkl_device_status(cudaStream_t stream) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(skl::g_skl_error, &zero, sizeof(zero)) != cudaSuccess)
       return STREAMKL_ERR_LAUNCH;
-    return STREAMKL_ERR_TIMEOUT;
+    // Malformed packed offsets are an argument error found on the device; every other
+    // bit is a watchdog (or the never-expected shared-memory alignment check).
+    return v == skl::kErrBadOffsets ? STREAMKL_ERR_INVALID_ARG : STREAMKL_ERR_TIMEOUT;
   }
   return STREAMKL_OK;
 }
 
-int streamkl_version(void) { return 100; }
+int streamkl_version(void) { return 200; }
 
 }  // extern "C"

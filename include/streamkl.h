@@ -49,7 +49,8 @@ extern "C" {
 
 typedef enum {
   STREAMKL_OK = 0,
-  STREAMKL_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, non-finite scale */
+  STREAMKL_ERR_INVALID_ARG = 1, /* null pointer, size out of range, non-finite scale,
+                                   malformed packed-sequence offsets (device-detected) */
   STREAMKL_ERR_UNSUPPORTED = 2, /* head dim outside {64,128} or sizes beyond the limits */
   STREAMKL_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned */
   STREAMKL_ERR_LAUNCH = 4,      /* the CUDA runtime rejected a launch or a set-up call */
@@ -138,13 +139,62 @@ streamkl_status streamkl_bwd_teacher_gqa(const void* q_t, const void* k_t, const
                                          const float* lse_t, const float* lse_s, const float* g,
                                          float* dq_t, float* dk_t, cudaStream_t stream);
 
+/*
+ * Packed variable-length sequences (the "varlen" layout). B sequences of different
+ * lengths are packed token-major into one tensor each:
+ *   q_t [total_q,H,d_T], q_s [total_q,H,d_S], k_t [total_k,H_kv_T,d_T], k_s [total_k,H_kv_S,d_S]
+ * (contiguous bf16; H_kv_* as in the GQA variants, H_kv = H for one K head per query head).
+ * cu_seqlens_q / cu_seqlens_k are DEVICE int32 arrays of B+1 offsets (4-byte aligned):
+ * sequence b owns query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and key rows
+ * cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1. max_seqlen_q / max_seqlen_k bound every
+ * sequence's length (they size the grid). Each sequence is its own problem: its queries
+ * see only its keys, and causal alignment is bottom-right within the sequence
+ * (j <= i + n_k(b) - n_q(b), with i, j counted from the sequence's first row).
+ * Row statistics, kl and g are fp32 [H, total_q] (head-major); gradients are fp32 in the
+ * packed shapes of Q and K of the differentiated side.
+ * - Sequences may be empty; a sequence with queries but no keys gets KL = 0, LSE = -inf.
+ * - total_q, total_k >= 0; H*total_q, H*total_k < 2^31. With total_q = 0 the forward
+ *   writes nothing; the backward zeroes its outputs and launches nothing when total_q or
+ *   total_k is 0.
+ * - kl / lse_* rows that belong to no sequence are not written; dq / dk are zeroed on
+ *   `stream` first, so their rows outside every sequence are 0. dk is accumulated with
+ *   fp32 reductions in L2 when K heads are shared, as in the GQA variants.
+ * - The offsets are read on the device. Offsets that are not 0 <= cu[b] <= cu[b+1] <= total
+ *   or describe a sequence longer than max_seqlen_* make the kernels skip that sequence
+ *   and record STREAMKL_ERR_INVALID_ARG in the device error word (streamkl_device_status).
+ */
+streamkl_status streamkl_fwd_varlen(const void* q_t, const void* k_t, const void* q_s,
+                                    const void* k_s, const int* cu_seqlens_q,
+                                    const int* cu_seqlens_k, int B, int H, int H_kv_T,
+                                    int H_kv_S, int total_q, int total_k, int max_seqlen_q,
+                                    int max_seqlen_k, int d_T, int d_S, float scale_T,
+                                    float scale_S, int causal, float* kl, float* lse_t,
+                                    float* lse_s, cudaStream_t stream);
+
+streamkl_status streamkl_bwd_varlen(const void* q_t, const void* k_t, const void* q_s,
+                                    const void* k_s, const int* cu_seqlens_q,
+                                    const int* cu_seqlens_k, int B, int H, int H_kv_T,
+                                    int H_kv_S, int total_q, int total_k, int max_seqlen_q,
+                                    int max_seqlen_k, int d_T, int d_S, float scale_T,
+                                    float scale_S, int causal, const float* lse_t,
+                                    const float* lse_s, const float* g, float* dq_s,
+                                    float* dk_s, cudaStream_t stream);
+
+streamkl_status streamkl_bwd_teacher_varlen(
+    const void* q_t, const void* k_t, const void* q_s, const void* k_s, const int* cu_seqlens_q,
+    const int* cu_seqlens_k, int B, int H, int H_kv_T, int H_kv_S, int total_q, int total_k,
+    int max_seqlen_q, int max_seqlen_k, int d_T, int d_S, float scale_T, float scale_S,
+    int causal, const float* kl, const float* lse_t, const float* lse_s, const float* g,
+    float* dq_t, float* dk_t, cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char* streamkl_status_string(streamkl_status status);
 
 /*
  * Synchronises `stream`, then reads and clears the current device's error word.
- * Returns STREAMKL_OK, STREAMKL_ERR_TIMEOUT if a kernel watchdog fired since the last
- * call, or STREAMKL_ERR_LAUNCH if the stream reports a CUDA error.
+ * Returns STREAMKL_OK, STREAMKL_ERR_INVALID_ARG if a varlen kernel found malformed
+ * sequence offsets, STREAMKL_ERR_TIMEOUT if a kernel watchdog fired since the last call,
+ * or STREAMKL_ERR_LAUNCH if the stream reports a CUDA error.
  */
 streamkl_status streamkl_device_status(cudaStream_t stream);
 

@@ -116,3 +116,58 @@ def test_host_validation_outputs(lib):
     assert bwd_teacher(kl=0) == 1
     assert bwd_teacher(kl=P + 4) == 3
     assert bwd_teacher(dk_t=P + 8) == 3
+
+
+def fwd_varlen(lib, **kw):
+    a = dict(q_t=P, k_t=P, q_s=P, k_s=P, cu_q=P, cu_k=P, B=2, H=4, H_kv_T=4, H_kv_S=2,
+             total_q=300, total_k=280, max_q=200, max_k=200, d_T=128, d_S=64, scale_T=0.1,
+             scale_S=0.1, causal=1, kl=P, lse_t=P, lse_s=P, stream=0)
+    a.update(kw)
+    return lib.streamkl_fwd_varlen(*a.values())
+
+
+def bwd_varlen(lib, teacher=False, **kw):
+    a = dict(q_t=P, k_t=P, q_s=P, k_s=P, cu_q=P, cu_k=P, B=2, H=4, H_kv_T=4, H_kv_S=2,
+             total_q=300, total_k=280, max_q=200, max_k=200, d_T=128, d_S=64, scale_T=0.1,
+             scale_S=0.1, causal=1)
+    if teacher:
+        a["kl"] = P
+    a.update(dict(lse_t=P, lse_s=P, g=P, dq=P, dk=P, stream=0))
+    a.update(kw)
+    fn = lib.streamkl_bwd_teacher_varlen if teacher else lib.streamkl_bwd_varlen
+    return fn(*a.values())
+
+
+@pytest.mark.parametrize("call", ["fwd", "bwd", "bwd_teacher"])
+def test_varlen_host_validation(lib, call):
+    fn = {"fwd": lambda **kw: fwd_varlen(lib, **kw),
+          "bwd": lambda **kw: bwd_varlen(lib, **kw),
+          "bwd_teacher": lambda **kw: bwd_varlen(lib, teacher=True, **kw)}[call]
+    assert fn(cu_q=0) == 1
+    assert fn(cu_k=0) == 1
+    assert fn(B=0) == 1
+    assert fn(total_q=-1) == 1
+    assert fn(total_k=-3) == 1
+    assert fn(max_q=-1) == 1
+    assert fn(q_t=0) == 1                       # rows but no Q
+    assert fn(k_s=0) == 1                       # keys but no K
+    assert fn(scale_S=float("nan")) == 1
+    assert fn(d_T=96) == 2
+    assert fn(H_kv_T=3) == 2                    # 3 does not divide 4
+    assert fn(H=64, H_kv_T=64, H_kv_S=64, total_q=1 << 25) == 2   # H*total_q >= 2^31
+    assert fn(cu_q=P + 2) == 3
+    assert fn(k_t=P + 8) == 3
+
+
+def test_varlen_host_validation_outputs(lib):
+    assert fwd_varlen(lib, kl=0) == 1
+    assert fwd_varlen(lib, lse_t=P + 4) == 3
+    assert bwd_varlen(lib, g=0) == 1
+    assert bwd_varlen(lib, dq=0) == 1
+    assert bwd_varlen(lib, dk=P + 4) == 3
+    assert bwd_varlen(lib, teacher=True, kl=0) == 1
+
+
+def test_varlen_without_query_rows_is_a_no_op(lib):
+    # No query rows: nothing to compute or write, so no CUDA call is made at all.
+    assert fwd_varlen(lib, q_t=0, q_s=0, kl=0, lse_t=0, lse_s=0, total_q=0, max_q=0) == 0

@@ -270,3 +270,121 @@ def _sampled(w, rows_n=256, dk_heads=2, dk_keys=64):
 def test_full_size_workload(name):
     w = WORKLOADS[name]
     _sampled(w, dk_heads=1 if w.N_K > 20000 else 2)
+
+
+# ------------------------------------------------ packed variable-length sequences
+
+from oracle import oracle_bwd_teacher_varlen, oracle_bwd_varlen, oracle_fwd_varlen  # noqa: E402
+from workloads import make_varlen_inputs, varlen_lengths  # noqa: E402
+
+# equal lengths, keys but no queries, a query with no keys, n_q > n_k (empty causal rows),
+# n_q < n_k, several tiles with a ragged tail
+VARLEN_Q = [300, 0, 1, 257, 64, 130]
+VARLEN_K = [300, 5, 0, 200, 190, 130]
+
+
+def run_varlen(x, H, scale_t, scale_s, causal, teacher=False):
+    d = {k: v.cuda() for k, v in x.items()}
+    mq = int((x["cu_q"][1:] - x["cu_q"][:-1]).max())
+    mk = int((x["cu_k"][1:] - x["cu_k"][:-1]).max())
+    a = (d["q_t"], d["k_t"], d["q_s"], d["k_s"], d["cu_q"], d["cu_k"], mq, mk, scale_t, scale_s,
+         causal)
+    kl, lt, ls = skl.streamkl_fwd_varlen(*a)
+    dq, dk = skl.streamkl_bwd_varlen(*a, lt, ls, d["g"])
+    out = {"kl": kl, "lse_t": lt, "lse_s": ls, "dq": dq, "dk": dk}
+    if teacher:
+        out["dq_t"], out["dk_t"] = skl.streamkl_bwd_teacher_varlen(*a, kl, lt, ls, d["g"])
+    assert skl.device_status() == 0
+    return {k: v.cpu().double() for k, v in out.items()}
+
+
+@pytest.mark.parametrize("H,hkt,hks,dt,ds,causal", [
+    (4, 4, 4, 128, 128, True), (4, 4, 4, 128, 128, False), (4, 2, 1, 128, 64, True),
+    (4, 1, 4, 64, 64, False), (2, 2, 2, 64, 128, True)])
+def test_varlen_full(H, hkt, hks, dt, ds, causal):
+    x = make_varlen_inputs(VARLEN_Q, VARLEN_K, H, hkt, hks, dt, ds, seed=41 + dt + hks)
+    st, ss = 1 / math.sqrt(dt), 1 / math.sqrt(ds)
+    g = run_varlen(x, H, st, ss, causal, teacher=True)
+    args = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], x["cu_q"].tolist(), x["cu_k"].tolist(), st,
+            ss, causal)
+    kl, lt, ls = oracle_fwd_varlen(*args)
+    check_kl(g["kl"], kl)
+    check_lse(g["lse_t"], lt)
+    check_lse(g["lse_s"], ls)
+    dq, dk = oracle_bwd_varlen(*args, x["g"])
+    assert rel_fro(g["dq"], dq) <= GRAD_REL, rel_fro(g["dq"], dq)
+    assert rel_fro(g["dk"], dk) <= GRAD_REL, rel_fro(g["dk"], dk)
+    dqt, dkt = oracle_bwd_teacher_varlen(*args, x["g"])
+    assert rel_fro(g["dq_t"], dqt) <= GRAD_REL, rel_fro(g["dq_t"], dqt)
+    assert rel_fro(g["dk_t"], dkt) <= GRAD_REL, rel_fro(g["dk_t"], dkt)
+    # the query without keys and the sequence without queries
+    q2 = int(x["cu_q"][2])
+    assert torch.all(g["kl"][:, q2] == 0) and torch.all(torch.isinf(g["lse_t"][:, q2]))
+    k1, k2 = int(x["cu_k"][1]), int(x["cu_k"][2])
+    assert torch.all(g["dk"][k1:k2] == 0) and torch.all(g["dk_t"][k1:k2] == 0)
+
+
+def test_varlen_one_sequence_equals_dense():
+    w = WORKLOADS["b2h16_n4096_d128_causal"]
+    x = make_varlen_inputs([700], [700], 4, 4, 4, 128, 128, seed=5)
+    g = run_varlen(x, 4, w.scale_T, w.scale_S, True)
+    dense = {k: x[k].permute(1, 0, 2).unsqueeze(0).contiguous().cuda()
+             for k in ("q_t", "k_t", "q_s", "k_s")}
+    kl, lt, ls = skl.streamkl_fwd(dense["q_t"], dense["k_t"], dense["q_s"], dense["k_s"],
+                                  w.scale_T, w.scale_S, True)
+    dq, dk = skl.streamkl_bwd(dense["q_t"], dense["k_t"], dense["q_s"], dense["k_s"], w.scale_T,
+                              w.scale_S, True, lt, ls, x["g"].unsqueeze(0).contiguous().cuda())
+    assert skl.device_status() == 0
+    # same tiles in the same order: the forward is bitwise identical
+    assert torch.equal(g["kl"], kl[0].cpu().double())
+    assert torch.equal(g["lse_t"], lt[0].cpu().double())
+    assert torch.equal(g["dk"], dk[0].permute(1, 0, 2).cpu().double())
+    assert rel_fro(g["dq"], dq[0].permute(1, 0, 2).cpu().double()) < 1e-6
+
+
+def test_varlen_degenerate_totals():
+    H = 2
+    # no query rows at all: nothing is written, dK is zero
+    x = make_varlen_inputs([0, 0], [50, 70], H, H, H, 64, 64, seed=3)
+    g = run_varlen(x, H, 0.125, 0.125, True)
+    assert g["kl"].numel() == 0 and g["dq"].numel() == 0 and torch.all(g["dk"] == 0)
+    # no keys at all: every row has KL 0 and LSE -inf, dQ is zero
+    x = make_varlen_inputs([40, 90], [0, 0], H, H, H, 64, 64, seed=4)
+    g = run_varlen(x, H, 0.125, 0.125, False)
+    assert torch.all(g["kl"] == 0) and torch.all(g["lse_s"] == float("-inf"))
+    assert torch.all(g["dq"] == 0) and g["dk"].numel() == 0
+
+
+def test_varlen_malformed_offsets_reported_on_device():
+    H = 2
+    x = make_varlen_inputs([100, 100, 100], [100, 100, 100], H, H, H, 64, 64, seed=8)
+    d = {k: v.cuda() for k, v in x.items()}
+    bad = torch.tensor([0, 200, 100, 300], dtype=torch.int32, device="cuda")  # decreasing
+    kl, _, _ = skl.streamkl_fwd_varlen(d["q_t"], d["k_t"], d["q_s"], d["k_s"], bad, d["cu_k"],
+                                       200, 100, 0.125, 0.125, False)
+    assert skl.device_status() == 1  # STREAMKL_ERR_INVALID_ARG
+    # a sequence longer than max_seqlen_q
+    kl, _, _ = skl.streamkl_fwd_varlen(d["q_t"], d["k_t"], d["q_s"], d["k_s"], d["cu_q"],
+                                       d["cu_k"], 64, 100, 0.125, 0.125, False)
+    assert skl.device_status() == 1
+    # the context is still usable and the status was cleared
+    g = run_varlen(x, H, 0.125, 0.125, True)
+    kl_r, _, _ = oracle_fwd_varlen(x["q_t"], x["k_t"], x["q_s"], x["k_s"], x["cu_q"].tolist(),
+                                   x["cu_k"].tolist(), 0.125, 0.125, True)
+    check_kl(g["kl"], kl_r)
+
+
+def test_varlen_length_mix_sampled():
+    """A packed batch with the length mix of the benchmark (seeded lengths 64..2048,
+    8192 tokens): every output row checked against the oracle."""
+    lens = varlen_lengths(8192, 64, 2048, seed=77)
+    x = make_varlen_inputs(lens, lens, 4, 4, 2, 128, 128, seed=78)
+    st = ss = 1 / math.sqrt(128)
+    g = run_varlen(x, 4, st, ss, True)
+    args = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], x["cu_q"].tolist(), x["cu_k"].tolist(), st,
+            ss, True)
+    kl, lt, ls = oracle_fwd_varlen(*args)
+    check_kl(g["kl"], kl)
+    check_lse(g["lse_s"], ls)
+    dq, dk = oracle_bwd_varlen(*args, x["g"])
+    assert rel_fro(g["dq"], dq) <= GRAD_REL and rel_fro(g["dk"], dk) <= GRAD_REL

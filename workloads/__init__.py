@@ -174,3 +174,62 @@ def allowed_pairs(w: Workload) -> float:
     as the throughput convention of attention kernels does.
     """
     return w.N_Q * w.N_K / (2.0 if w.causal else 1.0)
+
+
+# ------------------------------------------------ packed variable-length sequences
+
+def varlen_lengths(total: int, min_len: int, max_len: int, seed: int):
+    """Seeded sequence lengths, uniform in [min_len, max_len], summing to ``total``
+    (the last one is cut to fit): the length mix of a packed training batch."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    lens, left = [], total
+    while left > 0:
+        n = int(torch.randint(min_len, max_len + 1, (1,), generator=gen))
+        n = min(n, left)
+        lens.append(n)
+        left -= n
+    return lens
+
+
+def cu_seqlens(lens):
+    """[B+1] int32 offsets of packed sequences with the given lengths."""
+    out = [0]
+    for n in lens:
+        out.append(out[-1] + int(n))
+    return torch.tensor(out, dtype=torch.int32)
+
+
+def make_varlen_inputs(lens_q, lens_k, H: int, H_kv_T: int, H_kv_S: int, d_T: int, d_S: int,
+                       seed: int, sigma: Optional[float] = 0.3) -> Dict[str, torch.Tensor]:
+    """Packed inputs: q_* [total_q, H, d], k_* [total_k, H_kv, d] (bf16), g [H, total_q]
+    fp32 U(0, 1) and the offsets cu_q, cu_k (int32 [B+1]).
+
+    The student is the teacher plus sigma * N(0, 1) when the shapes allow it (same head
+    dims and K head counts; sigma not None), else an independent N(0, 1) draw. Draw order:
+    Q_T, K_T, then (noise_Q, noise_K) or (Q_S, K_S), then g.
+    """
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    tq, tk = int(sum(lens_q)), int(sum(lens_k))
+
+    def normal(*shape):
+        return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+    q_t = normal(tq, H, d_T).to(torch.bfloat16)
+    k_t = normal(tk, H_kv_T, d_T).to(torch.bfloat16)
+    if sigma is not None and d_S == d_T and H_kv_S == H_kv_T:
+        q_s = (q_t.float() + sigma * normal(tq, H, d_S)).to(torch.bfloat16)
+        k_s = (k_t.float() + sigma * normal(tk, H_kv_S, d_S)).to(torch.bfloat16)
+    else:
+        q_s = normal(tq, H, d_S).to(torch.bfloat16)
+        k_s = normal(tk, H_kv_S, d_S).to(torch.bfloat16)
+    g = torch.rand(H, tq, generator=gen, dtype=torch.float32)
+    return {"q_t": q_t, "k_t": k_t, "q_s": q_s, "k_s": k_s, "g": g,
+            "cu_q": cu_seqlens(lens_q), "cu_k": cu_seqlens(lens_k)}
+
+
+def varlen_pairs(lens_q, lens_k, causal: bool) -> float:
+    """(i, j) pairs per head counted for FLOPs: per sequence n_q*n_k, halved when causal
+    (the same convention as allowed_pairs)."""
+    return sum(a * b / (2.0 if causal else 1.0) for a, b in zip(lens_q, lens_k))
