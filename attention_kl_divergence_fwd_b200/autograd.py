@@ -8,6 +8,10 @@ backward); the backward calls ``streamkl_bwd`` with g = dLoss/dKL per row, which
 reduction determines: 1 for "sum", 1/(B*H*N_Q) for "mean", 1/B for "batchmean". Only
 the O(B*H*N_Q) row vector is touched by PyTorch; every O(N_Q*N_K) step runs in the CUDA
 kernels and nothing of that size is ever allocated.
+
+Packed variable-length batches use ``attention_kl_varlen`` / ``attention_kl_varlen_loss``
+(q_* [total_q, H, d], k_* [total_k, H_kv, d], int32 cu_seqlens on the device); there
+"batchmean" divides by the number of sequences.
 """
 from __future__ import annotations
 
@@ -17,7 +21,8 @@ from typing import Optional
 import torch
 
 from . import (streamkl_bwd, streamkl_bwd_gqa, streamkl_bwd_teacher, streamkl_bwd_teacher_gqa,
-               streamkl_fwd, streamkl_fwd_gqa)
+               streamkl_bwd_teacher_varlen, streamkl_bwd_varlen, streamkl_fwd, streamkl_fwd_gqa,
+               streamkl_fwd_varlen)
 
 REDUCTIONS = ("none", "sum", "mean", "batchmean")
 
@@ -92,3 +97,64 @@ def attention_kl_loss(q_t, k_t, q_s, k_s, scale_t: Optional[float] = None,
     if reduction not in REDUCTIONS:
         raise ValueError(f"reduction must be one of {REDUCTIONS}, got {reduction!r}")
     return reduce_kl(attention_kl(q_t, k_t, q_s, k_s, scale_t, scale_s, causal), reduction)
+
+
+class StreamKLVarlenFunction(torch.autograd.Function):
+    """Row-wise KL over packed variable-length sequences; KL is [H, total_q]."""
+
+    @staticmethod
+    def forward(ctx, q_t, k_t, q_s, k_s, cu_q, cu_k, max_q: int, max_k: int, scale_t: float,
+                scale_s: float, causal: bool):
+        H, tq = q_t.shape[1], q_t.shape[0]
+        # Rows that belong to no sequence are not written by the kernel: start them at 0
+        # (KL) so that reductions over the whole tensor ignore them.
+        kl = torch.zeros(H, tq, device=q_t.device, dtype=torch.float32)
+        kl, lse_t, lse_s = streamkl_fwd_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, max_q, max_k,
+                                               scale_t, scale_s, causal, kl=kl)
+        ctx.save_for_backward(q_t, k_t, q_s, k_s, cu_q, cu_k, kl, lse_t, lse_s)
+        ctx.params = (max_q, max_k, scale_t, scale_s, causal)
+        ctx.mark_non_differentiable(lse_t, lse_s)
+        return kl, lse_t, lse_s
+
+    @staticmethod
+    def backward(ctx, g_kl, _g_lse_t=None, _g_lse_s=None):
+        q_t, k_t, q_s, k_s, cu_q, cu_k, kl, lse_t, lse_s = ctx.saved_tensors
+        a = (q_t, k_t, q_s, k_s, cu_q, cu_k) + ctx.params
+        g = g_kl.detach().to(torch.float32).contiguous()
+        dq_t = dk_t = dq_s = dk_s = None
+        if ctx.needs_input_grad[2] or ctx.needs_input_grad[3]:
+            dq_s, dk_s = streamkl_bwd_varlen(*a, lse_t, lse_s, g)
+            dq_s, dk_s = dq_s.to(q_s.dtype), dk_s.to(k_s.dtype)
+        if ctx.needs_input_grad[0] or ctx.needs_input_grad[1]:
+            dq_t, dk_t = streamkl_bwd_teacher_varlen(*a, kl, lse_t, lse_s, g)
+            dq_t, dk_t = dq_t.to(q_t.dtype), dk_t.to(k_t.dtype)
+        return dq_t, dk_t, dq_s, dk_s, None, None, None, None, None, None, None
+
+
+def attention_kl_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                        max_seqlen_k: int, scale_t: Optional[float] = None,
+                        scale_s: Optional[float] = None, causal: bool = False):
+    """Per-row KL [H, total_q] (fp32) of packed sequences, differentiable like
+    ``attention_kl``. Rows outside every sequence are 0."""
+    scale_t = 1.0 / math.sqrt(q_t.shape[-1]) if scale_t is None else float(scale_t)
+    scale_s = 1.0 / math.sqrt(q_s.shape[-1]) if scale_s is None else float(scale_s)
+    kl, _, _ = StreamKLVarlenFunction.apply(
+        q_t.contiguous(), k_t.contiguous(), q_s.contiguous(), k_s.contiguous(),
+        cu_seqlens_q.to(torch.int32).contiguous(), cu_seqlens_k.to(torch.int32).contiguous(),
+        int(max_seqlen_q), int(max_seqlen_k), scale_t, scale_s, bool(causal))
+    return kl
+
+
+def attention_kl_varlen_loss(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                             max_seqlen_k: int, scale_t: Optional[float] = None,
+                             scale_s: Optional[float] = None, causal: bool = False,
+                             reduction: str = "mean") -> torch.Tensor:
+    """Reduction of the packed row-wise KL: "mean" over the H*total_q rows, "batchmean"
+    divided by the number of sequences B."""
+    if reduction not in REDUCTIONS:
+        raise ValueError(f"reduction must be one of {REDUCTIONS}, got {reduction!r}")
+    kl = attention_kl_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                             max_seqlen_k, scale_t, scale_s, causal)
+    if reduction == "batchmean":
+        return kl.sum() / (cu_seqlens_q.numel() - 1)
+    return reduce_kl(kl, reduction)

@@ -29,7 +29,8 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from workloads import WORKLOADS, flops_bwd, flops_bwd_teacher, flops_fwd, make_inputs  # noqa: E402
+from workloads import (WORKLOADS, flops_bwd, flops_bwd_teacher, flops_fwd, make_inputs,  # noqa: E402
+                       make_varlen_inputs, varlen_lengths, varlen_pairs)
 
 METRIC = "fwd/bwd TFLOP/s and % of B200 bf16 peak at N=16K,d=128; ms per fwd+bwd"
 DEFAULT_WORKLOAD = "long_b1h32_n16384_d128_causal"
@@ -335,6 +336,8 @@ def main():
                "fwd_tflops": ff / (gf * 1e-3) / 1e12, "bwd_tflops": fb / (gb * 1e-3) / 1e12}
         del k_s4, dk4
 
+    varlen = run_varlen(skl, w, dev, stream, args.steps, world) if w.d_T == w.d_S else None
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(skl, w, x, dev, stream, args.steps, world)
@@ -353,7 +356,7 @@ def main():
                "fwd_frac_burst_peak": fwd_tf / peak_burst,
                "bwd_frac_burst_peak": bwd_tf / peak_burst,
                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-               "gqa": gqa,
+               "gqa": gqa, "varlen": varlen,
                "bwd_teacher_ms": bwd_t_ms,
                "bwd_teacher_tflops": flops_bwd_teacher(w) / (bwd_t_ms * 1e-3) / 1e12,
                "gpu_launches": 2 * args.steps,
@@ -363,6 +366,42 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_varlen(skl, w, dev, stream, steps, world, tokens=65536, lo=512, hi=8192):
+    """Packed variable-length batch with the workload's heads and head dims: seeded
+    sequence lengths uniform in [lo, hi] filling ``tokens`` rows, timed on its own."""
+    lens = varlen_lengths(tokens, lo, hi, seed=2024)
+    x = make_varlen_inputs(lens, lens, w.H, w.H, w.H, w.d_T, w.d_S, seed=2025)
+    d = {k: v.to(dev) for k, v in x.items()}
+    a = (d["q_t"], d["k_t"], d["q_s"], d["k_s"], d["cu_q"], d["cu_k"], max(lens), max(lens),
+         w.scale_T, w.scale_S, w.causal)
+    kl = torch.empty(w.H, tokens, device=dev)
+    lt, ls = torch.empty_like(kl), torch.empty_like(kl)
+    dq = torch.empty(tokens, w.H, w.d_S, device=dev)
+    dk = torch.empty(tokens, w.H, w.d_S, device=dev)
+    for _ in range(3):
+        skl.streamkl_fwd_varlen(*a, kl=kl, lse_t=lt, lse_s=ls)
+        skl.streamkl_bwd_varlen(*a, lt, ls, d["g"], dq_s=dq, dk_s=dk)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record(stream)
+    for _ in range(steps):
+        skl.streamkl_fwd_varlen(*a, kl=kl, lse_t=lt, lse_s=ls)
+    ev[1].record(stream)
+    for _ in range(steps):
+        skl.streamkl_bwd_varlen(*a, lt, ls, d["g"], dq_s=dq, dk_s=dk)
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    if skl.device_status() != 0:
+        raise RuntimeError("kernel watchdog fired in the packed-sequence run")
+    fms = max_over_ranks(ev[0].elapsed_time(ev[1]) / steps, world)
+    bms = max_over_ranks(ev[1].elapsed_time(ev[2]) / steps, world)
+    pairs = varlen_pairs(lens, lens, w.causal) * w.H
+    ff, fb = 2 * pairs * (w.d_T + w.d_S), 2 * pairs * (w.d_T + 3 * w.d_S)
+    return {"tokens": tokens, "sequences": len(lens), "lengths": f"seeded uniform {lo}..{hi}",
+            "fwd_ms": fms, "bwd_ms": bms, "fwd_tflops": ff / (fms * 1e-3) / 1e12,
+            "bwd_tflops": fb / (bms * 1e-3) / 1e12}
 
 
 def run_e2e(skl, w, x, dev, stream, steps, world):

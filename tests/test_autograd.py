@@ -75,3 +75,31 @@ def test_default_scales_and_frozen_teacher():
     kl2 = ska.attention_kl(d["q_t"], d["k_t"], d["q_s"], d["k_s"], 1 / math.sqrt(64),
                            1 / math.sqrt(64))
     assert torch.equal(kl.detach(), kl2)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("reduction", ["mean", "batchmean"])
+def test_varlen_loss_and_grads_match_oracle(reduction):
+    from oracle import oracle_bwd_teacher_varlen, oracle_bwd_varlen, oracle_fwd_varlen
+    from workloads import make_varlen_inputs
+    lens_q, lens_k = [150, 0, 270, 33], [150, 20, 200, 80]
+    x = make_varlen_inputs(lens_q, lens_k, 4, 2, 4, 128, 64, seed=31)
+    d = {k: v.cuda() for k, v in x.items()}
+    q_t = d["q_t"].clone().requires_grad_(True)
+    q_s = d["q_s"].clone().requires_grad_(True)
+    k_s = d["k_s"].clone().requires_grad_(True)
+    st, ss = 0.09, 0.125
+    loss = ska.attention_kl_varlen_loss(q_t, d["k_t"], q_s, k_s, d["cu_q"], d["cu_k"], 270, 200,
+                                        st, ss, True, reduction)
+    loss.backward()
+    args = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], x["cu_q"].tolist(), x["cu_k"].tolist(), st,
+            ss, True)
+    kl, _, _ = oracle_fwd_varlen(*args)
+    g = 1.0 / kl.numel() if reduction == "mean" else 1.0 / len(lens_q)
+    assert abs(loss.item() - kl.sum().item() * g) <= 1e-4 * max(1.0, abs(kl.sum().item() * g))
+    gg = torch.full_like(x["g"], g)
+    rel = lambda a, b: ((a.double().cpu() - b).norm() / b.norm()).item()
+    dq, dk = oracle_bwd_varlen(*args, gg)
+    assert rel(q_s.grad, dq) < 1.5e-2 and rel(k_s.grad, dk) < 1.5e-2
+    dqt, _ = oracle_bwd_teacher_varlen(*args, gg)
+    assert rel(q_t.grad, dqt) < 1.5e-2
