@@ -388,3 +388,127 @@ def oracle_bwd_teacher_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, scale_t, scale_s, 
     """dQ_T [total_q, H, d_T], dK_T [total_k, H_kv_T, d_T] (float64); g is [H, total_q]."""
     return _bwd_varlen(oracle_bwd_teacher_gqa, q_t, k_t, q_s, k_s, cu_q, cu_k, scale_t,
                        scale_s, causal, g, "teacher", row_block)
+
+
+# ------------------------------------------------ context parallelism over N_K
+#
+# The keys of a sequence (N_K_total of them) are split into contiguous shards; shard r
+# holds keys k_offset .. k_offset + n_shard - 1. Per query row, a shard summarises what it
+# saw in a state, in base-2 units (t_X = s_X / ln 2):
+#   m_X = max_j t_X[j],   l_X = sum_j 2^(t_X[j] - m_X)      (X = T, S)
+#   A   = sum_j 2^(t_T[j] - m_T) * (t_T[j] - t_S[j])
+# over the shard's allowed keys (global index j allowed iff j <= i + N_K_total - N_Q when
+# causal); a row with no allowed key in the shard has m = -inf, l = 0, A = 0. States merge
+# by rescaling to the larger maximum and adding, which is associative, and the merged
+# state gives LSE_X = ln2 * (m_X + log2 l_X) and KL = ln2 * (A / l_T + m_S - m_T +
+# log2 l_S - log2 l_T), the same KL as the unsplit definition.
+
+LN2 = math.log(2.0)
+
+
+def _shard_scores(q_t, k_t, q_s, k_s, b, h, scale_t, scale_s, causal, k_offset, n_k_total):
+    qt, qs = _f64(q_t[b, h]), _f64(q_s[b, h])
+    kt, ks = _f64(k_t[b, h]), _f64(k_s[b, h])
+    n_q = qt.shape[0]
+    i = torch.arange(n_q)[:, None]
+    j = k_offset + torch.arange(kt.shape[0])[None, :]
+    mask = (j <= i + (n_k_total - n_q)) if causal else torch.ones(n_q, kt.shape[0],
+                                                                    dtype=torch.bool)
+    return scale_t * (qt @ kt.T), scale_s * (qs @ ks.T), mask, qt, qs, kt, ks
+
+
+def oracle_partial_state(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, k_offset: int,
+                         n_k_total: int):
+    """State planes (m_T, m_S, l_T, l_S, A) as float64 [5, B, H, N_Q] of one key shard
+    (k_* hold the shard's keys; grouped K heads are expanded)."""
+    B, H, n_q, _ = q_t.shape
+    k_t, k_s = expand_kv(k_t, H), expand_kv(k_s, H)
+    out = torch.zeros(5, B, H, n_q, dtype=F64)
+    if k_t.shape[2] == 0:  # an empty shard: the identity state
+        out[:2] = NEG_INF
+        return out
+    for b in range(B):
+        for h in range(H):
+            s_t, s_s, mask, *_ = _shard_scores(q_t, k_t, q_s, k_s, b, h, scale_t, scale_s,
+                                               causal, k_offset, n_k_total)
+            t_t = torch.where(mask, s_t / LN2, torch.full_like(s_t, NEG_INF))
+            t_s = torch.where(mask, s_s / LN2, torch.full_like(s_s, NEG_INF))
+            m_t, m_s = t_t.max(dim=1).values, t_s.max(dim=1).values
+            live = mask.any(dim=1)
+            mt0 = torch.where(live, m_t, torch.zeros_like(m_t))
+            ms0 = torch.where(live, m_s, torch.zeros_like(m_s))
+            e_t = torch.where(mask, torch.exp2(t_t - mt0[:, None]), torch.zeros_like(t_t))
+            e_s = torch.where(mask, torch.exp2(t_s - ms0[:, None]), torch.zeros_like(t_s))
+            diff = torch.where(mask, s_t / LN2 - s_s / LN2, torch.zeros_like(s_t))
+            out[0, b, h] = m_t
+            out[1, b, h] = m_s
+            out[2, b, h] = e_t.sum(dim=1)
+            out[3, b, h] = e_s.sum(dim=1)
+            out[4, b, h] = (e_t * diff).sum(dim=1)
+    return out
+
+
+def oracle_merge_states(states):
+    """Merge [R, 5, ...] shard states and finalise: (KL, LSE_T, LSE_S) float64."""
+    st = states.to(F64)
+    m_t, m_s = st[:, 0].max(dim=0).values, st[:, 1].max(dim=0).values
+    empty_t = torch.isinf(m_t) & (m_t < 0)
+    empty_s = torch.isinf(m_s) & (m_s < 0)
+    mt0 = torch.where(empty_t, torch.zeros_like(m_t), m_t)
+    ms0 = torch.where(empty_s, torch.zeros_like(m_s), m_s)
+    w_t = torch.exp2(st[:, 0] - mt0)  # -inf - m -> weight 0
+    w_s = torch.exp2(st[:, 1] - ms0)
+    l_t = (st[:, 2] * w_t).sum(dim=0)
+    l_s = (st[:, 3] * w_s).sum(dim=0)
+    a = (st[:, 4] * w_t).sum(dim=0)
+    empty = l_t == 0
+    l_t1, l_s1 = torch.where(empty, torch.ones_like(l_t), l_t), torch.where(empty, torch.ones_like(l_s), l_s)
+    kl = LN2 * (a / l_t1 + (ms0 - mt0) + torch.log2(l_s1) - torch.log2(l_t1))
+    lse_t = LN2 * (mt0 + torch.log2(l_t1))
+    lse_s = LN2 * (ms0 + torch.log2(l_s1))
+    kl = torch.where(empty, torch.zeros_like(kl), kl)
+    lse_t = torch.where(empty, torch.full_like(lse_t, NEG_INF), lse_t)
+    lse_s = torch.where(empty, torch.full_like(lse_s, NEG_INF), lse_s)
+    return kl, lse_t, lse_s
+
+
+def _bwd_shard(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, k_offset, n_k_total, kl, lse_t,
+               lse_s, g, teacher):
+    B, H, n_q, _ = q_t.shape
+    h_kv = (k_t if teacher else k_s).shape[1]
+    k_t, k_s = expand_kv(k_t, H), expand_kv(k_s, H)
+    q_g, k_g = (q_t, k_t) if teacher else (q_s, k_s)
+    dq = torch.zeros(q_g.shape, dtype=F64)
+    dk = torch.zeros(k_g.shape, dtype=F64)
+    for b in range(B):
+        for h in range(H):
+            s_t, s_s, mask, qt, qs, kt, ks = _shard_scores(q_t, k_t, q_s, k_s, b, h, scale_t,
+                                                          scale_s, causal, k_offset, n_k_total)
+            lt, ls = _f64(lse_t[b, h]), _f64(lse_s[b, h])
+            p_t, _ = _probs(s_t, lt, mask)
+            p_s, _ = _probs(s_s, ls, mask)
+            gi = _f64(g[b, h])[:, None]
+            if teacher:
+                e = _f64(kl[b, h]) + torch.where(torch.isinf(lt), torch.zeros_like(lt), lt - ls)
+                ds = gi * scale_t * p_t * ((s_t - s_s) - e[:, None])
+                ds = torch.where(mask, ds, torch.zeros_like(ds))
+                dq[b, h], dk[b, h] = ds @ kt, ds.T @ qt
+            else:
+                ds = gi * scale_s * (p_s - p_t)
+                dq[b, h], dk[b, h] = ds @ ks, ds.T @ qs
+    return dq, group_sum_kv(dk, h_kv)
+
+
+def oracle_bwd_shard(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, k_offset: int,
+                     n_k_total: int, lse_t, lse_s, g):
+    """Student gradients of one key shard with the global LSE_T / LSE_S: the shard's part
+    of dQ_S (summed over shards it gives dQ_S) and dK_S of the shard's keys."""
+    return _bwd_shard(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, k_offset, n_k_total, None,
+                      lse_t, lse_s, g, teacher=False)
+
+
+def oracle_bwd_teacher_shard(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, k_offset: int,
+                             n_k_total: int, kl, lse_t, lse_s, g):
+    """Trainable-teacher gradients of one key shard with the global KL and LSEs."""
+    return _bwd_shard(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, k_offset, n_k_total, kl,
+                      lse_t, lse_s, g, teacher=True)

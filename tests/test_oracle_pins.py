@@ -586,3 +586,92 @@ def test_varlen_rejects_bad_offsets():
         O.oracle_fwd_varlen(q, q, q, q, [0, 3, 2, 4], [0, 1, 2, 4], 1.0, 1.0, False)
     with pytest.raises(ValueError):
         O.oracle_fwd_varlen(q, q, q, q, [1, 4], [0, 4], 1.0, 1.0, False)
+
+
+# ------------------------------------------------ context parallelism over N_K
+
+def brute_force_state(q_t, k_t, q_s, k_s, st, ss, causal, k_offset, n_k_total):
+    """Shard state from its definition with pure-Python loops, base-2 units."""
+    B, H, nq, dt = q_t.shape
+    n_sh, ds_ = k_t.shape[2], q_s.shape[3]
+    L = lambda t: t.double().tolist()
+    QT, KT, QS, KS = L(q_t), L(k_t), L(q_s), L(k_s)
+    out = [[[[0.0] * nq for _ in range(H)] for _ in range(B)] for _ in range(5)]
+    for b in range(B):
+        for h in range(H):
+            for i in range(nq):
+                js = [j for j in range(n_sh)
+                      if (not causal) or (k_offset + j) <= i + n_k_total - nq]
+                if not js:
+                    out[0][b][h][i] = out[1][b][h][i] = float("-inf")
+                    continue
+                tT = {j: st * sum(QT[b][h][i][c] * KT[b][h][j][c] for c in range(dt)) / math.log(2)
+                      for j in js}
+                tS = {j: ss * sum(QS[b][h][i][c] * KS[b][h][j][c] for c in range(ds_)) / math.log(2)
+                      for j in js}
+                mT, mS = max(tT.values()), max(tS.values())
+                out[0][b][h][i], out[1][b][h][i] = mT, mS
+                out[2][b][h][i] = sum(2.0 ** (tT[j] - mT) for j in js)
+                out[3][b][h][i] = sum(2.0 ** (tS[j] - mS) for j in js)
+                out[4][b][h][i] = sum(2.0 ** (tT[j] - mT) * (tT[j] - tS[j]) for j in js)
+    return torch.tensor(out, dtype=F64)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_partial_state_against_brute_force(causal):
+    q_t, k_t, q_s, k_s, _ = rand_case(1, 2, 5, 9, 3, 2, seed=61)
+    sh = slice(6, 9)  # causal: row i sees global keys j <= i + 4, so rows 0, 1 see none
+    ref = brute_force_state(q_t, k_t[:, :, sh], q_s, k_s[:, :, sh], 0.8, 1.3, causal, 6, 9)
+    got = O.oracle_partial_state(q_t, k_t[:, :, sh], q_s, k_s[:, :, sh], 0.8, 1.3, causal, 6, 9)
+    fin = torch.isfinite(ref)
+    assert torch.equal(fin, torch.isfinite(got))
+    torch.testing.assert_close(got[fin], ref[fin], rtol=1e-12, atol=1e-12)
+    if causal:  # the identity state
+        assert torch.all(got[2:, :, :, :2] == 0) and torch.all(torch.isinf(got[:2, :, :, :2]))
+        assert torch.all(torch.isfinite(got[:, :, :, 2:]))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("cuts", [[0, 11], [0, 4, 11], [0, 1, 7, 11], [0, 5, 5, 11]])
+def test_merged_shards_equal_the_unsplit_oracle(causal, cuts):
+    q_t, k_t, q_s, k_s, g = rand_case(2, 2, 8, 11, 4, 3, seed=62)
+    args = (0.7, 1.1, causal)
+    states = torch.stack([
+        O.oracle_partial_state(q_t, k_t[:, :, a:b], q_s, k_s[:, :, a:b], *args, a, 11)
+        for a, b in zip(cuts, cuts[1:])])
+    kl, lt, ls = O.oracle_merge_states(states)
+    kl_r, lt_r, ls_r = O.oracle_fwd(q_t, k_t, q_s, k_s, *args)
+    torch.testing.assert_close(kl, kl_r, rtol=1e-11, atol=1e-12)
+    torch.testing.assert_close(lt, lt_r, rtol=1e-12, atol=1e-12)
+    torch.testing.assert_close(ls, ls_r, rtol=1e-12, atol=1e-12)
+    # merge order does not matter
+    kl2, _, _ = O.oracle_merge_states(states.flip(0))
+    torch.testing.assert_close(kl2, kl, rtol=1e-13, atol=1e-14)
+    # shard gradients: dQ parts sum to dQ, dK shards concatenate to dK (student, teacher)
+    dq_r, dk_r = O.oracle_bwd(q_t, k_t, q_s, k_s, *args, g)
+    dqt_r, dkt_r = O.oracle_bwd_teacher(q_t, k_t, q_s, k_s, *args, g)
+    parts = [O.oracle_bwd_shard(q_t, k_t[:, :, a:b], q_s, k_s[:, :, a:b], *args, a, 11, lt_r,
+                                ls_r, g) for a, b in zip(cuts, cuts[1:])]
+    tparts = [O.oracle_bwd_teacher_shard(q_t, k_t[:, :, a:b], q_s, k_s[:, :, a:b], *args, a, 11,
+                                         kl_r, lt_r, ls_r, g) for a, b in zip(cuts, cuts[1:])]
+    torch.testing.assert_close(sum(p[0] for p in parts), dq_r, rtol=1e-10, atol=1e-12)
+    torch.testing.assert_close(torch.cat([p[1] for p in parts], dim=2), dk_r, rtol=1e-10,
+                               atol=1e-12)
+    torch.testing.assert_close(sum(p[0] for p in tparts), dqt_r, rtol=1e-10, atol=1e-12)
+    torch.testing.assert_close(torch.cat([p[1] for p in tparts], dim=2), dkt_r, rtol=1e-10,
+                               atol=1e-12)
+
+
+def test_merge_identity_and_grouped_heads():
+    """A shard that no row can see merges as the identity; grouped K heads work per shard."""
+    q_t, k_t, q_s, k_s, g = rand_case(1, 4, 6, 10, 3, 3, seed=63)
+    k_t, k_s = k_t[:, :2], k_s[:, :1]
+    st = [O.oracle_partial_state(q_t, k_t[:, :, a:b], q_s, k_s[:, :, a:b], 0.9, 0.6, True, a, 10)
+          for a, b in [(0, 6), (6, 10)]]
+    empty = O.oracle_partial_state(q_t, k_t[:, :, :2], q_s, k_s[:, :, :2], 0.9, 0.6, True, 50, 10)
+    assert torch.all(torch.isinf(empty[:2])) and torch.all(empty[2:] == 0)
+    kl, lt, _ = O.oracle_merge_states(torch.stack(st))
+    kl_e, lt_e, _ = O.oracle_merge_states(torch.stack(st + [empty]))
+    assert torch.equal(kl, kl_e) and torch.equal(lt, lt_e)
+    kl_r, _, _ = O.oracle_fwd_gqa(q_t, k_t, q_s, k_s, 0.9, 0.6, True)
+    torch.testing.assert_close(kl, kl_r, rtol=1e-11, atol=1e-12)
