@@ -29,8 +29,9 @@ LIB_PATH = os.path.join(_PKG, "lib", "libstreamkl.so")
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "MISALIGNED", 4: "LAUNCH", 5: "TIMEOUT"}
 EXPORTS = ("streamkl_fwd", "streamkl_bwd", "streamkl_bwd_teacher", "streamkl_fwd_gqa",
            "streamkl_bwd_gqa", "streamkl_bwd_teacher_gqa", "streamkl_fwd_varlen",
-           "streamkl_bwd_varlen", "streamkl_bwd_teacher_varlen", "streamkl_status_string",
-           "streamkl_device_status", "streamkl_version")
+           "streamkl_bwd_varlen", "streamkl_bwd_teacher_varlen", "streamkl_fwd_partial",
+           "streamkl_merge_partial", "streamkl_bwd_shard", "streamkl_bwd_teacher_shard",
+           "streamkl_status_string", "streamkl_device_status", "streamkl_version")
 
 
 class StreamKLError(RuntimeError):
@@ -77,6 +78,17 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.streamkl_bwd_varlen.restype = i
     lib.streamkl_bwd_teacher_varlen.argtypes = head + [vp, vp, vp, vp, vp, vp, vp]
     lib.streamkl_bwd_teacher_varlen.restype = i
+    # shard entry points: q_t, k_t, q_s, k_s, B, H, H_kv_T, H_kv_S, N_Q, N_K_shard, k_offset,
+    # N_K_total, d_T, d_S, scale_T, scale_S, causal, then the outputs / row inputs.
+    shead = [vp] * 4 + [i] * 10 + [f, f, i]
+    lib.streamkl_fwd_partial.argtypes = shead + [vp, vp]
+    lib.streamkl_fwd_partial.restype = i
+    lib.streamkl_merge_partial.argtypes = [vp, i, ctypes.c_longlong, vp, vp, vp, vp]
+    lib.streamkl_merge_partial.restype = i
+    lib.streamkl_bwd_shard.argtypes = shead + [vp, vp, vp, vp, vp, vp]
+    lib.streamkl_bwd_shard.restype = i
+    lib.streamkl_bwd_teacher_shard.argtypes = shead + [vp, vp, vp, vp, vp, vp, vp]
+    lib.streamkl_bwd_teacher_shard.restype = i
     lib.streamkl_status_string.argtypes = [i]
     lib.streamkl_status_string.restype = ctypes.c_char_p
     lib.streamkl_device_status.argtypes = [vp]
@@ -378,6 +390,83 @@ def streamkl_bwd_teacher_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k,
         lse_t.data_ptr(), lse_s.data_ptr(), g.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(),
         _stream_ptr(stream))
     _check(st, "streamkl_bwd_teacher_varlen")
+    return dq_t, dk_t
+
+
+def streamkl_fwd_partial(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
+                         k_offset: int, n_k_total: int, state=None, stream=None):
+    """Row state of one key shard (k_* hold the shard's keys): fp32 [5, B, H, N_Q], planes
+    m_T, m_S, l_T, l_S, A in base-2 units."""
+    import torch
+    B, H, h_kt, h_ks, n_q, n_k, d_t, d_s = _shape_gqa(q_t, k_t, q_s, k_s)
+    state = (torch.empty(5, B, H, n_q, device=q_t.device, dtype=torch.float32) if state is None
+             else _check_out(state, (5, B, H, n_q), "state"))
+    st = load_library().streamkl_fwd_partial(
+        q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), B, H, h_kt, h_ks, n_q,
+        n_k, int(k_offset), int(n_k_total), d_t, d_s, float(scale_T), float(scale_S),
+        int(bool(causal)), state.data_ptr(), _stream_ptr(stream))
+    _check(st, "streamkl_fwd_partial")
+    return state
+
+
+def streamkl_merge_partial(states, kl=None, lse_t=None, lse_s=None, stream=None):
+    """Merge gathered shard states [R, 5, B, H, N_Q] into KL, LSE_T, LSE_S [B, H, N_Q]."""
+    import torch
+    if states.dtype != torch.float32 or not states.is_cuda or not states.is_contiguous() or \
+            states.dim() != 5 or states.shape[1] != 5:
+        raise ValueError("states must be a contiguous fp32 CUDA tensor [R, 5, B, H, N_Q]")
+    R, _, B, H, n_q = states.shape
+    mk = lambda: torch.empty(B, H, n_q, device=states.device, dtype=torch.float32)
+    kl = mk() if kl is None else _check_out(kl, (B, H, n_q), "kl")
+    lse_t = mk() if lse_t is None else _check_out(lse_t, (B, H, n_q), "lse_t")
+    lse_s = mk() if lse_s is None else _check_out(lse_s, (B, H, n_q), "lse_s")
+    st = load_library().streamkl_merge_partial(states.data_ptr(), R, B * H * n_q, kl.data_ptr(),
+                                               lse_t.data_ptr(), lse_s.data_ptr(),
+                                               _stream_ptr(stream))
+    _check(st, "streamkl_merge_partial")
+    return kl, lse_t, lse_s
+
+
+def streamkl_bwd_shard(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
+                       k_offset: int, n_k_total: int, lse_t, lse_s, g, dq_s=None, dk_s=None,
+                       stream=None):
+    """Student gradients of one key shard with the merged LSEs: the shard's part of dQ_S
+    [B,H,N_Q,d_S] (sum over shards = dQ_S) and dK_S of its keys [B,H_kv_S,N_K_shard,d_S]."""
+    import torch
+    B, H, h_kt, h_ks, n_q, n_k, d_t, d_s = _shape_gqa(q_t, k_t, q_s, k_s)
+    _check_rows((("lse_t", lse_t), ("lse_s", lse_s), ("g", g)), (B, H, n_q))
+    dev = q_t.device
+    dq_s = (torch.empty(B, H, n_q, d_s, device=dev, dtype=torch.float32) if dq_s is None
+            else _check_out(dq_s, (B, H, n_q, d_s), "dq_s"))
+    dk_s = (torch.empty(B, h_ks, n_k, d_s, device=dev, dtype=torch.float32) if dk_s is None
+            else _check_out(dk_s, (B, h_ks, n_k, d_s), "dk_s"))
+    st = load_library().streamkl_bwd_shard(
+        q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), B, H, h_kt, h_ks, n_q,
+        n_k, int(k_offset), int(n_k_total), d_t, d_s, float(scale_T), float(scale_S),
+        int(bool(causal)), lse_t.data_ptr(), lse_s.data_ptr(), g.data_ptr(), dq_s.data_ptr(),
+        dk_s.data_ptr(), _stream_ptr(stream))
+    _check(st, "streamkl_bwd_shard")
+    return dq_s, dk_s
+
+
+def streamkl_bwd_teacher_shard(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float,
+                               causal: bool, k_offset: int, n_k_total: int, kl, lse_t, lse_s, g,
+                               dq_t=None, dk_t=None, stream=None):
+    """Trainable-teacher gradients of one key shard with the merged KL and LSEs."""
+    import torch
+    B, H, h_kt, h_ks, n_q, n_k, d_t, d_s = _shape_gqa(q_t, k_t, q_s, k_s)
+    _check_rows((("kl", kl), ("lse_t", lse_t), ("lse_s", lse_s), ("g", g)), (B, H, n_q))
+    dev = q_t.device
+    dq_t = (torch.empty(B, H, n_q, d_t, device=dev, dtype=torch.float32) if dq_t is None
+            else _check_out(dq_t, (B, H, n_q, d_t), "dq_t"))
+    dk_t = (torch.empty(B, h_kt, n_k, d_t, device=dev, dtype=torch.float32) if dk_t is None
+            else _check_out(dk_t, (B, h_kt, n_k, d_t), "dk_t"))
+    st = load_library().streamkl_bwd_teacher_shard(
+        q_t.data_ptr(), k_t.data_ptr(), q_s.data_ptr(), k_s.data_ptr(), B, H, h_kt, h_ks, n_q,
+        n_k, int(k_offset), int(n_k_total), d_t, d_s, float(scale_T), float(scale_S),
+        int(bool(causal)), kl.data_ptr(), lse_t.data_ptr(), lse_s.data_ptr(), g.data_ptr(),
+        dq_t.data_ptr(), dk_t.data_ptr(), _stream_ptr(stream))
+    _check(st, "streamkl_bwd_teacher_shard")
     return dq_t, dk_t
 
 

@@ -53,6 +53,7 @@ struct BwdArgs {
   const int* cu_k;
   int total_q, total_k;    // packed layout: rows of the packed Q / K tensors
   long long dk_hs, dk_rs;  // dk element strides of a K head and of a key row
+  int off_adj;             // causal shift of a key shard (context parallelism), else 0
   const float* lse_t;
   const float* lse_s;
   const float* g;
@@ -145,7 +146,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   grouped_order(blockIdx.x, args.BH, args.n_ktiles, args.group, bh, kt);
   SeqView seq;
   if (!seq_view(args.cu_q, args.cu_k, bh, args.H, args.gT, args.gS, args.N_Q, args.N_K,
-                args.total_q, args.total_k, seq)) {
+                args.total_q, args.total_k, args.off_adj, seq)) {
     if (threadIdx.x == 0) atomicOr(&g_skl_error, kErrBadOffsets);
     return;
   }

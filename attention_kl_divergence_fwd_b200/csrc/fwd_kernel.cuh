@@ -37,6 +37,9 @@ struct FwdArgs {
   const int* cu_q;    // packed layout: [B+1] sequence offsets (null: dense [B, H, N, d])
   const int* cu_k;
   int total_q, total_k;  // packed layout: rows of the packed Q / K tensors
+  int off_adj;           // causal shift of a key shard (context parallelism), else 0
+  float* state;          // non-null: write the raw row state (5 planes of plane floats)
+  long long plane;       //   instead of KL / LSE (context parallelism)
   float* kl;
   float* lse_t;
   float* lse_s;
@@ -219,7 +222,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   const int qpair = args.n_ctas_per_bh - 1 - unit;
   SeqView seq;
   if (!seq_view(args.cu_q, args.cu_k, bh, args.H, args.gT, args.gS, args.N_Q, args.N_K,
-                args.total_q, args.total_k, seq)) {
+                args.total_q, args.total_k, args.off_adj, seq)) {
     if (threadIdx.x == 0) atomicOr(&g_skl_error, kErrBadOffsets);
     return;
   }
@@ -303,23 +306,21 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     }
 
     if (ok && row < seq.nq) {
-      const float LN2 = 0.69314718055994530942f;
-      float kl, lse_t, lse_s;
-      if (st.lT > 0.f) {
-        const float l2T = log2f(st.lT), l2S = log2f(st.lS);
-        lse_t = LN2 * (st.mT + l2T);
-        lse_s = LN2 * (st.mS + l2S);
-        // Grouped so that identical teacher and student statistics give exactly 0.
-        kl = LN2 * ((st.A / st.lT) + ((st.mS - st.mT) + (l2S - l2T)));
-      } else {
-        kl = 0.f;
-        lse_t = -INFINITY;
-        lse_s = -INFINITY;
-      }
       const size_t o = (size_t)(seq.ob + row);
-      args.kl[o] = kl;
-      args.lse_t[o] = lse_t;
-      args.lse_s[o] = lse_s;
+      if (args.state) {
+        float* p = args.state + o;
+        p[0] = st.mT;
+        p[args.plane] = st.mS;
+        p[2 * args.plane] = st.lT;
+        p[3 * args.plane] = st.lS;
+        p[4 * args.plane] = st.A;
+      } else {
+        float kl, lse_t, lse_s;
+        finalize_row(st.mT, st.mS, st.lT, st.lS, st.A, kl, lse_t, lse_s);
+        args.kl[o] = kl;
+        args.lse_t[o] = lse_t;
+        args.lse_s[o] = lse_s;
+      }
     }
   } else {
     regs_dec<104>();

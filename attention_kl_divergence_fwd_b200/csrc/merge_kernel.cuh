@@ -1,0 +1,50 @@
+// merge_kernel.cuh - merge of per-row StreamKL states from several key shards.
+//
+// Context parallelism over N_K splits the keys of a sequence into contiguous shards; the
+// forward of each shard leaves, per query row, the online state of the one-pass
+// reduction ("StreamKL: Fast and Memory-Efficient KL Divergence for Boosting Attention
+// Distillation", abstract: online formulation of the coupled two-distribution KL
+// reduction): maxima m_T, m_S and sums l_T, l_S, A in base-2 units. States combine by
+// rescaling to the larger maximum and adding, so R shard states merge into the state of
+// the whole key range, which is then finalised exactly as the one-pass forward does.
+//
+// One thread per query row, a grid-stride loop; each state plane is read once, coalesced.
+// Bound: HBM (20 R + 12 bytes per row).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace skl {
+
+// states: [R][5][rows] fp32 (planes m_T, m_S, l_T, l_S, A); outputs [rows].
+__global__ void __launch_bounds__(256)
+streamkl_merge_kernel(const float* __restrict__ states, int R, long long rows,
+                      float* __restrict__ kl, float* __restrict__ lse_t,
+                      float* __restrict__ lse_s) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += stride) {
+    float mT = -INFINITY, mS = -INFINITY, lT = 0.f, lS = 0.f, A = 0.f;
+    for (int r = 0; r < R; ++r) {
+      const float* p = states + (long long)r * 5 * rows + i;
+      const float rmT = __ldg(p), rmS = __ldg(p + rows);
+      const float rlT = __ldg(p + 2 * rows), rlS = __ldg(p + 3 * rows), rA = __ldg(p + 4 * rows);
+      const float nT = fmaxf(mT, rmT), nS = fmaxf(mS, rmS);
+      const float uT = nT == -INFINITY ? 0.f : nT;  // reference while every max is -inf
+      const float uS = nS == -INFINITY ? 0.f : nS;
+      const float wT0 = exp2f(mT - uT), wT1 = exp2f(rmT - uT);  // -inf - x -> 0
+      const float wS0 = exp2f(mS - uS), wS1 = exp2f(rmS - uS);
+      lT = lT * wT0 + rlT * wT1;
+      A = A * wT0 + rA * wT1;
+      lS = lS * wS0 + rlS * wS1;
+      mT = nT;
+      mS = nS;
+    }
+    float k, a, b;
+    finalize_row(mT, mS, lT, lS, A, k, a, b);
+    kl[i] = k;
+    lse_t[i] = a;
+    lse_s[i] = b;
+  }
+}
+
+}  // namespace skl

@@ -13,9 +13,10 @@
 namespace skl {
 
 // Device-side error word of this library (one per device, in the library's module):
-// bit 0 = a forward watchdog fired, bit 1 = a backward watchdog fired. Read and
-// cleared by streamkl_device_status(). The library is built as one translation unit,
-// so this is the only definition.
+// bit 0 = a forward watchdog fired, bit 1 = a backward watchdog fired, bit 2 = the
+// dynamic shared memory was not 1024-byte aligned, bit 3 = malformed packed-sequence
+// offsets. Read and cleared by streamkl_device_status(). The library is built as one
+// translation unit, so this is the only definition.
 __device__ unsigned int g_skl_error = 0;
 
 // ----------------------------------------------------------------- misc
@@ -284,9 +285,12 @@ struct SeqView {
 
 // Returns false when the packed offsets of this sequence are malformed (not
 // 0 <= cu[b] <= cu[b+1] <= total, or longer than the longest length given).
+// off_adj shifts the causal alignment of a dense problem whose keys are one shard of a
+// longer sequence (context parallelism): shard key j is global key k_offset + j and
+// off_adj = N_K_total - N_K_shard - k_offset; 0 otherwise.
 __device__ __forceinline__ bool seq_view(const int* cu_q, const int* cu_k, int bh, int H,
                                          int gT, int gS, int N_Q, int N_K, int total_q,
-                                         int total_k, SeqView& v) {
+                                         int total_k, int off_adj, SeqView& v) {
   const int b = bh / H, h = bh - b * H;
   if (cu_q == nullptr) {
     v.nq = N_Q;
@@ -297,6 +301,7 @@ __device__ __forceinline__ bool seq_view(const int* cu_q, const int* cu_k, int b
     v.zkt = b * (H / gT) + h / gT;
     v.zks = b * (H / gS) + h / gS;
     v.ob = (long long)bh * N_Q;
+    v.off = N_K - N_Q + off_adj;
   } else {
     const int q_lo = __ldg(cu_q + b), q_hi = __ldg(cu_q + b + 1);
     const int k_lo = __ldg(cu_k + b), k_hi = __ldg(cu_k + b + 1);
@@ -310,9 +315,28 @@ __device__ __forceinline__ bool seq_view(const int* cu_q, const int* cu_k, int b
     v.zkt = h / gT;
     v.zks = h / gS;
     v.ob = (long long)h * total_q + q_lo;
+    v.off = v.nk - v.nq;
   }
-  v.off = v.nk - v.nq;
   return true;
+}
+
+// KL and the two natural-log log-sum-exps of one query row from its online state in
+// base-2 units: running maxima m_T, m_S, sums l_X = sum 2^(t_X - m_X) and
+// A = sum 2^(t_T - m_T) (t_T - t_S). A row with no allowed key (l_T = 0) gets KL = 0 and
+// LSE = -inf. Grouped so that identical teacher and student statistics give exactly 0.
+__device__ __forceinline__ void finalize_row(float mT, float mS, float lT, float lS, float A,
+                                             float& kl, float& lse_t, float& lse_s) {
+  const float LN2 = 0.69314718055994530942f;
+  if (lT > 0.f) {
+    const float l2T = log2f(lT), l2S = log2f(lS);
+    lse_t = LN2 * (mT + l2T);
+    lse_s = LN2 * (mS + l2S);
+    kl = LN2 * ((A / lT) + ((mS - mT) + (l2S - l2T)));
+  } else {
+    kl = 0.f;
+    lse_t = -INFINITY;
+    lse_s = -INFINITY;
+  }
 }
 
 // Error word bit for malformed packed-sequence offsets (found on the device).

@@ -16,6 +16,7 @@
 #include "streamkl.h"
 #include "fwd_kernel.cuh"
 #include "bwd_kernel.cuh"
+#include "merge_kernel.cuh"
 
 namespace {
 
@@ -77,6 +78,7 @@ struct Problem {
   int B = 0, H = 0, H_kv_T = 0, H_kv_S = 0;
   int N_Q = 0, N_K = 0;          // dense sizes; packed: longest query / key sequence
   int total_q = 0, total_k = 0;  // packed: rows of the packed Q / K tensors
+  int off_adj = 0;               // dense key shard: N_K_total - N_K - k_offset
   bool packed() const { return cu_q != nullptr; }
   long long q_rows() const { return packed() ? total_q : (long long)B * H * N_Q; }
   long long k_rows(int h_kv) const { return packed() ? total_k : (long long)B * h_kv * N_K; }
@@ -189,15 +191,22 @@ streamkl_status launch_bwd(const CUtensorMap* maps, const skl::BwdArgs& a, bool 
   return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
 }
 
+// With state != nullptr the forward writes the raw row state (context parallelism)
+// instead of KL / LSE.
 streamkl_status fwd_common(const void* q_t, const void* k_t, const void* q_s, const void* k_s,
                            const Problem& P, int d_T, int d_S, float scale_T, float scale_S,
                            int causal, float* kl, float* lse_t, float* lse_s,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, float* state = nullptr) {
   streamkl_status st = check_common(q_t, k_t, q_s, k_s, P, d_T, d_S, scale_T, scale_S);
   if (st != STREAMKL_OK) return st;
   if (P.q_rows() == 0) return STREAMKL_OK;  // packed, no query rows: nothing to write
-  if (!kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
-  if (!aligned16(kl) || !aligned16(lse_t) || !aligned16(lse_s)) return STREAMKL_ERR_MISALIGNED;
+  if (state) {
+    if (!aligned16(state)) return STREAMKL_ERR_MISALIGNED;
+  } else {
+    if (!kl || !lse_t || !lse_s) return STREAMKL_ERR_INVALID_ARG;
+    if (!aligned16(kl) || !aligned16(lse_t) || !aligned16(lse_s))
+      return STREAMKL_ERR_MISALIGNED;
+  }
   const bool no_keys = P.packed() && P.total_k == 0;
   CUtensorMap maps[4];
   if (!map_of(&maps[0], q_t, P, d_T, false, 0, 128) ||
@@ -222,6 +231,9 @@ streamkl_status fwd_common(const void* q_t, const void* k_t, const void* q_s, co
   a.cu_k = P.cu_k;
   a.total_q = P.total_q;
   a.total_k = P.total_k;
+  a.off_adj = P.off_adj;
+  a.state = state;
+  a.plane = (long long)bh * P.N_Q;
   a.kl = kl;
   a.lse_t = lse_t;
   a.lse_s = lse_s;
@@ -293,6 +305,7 @@ streamkl_status bwd_common(const void* q_t, const void* k_t, const void* q_s, co
   a.total_k = P.total_k;
   a.dk_hs = P.packed() ? d_g : (long long)P.N_K * d_g;
   a.dk_rs = P.packed() ? (long long)h_kv_g * d_g : d_g;
+  a.off_adj = P.off_adj;
   a.lse_t = lse_t;
   a.lse_s = lse_s;
   a.g = g;
@@ -316,6 +329,13 @@ Problem dense(int B, int H, int H_kv_T, int H_kv_S, int N_Q, int N_K) {
   P.N_Q = N_Q;
   P.N_K = N_K;
   return P;
+}
+
+// Dense problem whose keys are one shard [k_offset, k_offset + N_K) of N_K_total keys.
+bool shard(Problem& P, int k_offset, int N_K_total) {
+  if (k_offset < 0 || N_K_total < 1 || (long long)k_offset + P.N_K > N_K_total) return false;
+  P.off_adj = N_K_total - P.N_K - k_offset;
+  return true;
 }
 
 Problem packed(const int* cu_q, const int* cu_k, int B, int H, int H_kv_T, int H_kv_S,
@@ -429,6 +449,56 @@ streamkl_status streamkl_bwd_teacher_varlen(
                                  total_k, max_seqlen_q, max_seqlen_k),
                           d_T, d_S, scale_T, scale_S, causal, kl, lse_t, lse_s, g, dq_t, dk_t,
                           stream);
+}
+
+streamkl_status streamkl_fwd_partial(const void* q_t, const void* k_t, const void* q_s,
+                                     const void* k_s, int B, int H, int H_kv_T, int H_kv_S,
+                                     int N_Q, int N_K_shard, int k_offset, int N_K_total,
+                                     int d_T, int d_S, float scale_T, float scale_S, int causal,
+                                     float* state, cudaStream_t stream) {
+  Problem P = dense(B, H, H_kv_T, H_kv_S, N_Q, N_K_shard);
+  if (!state || N_K_shard < 1 || !shard(P, k_offset, N_K_total)) return STREAMKL_ERR_INVALID_ARG;
+  return fwd_common(q_t, k_t, q_s, k_s, P, d_T, d_S, scale_T, scale_S, causal, nullptr, nullptr,
+                    nullptr, stream, state);
+}
+
+streamkl_status streamkl_merge_partial(const float* states, int R, long long rows, float* kl,
+                                       float* lse_t, float* lse_s, cudaStream_t stream) {
+  if (!states || !kl || !lse_t || !lse_s || R < 1 || rows < 1) return STREAMKL_ERR_INVALID_ARG;
+  if ((long long)R * 5 * rows >= (1ll << 40)) return STREAMKL_ERR_UNSUPPORTED;
+  if (!aligned16(states) || !aligned16(kl) || !aligned16(lse_t) || !aligned16(lse_s))
+    return STREAMKL_ERR_MISALIGNED;
+  // Enough 256-thread blocks to cover every row, at most 16 per SM of the 148.
+  const long long need = (rows + 255) / 256;
+  const unsigned grid = (unsigned)(need < 148 * 16 ? need : 148 * 16);
+  skl::streamkl_merge_kernel<<<grid, 256, 0, stream>>>(states, R, rows, kl, lse_t, lse_s);
+  return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
+}
+
+streamkl_status streamkl_bwd_shard(const void* q_t, const void* k_t, const void* q_s,
+                                   const void* k_s, int B, int H, int H_kv_T, int H_kv_S,
+                                   int N_Q, int N_K_shard, int k_offset, int N_K_total, int d_T,
+                                   int d_S, float scale_T, float scale_S, int causal,
+                                   const float* lse_t, const float* lse_s, const float* g,
+                                   float* dq_s, float* dk_s, cudaStream_t stream) {
+  Problem P = dense(B, H, H_kv_T, H_kv_S, N_Q, N_K_shard);
+  if (N_K_shard < 1 || !shard(P, k_offset, N_K_total)) return STREAMKL_ERR_INVALID_ARG;
+  return bwd_common<false>(q_t, k_t, q_s, k_s, P, d_T, d_S, scale_T, scale_S, causal, nullptr,
+                           lse_t, lse_s, g, dq_s, dk_s, stream);
+}
+
+streamkl_status streamkl_bwd_teacher_shard(const void* q_t, const void* k_t, const void* q_s,
+                                           const void* k_s, int B, int H, int H_kv_T,
+                                           int H_kv_S, int N_Q, int N_K_shard, int k_offset,
+                                           int N_K_total, int d_T, int d_S, float scale_T,
+                                           float scale_S, int causal, const float* kl,
+                                           const float* lse_t, const float* lse_s,
+                                           const float* g, float* dq_t, float* dk_t,
+                                           cudaStream_t stream) {
+  Problem P = dense(B, H, H_kv_T, H_kv_S, N_Q, N_K_shard);
+  if (N_K_shard < 1 || !shard(P, k_offset, N_K_total)) return STREAMKL_ERR_INVALID_ARG;
+  return bwd_common<true>(q_t, k_t, q_s, k_s, P, d_T, d_S, scale_T, scale_S, causal, kl, lse_t,
+                          lse_s, g, dq_t, dk_t, stream);
 }
 
 const char* streamkl_status_string(streamkl_status s) {

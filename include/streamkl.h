@@ -187,6 +187,54 @@ streamkl_status streamkl_bwd_teacher_varlen(
     int causal, const float* kl, const float* lse_t, const float* lse_s, const float* g,
     float* dq_t, float* dk_t, cudaStream_t stream);
 
+/*
+ * Context parallelism over N_K (keys of one sequence split across GPUs or passes). The
+ * abstract's forward keeps an online per-row state; states of disjoint key ranges merge
+ * associatively, so each shard runs the forward on its keys and a merge finalises.
+ * Dense layout, grouped K heads allowed (H_kv_* as above); k_t / k_s hold only the shard's
+ * keys: k_t [B,H_kv_T,N_K_shard,d_T], k_s [B,H_kv_S,N_K_shard,d_S]. Shard key j is global key
+ * k_offset + j; causal alignment uses the global indices (j_global <= i + N_K_total - N_Q);
+ * 0 <= k_offset, k_offset + N_K_shard <= N_K_total, N_K_shard >= 1 (else INVALID_ARG).
+ *
+ * streamkl_fwd_partial writes the row state of its shard, fp32 [5,B,H,N_Q], planes in
+ * base-2 units (t_X = s_X * log2 e): m_T, m_S (maxima over the shard's allowed keys),
+ * l_T, l_S (sum 2^(t_X - m_X)), A (sum 2^(t_T - m_T) (t_T - t_S)); a row that sees no key
+ * of the shard gets m = -inf, l = 0, A = 0 (the identity of the merge).
+ *
+ * streamkl_merge_partial merges R such states, laid out [R,5,rows] (rows = B*H*N_Q, the
+ * gathered states of all shards in any order), and writes kl, lse_t, lse_s [rows] exactly
+ * as streamkl_fwd would for the whole key range (R = 1 reproduces it bit for bit).
+ *
+ * streamkl_bwd_shard / streamkl_bwd_teacher_shard take the merged (global) lse_t, lse_s
+ * (and kl for the teacher) and g, and write the gradients of the shard's keys (dk, final)
+ * and the shard's part of dq (fp32 [B,H,N_Q,d], zeroed first): the full dq is the sum of
+ * the parts over all shards (an all-reduce across the shards' ranks).
+ */
+streamkl_status streamkl_fwd_partial(const void* q_t, const void* k_t, const void* q_s,
+                                     const void* k_s, int B, int H, int H_kv_T, int H_kv_S,
+                                     int N_Q, int N_K_shard, int k_offset, int N_K_total,
+                                     int d_T, int d_S, float scale_T, float scale_S, int causal,
+                                     float* state, cudaStream_t stream);
+
+streamkl_status streamkl_merge_partial(const float* states, int R, long long rows, float* kl,
+                                       float* lse_t, float* lse_s, cudaStream_t stream);
+
+streamkl_status streamkl_bwd_shard(const void* q_t, const void* k_t, const void* q_s,
+                                   const void* k_s, int B, int H, int H_kv_T, int H_kv_S,
+                                   int N_Q, int N_K_shard, int k_offset, int N_K_total, int d_T,
+                                   int d_S, float scale_T, float scale_S, int causal,
+                                   const float* lse_t, const float* lse_s, const float* g,
+                                   float* dq_s, float* dk_s, cudaStream_t stream);
+
+streamkl_status streamkl_bwd_teacher_shard(const void* q_t, const void* k_t, const void* q_s,
+                                           const void* k_s, int B, int H, int H_kv_T,
+                                           int H_kv_S, int N_Q, int N_K_shard, int k_offset,
+                                           int N_K_total, int d_T, int d_S, float scale_T,
+                                           float scale_S, int causal, const float* kl,
+                                           const float* lse_t, const float* lse_s,
+                                           const float* g, float* dq_t, float* dk_t,
+                                           cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char* streamkl_status_string(streamkl_status status);
 

@@ -171,3 +171,26 @@ def test_varlen_host_validation_outputs(lib):
 def test_varlen_without_query_rows_is_a_no_op(lib):
     # No query rows: nothing to compute or write, so no CUDA call is made at all.
     assert fwd_varlen(lib, q_t=0, q_s=0, kl=0, lse_t=0, lse_s=0, total_q=0, max_q=0) == 0
+
+
+def test_shard_host_validation(lib):
+    def fwd_partial(k_offset=0, n_sh=128, n_tot=256, state=P, **kw):
+        a = dict(q_t=P, k_t=P, q_s=P, k_s=P, B=1, H=2, H_kv_T=2, H_kv_S=1, N_Q=128)
+        a.update(kw)
+        return lib.streamkl_fwd_partial(*a.values(), n_sh, k_offset, n_tot, 128, 128, 0.1, 0.1,
+                                        1, state, 0)
+    assert fwd_partial(k_offset=-1) == 1
+    assert fwd_partial(k_offset=200) == 1          # shard runs past N_K_total
+    assert fwd_partial(n_sh=0) == 1
+    assert fwd_partial(state=0) == 1
+    assert fwd_partial(state=P + 4) == 3
+    assert fwd_partial(q_t=0) == 1
+    assert fwd_partial(H_kv_S=3) == 2
+    assert lib.streamkl_bwd_shard(P, P, P, P, 1, 2, 2, 2, 128, 128, 200, 256, 128, 128, 0.1, 0.1,
+                                  1, P, P, P, P, P, 0) == 1
+    assert lib.streamkl_bwd_teacher_shard(P, P, P, P, 1, 2, 2, 2, 128, 128, 0, 256, 128, 128,
+                                          0.1, 0.1, 1, 0, P, P, P, P, P, 0) == 1
+    assert lib.streamkl_merge_partial(P, 0, 100, P, P, P, 0) == 1
+    assert lib.streamkl_merge_partial(P, 2, 0, P, P, P, 0) == 1
+    assert lib.streamkl_merge_partial(P + 4, 2, 100, P, P, P, 0) == 3
+    assert lib.streamkl_merge_partial(0, 2, 100, P, P, P, 0) == 1

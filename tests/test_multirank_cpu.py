@@ -38,7 +38,7 @@ def _worker(rank, world, port, out):
 def test_max_over_ranks_gloo_world2():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     assert dict(out) == {0: 11.0, 1: 11.0}

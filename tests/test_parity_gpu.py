@@ -388,3 +388,105 @@ def test_varlen_length_mix_sampled():
     check_lse(g["lse_s"], ls)
     dq, dk = oracle_bwd_varlen(*args, x["g"])
     assert rel_fro(g["dq"], dq) <= GRAD_REL and rel_fro(g["dk"], dk) <= GRAD_REL
+
+
+# ------------------------------------------------ context parallelism over N_K
+#
+# R key shards run one after another on one GPU (independent launches; nothing waits on
+# another kernel), their states are stacked as an all-gather would and merged.
+
+from oracle import oracle_partial_state  # noqa: E402
+
+
+def _shard_run(x, cuts, st, ss, causal, teacher=False):
+    d = {k: v.cuda() for k, v in x.items()}
+    nk = d["k_t"].shape[2]
+    states = []
+    for a, b in zip(cuts, cuts[1:]):
+        states.append(skl.streamkl_fwd_partial(
+            d["q_t"], d["k_t"][:, :, a:b].contiguous(), d["q_s"], d["k_s"][:, :, a:b].contiguous(),
+            st, ss, causal, a, nk))
+    states = torch.stack(states)
+    kl, lt, ls = skl.streamkl_merge_partial(states)
+    dq = dk = dqt = dkt = None
+    parts = []
+    for a, b in zip(cuts, cuts[1:]):
+        sa = (d["q_t"], d["k_t"][:, :, a:b].contiguous(), d["q_s"],
+              d["k_s"][:, :, a:b].contiguous(), st, ss, causal, a, nk)
+        p = skl.streamkl_bwd_shard(*sa, lt, ls, d["g"])
+        pt = skl.streamkl_bwd_teacher_shard(*sa, kl, lt, ls, d["g"]) if teacher else (None, None)
+        parts.append((p[0].cpu().double(), p[1].cpu().double(),
+                      None if pt[0] is None else pt[0].cpu().double(),
+                      None if pt[1] is None else pt[1].cpu().double()))
+    assert skl.device_status() == 0
+    dq = sum(p[0] for p in parts)
+    dk = torch.cat([p[1] for p in parts], dim=2)
+    if teacher:
+        dqt = sum(p[2] for p in parts)
+        dkt = torch.cat([p[3] for p in parts], dim=2)
+    c = lambda t: t.cpu().double()
+    return states.cpu().double(), c(kl), c(lt), c(ls), dq, dk, dqt, dkt
+
+
+@pytest.mark.parametrize("causal,cuts,hk", [
+    (True, [0, 256, 640, 900], 4), (True, [0, 300, 900], 2), (False, [0, 128, 900], 4),
+    (True, [0, 900], 1)])
+def test_context_parallel_shards_match_oracle(causal, cuts, hk):
+    w = WORKLOADS["b2h16_n4096_d128_causal"].with_sizes(B=1, H=4, N_Q=700, N_K=900)
+    x = make_inputs(w, seed=91)
+    x["k_t"], x["k_s"] = x["k_t"][:, :hk].contiguous(), x["k_s"][:, :hk].contiguous()
+    st, ss = w.scale_T, w.scale_S
+    states, kl, lt, ls, dq, dk, dqt, dkt = _shard_run(x, cuts, st, ss, causal, teacher=True)
+    args = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], st, ss, causal)
+    kl_r, lt_r, ls_r = oracle_fwd_gqa(*args)
+    check_kl(kl, kl_r)
+    check_lse(lt, lt_r)
+    check_lse(ls, ls_r)
+    dq_r, dk_r = oracle_bwd_gqa(*args, x["g"])
+    assert rel_fro(dq, dq_r) <= GRAD_REL and rel_fro(dk, dk_r) <= GRAD_REL
+    dqt_r, dkt_r = oracle_bwd_teacher_gqa(*args, x["g"])
+    assert rel_fro(dqt, dqt_r) <= GRAD_REL and rel_fro(dkt, dkt_r) <= GRAD_REL
+    # each shard's state: its own log-sum-exps ln2 * (m + log2 l) and expectation A / l_T
+    for r, (a, b) in enumerate(zip(cuts, cuts[1:])):
+        ref = oracle_partial_state(x["q_t"], x["k_t"][:, :, a:b], x["q_s"], x["k_s"][:, :, a:b],
+                                   st, ss, causal, a, 900)
+        got = states[r]
+        live = ref[2] > 0
+        assert torch.equal(live, got[2] > 0)
+        LN2 = math.log(2)
+        check_lse(torch.where(live, LN2 * (got[0] + torch.log2(got[2])), -math.inf),
+                  torch.where(live, LN2 * (ref[0] + torch.log2(ref[2])), -math.inf))
+        e_got, e_ref = got[4][live] / got[2][live], ref[4][live] / ref[2][live]
+        assert (e_got - e_ref).abs().max().item() <= 1e-3 * max(1.0, e_ref.abs().max().item())
+
+
+def test_context_parallel_one_shard_is_the_forward_bitwise():
+    w = WORKLOADS["b2h16_n4096_d128_causal"].with_sizes(B=1, H=2, N_Q=500, N_K=640)
+    x = to_dev(make_inputs(w, seed=92))
+    a = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S, True)
+    kl, lt, ls = skl.streamkl_fwd(*a)
+    kl1, lt1, ls1 = skl.streamkl_merge_partial(skl.streamkl_fwd_partial(*a, 0, 640).unsqueeze(0))
+    dq, dk = skl.streamkl_bwd(*a, lt, ls, x["g"])
+    dq1, dk1 = skl.streamkl_bwd_shard(*a, 0, 640, lt1, ls1, x["g"])
+    assert skl.device_status() == 0
+    assert torch.equal(kl, kl1) and torch.equal(lt, lt1) and torch.equal(ls, ls1)
+    assert torch.equal(dk, dk1) and rel_fro(dq1.cpu().double(), dq.cpu().double()) < 1e-6
+
+
+def test_context_parallel_autograd_single_rank():
+    from attention_kl_divergence_fwd_b200.autograd import attention_kl
+    from attention_kl_divergence_fwd_b200.context_parallel import attention_kl_context_parallel
+    w = WORKLOADS["tiny_n256_d64"]
+    x = to_dev(make_inputs(w, seed=93))
+    grads = []
+    for fn in (lambda q, k: attention_kl(x["q_t"], x["k_t"], q, k, causal=True),
+               lambda q, k: attention_kl_context_parallel(x["q_t"], x["k_t"], q, k, 0, 256,
+                                                          causal=True)):
+        q_s = x["q_s"].clone().requires_grad_(True)
+        k_s = x["k_s"].clone().requires_grad_(True)
+        kl = fn(q_s, k_s)
+        (kl * x["g"]).sum().backward()
+        grads.append((kl.detach(), q_s.grad.float(), k_s.grad.float()))
+    assert torch.equal(grads[0][0], grads[1][0])
+    assert torch.equal(grads[0][2], grads[1][2])
+    assert rel_fro(grads[1][1].cpu().double(), grads[0][1].cpu().double()) < 1e-2
