@@ -337,6 +337,7 @@ def main():
         del k_s4, dk4
 
     varlen = run_varlen(skl, w, dev, stream, args.steps, world) if w.d_T == w.d_S else None
+    cp = run_context_parallel(skl, w, d, dev, stream, args.steps, world)
 
     e2e = None
     if not args.no_e2e:
@@ -356,7 +357,7 @@ def main():
                "fwd_frac_burst_peak": fwd_tf / peak_burst,
                "bwd_frac_burst_peak": bwd_tf / peak_burst,
                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-               "gqa": gqa, "varlen": varlen,
+               "gqa": gqa, "varlen": varlen, "context_parallel": cp,
                "bwd_teacher_ms": bwd_t_ms,
                "bwd_teacher_tflops": flops_bwd_teacher(w) / (bwd_t_ms * 1e-3) / 1e12,
                "gpu_launches": 2 * args.steps,
@@ -402,6 +403,61 @@ def run_varlen(skl, w, dev, stream, steps, world, tokens=65536, lo=512, hi=8192)
     return {"tokens": tokens, "sequences": len(lens), "lengths": f"seeded uniform {lo}..{hi}",
             "fwd_ms": fms, "bwd_ms": bms, "fwd_tflops": ff / (fms * 1e-3) / 1e12,
             "bwd_tflops": fb / (bms * 1e-3) / 1e12}
+
+
+def run_context_parallel(skl, w, d, dev, stream, steps, world, shards=4):
+    """The workload with its keys split into ``shards`` contiguous shards, run one after
+    another on this GPU as the shard ranks of a context-parallel group would run them
+    side by side: partial forwards, the merge of their states, shard backwards. The
+    all-gather / all-reduce between ranks is not part of it (one GPU)."""
+    from attention_kl_divergence_fwd_b200.context_parallel import even_shards
+    cuts = even_shards(w.N_K, shards)
+    ks = [(d["k_t"][:, :, a:a + n].contiguous(), d["k_s"][:, :, a:a + n].contiguous(), a)
+          for a, n in cuts]
+    B, H, nq = w.B, w.H, w.N_Q
+    states = torch.empty(shards, 5, B, H, nq, device=dev)
+    kl = torch.empty(B, H, nq, device=dev)
+    lt, ls = torch.empty_like(kl), torch.empty_like(kl)
+    dq = torch.empty(B, H, nq, w.d_S, device=dev)
+    dks = [torch.empty(B, H, kt.shape[2], w.d_S, device=dev) for kt, _, _ in ks]
+    base = (d["q_t"], d["q_s"])
+
+    def fwd():
+        for r, (kt, kss, a) in enumerate(ks):
+            skl.streamkl_fwd_partial(base[0], kt, base[1], kss, w.scale_T, w.scale_S, w.causal,
+                                     a, w.N_K, state=states[r])
+
+    def merge():
+        skl.streamkl_merge_partial(states, kl=kl, lse_t=lt, lse_s=ls)
+
+    def bwd():
+        for r, (kt, kss, a) in enumerate(ks):
+            skl.streamkl_bwd_shard(base[0], kt, base[1], kss, w.scale_T, w.scale_S, w.causal, a,
+                                   w.N_K, lt, ls, d["g"], dq_s=dq, dk_s=dks[r])
+
+    for _ in range(3):
+        fwd(); merge(); bwd()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ev[0].record(stream)
+    for _ in range(steps):
+        fwd()
+    ev[1].record(stream)
+    for _ in range(steps):
+        merge()
+    ev[2].record(stream)
+    for _ in range(steps):
+        bwd()
+    ev[3].record(stream)
+    torch.cuda.synchronize()
+    if skl.device_status() != 0:
+        raise RuntimeError("kernel watchdog fired in the context-parallel run")
+    t = [max_over_ranks(ev[i].elapsed_time(ev[i + 1]) / steps, world) for i in range(3)]
+    merge_bytes = (shards * 20 + 12) * B * H * nq
+    return {"shards": shards, "fwd_partial_ms": t[0], "merge_ms": t[1], "bwd_shard_ms": t[2],
+            "fwd_tflops": flops_fwd(w) / ((t[0] + t[1]) * 1e-3) / 1e12,
+            "bwd_tflops": flops_bwd(w) / (t[2] * 1e-3) / 1e12,
+            "merge_gbs": merge_bytes / (t[1] * 1e-3) / 1e9}
 
 
 def run_e2e(skl, w, x, dev, stream, steps, world):
