@@ -7,19 +7,21 @@
 // CTA = two 128-row query tiles of one (batch, head). Key tiles of 64 rows stream
 // through a TMA ring. Per key tile and query tile the tensor core computes the teacher
 // and student score tiles into TMEM (two buffers per query tile, so the next tile is
-// computed while the current one is folded). One warpgroup per query tile, one thread
-// per query row, folds each tile into the row's online state
+// computed while the current one is folded). Each query row is folded by two threads
+// (one per 32-key half of every tile), each keeping its own online state
 //     m_T, m_S   running maxima of t = s * log2(e)
 //     l_T, l_S   running sums of 2^(t - m)
 //     A          running sum of 2^(t_T - m_T) * (t_T - t_S)
-// so that KL = ln2 * A / l_T - LSE_T + LSE_S at the end. Per tile: one pass over TMEM
-// for the row maxima, a second pass (two 32-key halves) for the exponentials, with the
-// fp32 work issued as packed pairs and a share of the exponentials on the FMA pipe.
+// which merge at the end, so that KL = ln2 * A / l_T - LSE_T + LSE_S. Per tile a thread
+// reads its 64 scores from TMEM in one round trip and releases the buffer at once; the
+// fp32 work is issued as packed pairs, with a share of the exponentials on the FMA pipe.
 // Nothing of size N_Q x N_K ever leaves the SM.
 //
-// Warp roles (384 threads): warps 0-3 query tile 0, warps 4-7 query tile 1 (224 registers
-// each), warp 8 TMA producer, warp 9 TMEM allocator + MMA issuer, warps 10-11 idle (the
-// control warpgroup runs with 56 registers).
+// Warp roles (640 threads, SKL_FWD_SPLIT): warps 0-7 query tile 0 and 8-15 query tile 1
+// (warps 4k..4k+3 cover the tile's four 32-row quarters for one key half; 104 registers
+// each), warp 16 TMA producer, warp 17 TMEM allocator + MMA issuer, warps 18-19 idle (the
+// control warpgroup runs with 56 registers). With SKL_FWD_SPLIT = 0: 384 threads, one
+// thread per row over whole tiles (200 registers), warps 8 / 9 TMA / MMA.
 #pragma once
 
 #include "ptx.cuh"
@@ -45,6 +47,30 @@ struct FwdArgs {
   float* lse_s;
 };
 
+// Warp layout. Default: 8 statistics warps (one thread per query row, whole key tiles).
+// SKL_FWD_SPLIT: 16 statistics warps, two per row quarter, each folding one half (32 keys)
+// of every tile into its own row state; the two states merge once at the end.
+#ifndef SKL_FWD_SPLIT
+#define SKL_FWD_SPLIT 1
+#endif
+constexpr int kFwdHalves = SKL_FWD_SPLIT ? 2 : 1;        // key halves per tile
+constexpr int kFwdStatWarps = 8 * kFwdHalves;            // warps 0 .. kFwdStatWarps-1
+constexpr int kFwdTmaWarp = kFwdStatWarps;               // TMA producer
+constexpr int kFwdMmaWarp = kFwdStatWarps + 1;           // TMEM owner + MMA issuer
+constexpr int kFwdThreads = 32 * (kFwdStatWarps + 4);    // + TMA, MMA and two idle warps
+// Registers after setmaxnreg: statistics / control warps (sum within the launch's pool).
+#ifndef SKL_FWD_RS
+#define SKL_FWD_RS (SKL_FWD_SPLIT ? 104 : 200)
+#endif
+#ifndef SKL_FWD_RC
+#define SKL_FWD_RC (SKL_FWD_SPLIT ? 56 : 104)
+#endif
+constexpr int kFwdRegsStat = SKL_FWD_RS;
+constexpr int kFwdRegsCtrl = SKL_FWD_RC;
+static_assert(kFwdStatWarps * kFwdRegsStat + 4 * kFwdRegsCtrl <=
+                  (kFwdStatWarps + 4) * ((65536 / kFwdThreads) & ~7),
+              "register split exceeds the launch's register pool");
+
 template <int DT, int DS>
 struct FwdCfg {
   static constexpr int BM = 128;  // query rows per tile = TMEM lanes
@@ -61,7 +87,7 @@ struct FwdCfg {
   static constexpr int NST_FIT = (SMEM_MAX - BAR_BYTES - QBYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
   static constexpr int SMEM = QBYTES + NST * STAGE + BAR_BYTES;  // base is 1024-aligned
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = kFwdThreads;
   static_assert(NST >= 2, "key ring needs two stages");
   static_assert(SMEM <= SMEM_MAX, "shared memory budget");
 };
@@ -87,12 +113,17 @@ struct RowState {
   float mT, mS, lT, lS, A;
 };
 
-// Which column pairs (c, c+1) of a 32-key chunk send their second exponential of both
-// distributions to the FMA pipe: pairs 1, 3, 5, 7 of every 8 (25 % of the exponentials),
-// plus pair 6 when kPolyHeavy (37.5 %).
-constexpr bool kPolyHeavy = true;
+// Which column pairs (c, c+1) send their second exponential of both distributions to the
+// FMA pipe: the first SKL_FWD_POLY entries of the order 1, 5, 3, 7, 6, 2, 4, 0 over every 8
+// consecutive pairs, i.e. SKL_FWD_POLY/16 of all exponentials (2: 12.5 %).
+#ifndef SKL_FWD_POLY
+#define SKL_FWD_POLY 2
+#endif
+__host__ __device__ constexpr int poly_rank(int p) {
+  return p == 1 ? 0 : p == 5 ? 1 : p == 3 ? 2 : p == 7 ? 3 : p == 6 ? 4 : p == 2 ? 5 : p == 4 ? 6 : 7;
+}
 __host__ __device__ constexpr bool poly_pair(int pair) {
-  return (pair & 1) || (kPolyHeavy && (pair & 7) == 6);
+  return poly_rank(pair & 7) < SKL_FWD_POLY;
 }
 
 // New running maxima from a tile's raw maxima; rescales the sums when any row of the
@@ -114,17 +145,18 @@ __device__ __forceinline__ void update_max(RowState& st, float mxT, float mxS, f
   st.mS = mS_new;
 }
 
-// Accumulates 16 keys (v[0..15] teacher scores, v[16..31] student scores, raw dot
+// Accumulates 16 keys (v[tb..tb+15] teacher scores, v[sb..sb+15] student scores, raw dot
 // products) into the packed partial sums. Columns c > lim are masked (MASK).
-template <bool MASK>
-__device__ __forceinline__ void fold_part(const uint32_t (&v)[32], uint64_t cT2, uint64_t cS2,
-                                          uint64_t nmT2, uint64_t nmS2, int lim, int pair0,
-                                          uint64_t& sT2, uint64_t& sS2, uint64_t& b2) {
+template <bool MASK, int N>
+__device__ __forceinline__ void fold_part(const uint32_t (&v)[N], int tb, int sb, uint64_t cT2,
+                                          uint64_t cS2, uint64_t nmT2, uint64_t nmS2, int lim,
+                                          int pair0, uint64_t& sT2, uint64_t& sS2, uint64_t& b2) {
 #pragma unroll
   for (int c = 0; c < 16; c += 2) {
-    const uint64_t xT = f2_fma(f2_pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), cT2, nmT2);
+    const uint64_t xT =
+        f2_fma(f2_pack(__uint_as_float(v[tb + c]), __uint_as_float(v[tb + c + 1])), cT2, nmT2);
     const uint64_t xS =
-        f2_fma(f2_pack(__uint_as_float(v[16 + c]), __uint_as_float(v[16 + c + 1])), cS2, nmS2);
+        f2_fma(f2_pack(__uint_as_float(v[sb + c]), __uint_as_float(v[sb + c + 1])), cS2, nmS2);
     float xT0, xT1, xS0, xS1;
     f2_unpack(xT, xT0, xT1);
     f2_unpack(xS, xS0, xS1);
@@ -159,29 +191,24 @@ template <bool MASK>
 __device__ __forceinline__ void fold_tile(RowState& st, uint32_t ta, float cT, float cS, int lim,
                                           uint32_t s_free, int lane) {
   float mxT, mxS;
-  {
-    uint32_t v[64];
-    tmem_ld_2x32_wait(ta, ta + 32, v);
-    mxT = fmaxf(max_tree32<MASK>(v, 0, lim), max_tree32<MASK>(v, 32, lim - 32));
-    tmem_ld_2x32_wait(ta + 64, ta + 96, v);
-    mxS = fmaxf(max_tree32<MASK>(v, 0, lim), max_tree32<MASK>(v, 32, lim - 32));
-  }
+  // One TMEM round trip for the whole tile (v[0..63] teacher, v[64..127] student); the
+  // buffer is released at once, so the next tile's MMAs overlap all of the arithmetic.
+  uint32_t v[128];
+  tmem_ld_4x32_wait(ta, ta + 32, ta + 64, ta + 96, v);
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(s_free);
+  mxT = fmaxf(max_tree32<MASK>(v, 0, lim), max_tree32<MASK>(v, 32, lim - 32));
+  mxS = fmaxf(max_tree32<MASK>(v, 64, lim), max_tree32<MASK>(v, 96, lim - 32));
   float mT_use, mS_use;
   update_max(st, mxT, mxS, cT, cS, mT_use, mS_use);
   const uint64_t cT2 = f2_pack(cT, cT), cS2 = f2_pack(cS, cS);
   const uint64_t nmT2 = f2_pack(-mT_use, -mT_use), nmS2 = f2_pack(-mS_use, -mS_use);
   uint64_t sT2 = f2_pack(0.f, 0.f), sS2 = sT2, b2 = sT2;
 #pragma unroll
-  for (int h = 0; h < 4; ++h) {
-    uint32_t v[32];  // keys 16h .. 16h+15: v[0..15] teacher, v[16..31] student
-    tmem_ld_2x16_wait(ta + 16 * h, ta + 64 + 16 * h, v);
-    if (h == 3) {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-    }
-    fold_part<MASK>(v, cT2, cS2, nmT2, nmS2, lim - 16 * h, 8 * h, sT2, sS2, b2);
-  }
+  for (int h = 0; h < 4; ++h)
+    fold_part<MASK>(v, 16 * h, 64 + 16 * h, cT2, cS2, nmT2, nmS2, lim - 16 * h, 8 * h, sT2, sS2,
+                    b2);
   float s0, s1, u0, u1, w0, w1;
   f2_unpack(sT2, s0, s1);
   f2_unpack(sS2, u0, u1);
@@ -192,8 +219,52 @@ __device__ __forceinline__ void fold_tile(RowState& st, uint32_t ta, float cT, f
   st.A += (w0 + w1) + (mT_use - mS_use) * sumT;
 }
 
+// Half a tile (32 keys: TMEM columns tT .. tT+31 teacher, tS .. tS+31 student) folded
+// into the row state of one warp of a split pair; lim as in fold_tile, relative to the
+// half's first key.
+template <bool MASK>
+__device__ __forceinline__ void fold_half(RowState& st, uint32_t tT, uint32_t tS, float cT,
+                                          float cS, int lim, uint32_t s_free, int lane) {
+  uint32_t v[64];
+  tmem_ld_2x32_wait(tT, tS, v);
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(s_free);
+  const float mxT = max_tree32<MASK>(v, 0, lim), mxS = max_tree32<MASK>(v, 32, lim);
+  float mT_use, mS_use;
+  update_max(st, mxT, mxS, cT, cS, mT_use, mS_use);
+  const uint64_t cT2 = f2_pack(cT, cT), cS2 = f2_pack(cS, cS);
+  const uint64_t nmT2 = f2_pack(-mT_use, -mT_use), nmS2 = f2_pack(-mS_use, -mS_use);
+  uint64_t sT2 = f2_pack(0.f, 0.f), sS2 = sT2, b2 = sT2;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+    fold_part<MASK>(v, 16 * h, 32 + 16 * h, cT2, cS2, nmT2, nmS2, lim - 16 * h, 8 * h, sT2, sS2,
+                    b2);
+  float s0, s1, u0, u1, w0, w1;
+  f2_unpack(sT2, s0, s1);
+  f2_unpack(sS2, u0, u1);
+  f2_unpack(b2, w0, w1);
+  const float sumT = s0 + s1;
+  st.lT += sumT;
+  st.lS += u0 + u1;
+  st.A += (w0 + w1) + (mT_use - mS_use) * sumT;
+}
+
+// Merge of two row states (rescale both to the larger maxima and add).
+__device__ __forceinline__ void merge_state(RowState& a, const RowState& b) {
+  const float nT = fmaxf(a.mT, b.mT), nS = fmaxf(a.mS, b.mS);
+  const float uT = nT == -INFINITY ? 0.f : nT, uS = nS == -INFINITY ? 0.f : nS;
+  const float aT = ex2_approx(a.mT - uT), bT = ex2_approx(b.mT - uT);
+  const float aS = ex2_approx(a.mS - uS), bS = ex2_approx(b.mS - uS);
+  a.lT = a.lT * aT + b.lT * bT;
+  a.A = a.A * aT + b.A * bT;
+  a.lS = a.lS * aS + b.lS * bS;
+  a.mT = nT;
+  a.mS = nS;
+}
+
 template <int DT, int DS>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
 streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                     const __grid_constant__ CUtensorMap map_kt,
                     const __grid_constant__ CUtensorMap map_qs,
@@ -256,13 +327,13 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     for (int q = 0; q < 2; ++q)
       for (int b = 0; b < 2; ++b) {
         mbar_init(smem_u32(&bars->s_full[q][b]), 1);
-        mbar_init(smem_u32(&bars->s_free[q][b]), 4);
+        mbar_init(smem_u32(&bars->s_free[q][b]), 4 * kFwdHalves);
       }
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kFwdMmaWarp) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
   }
@@ -271,11 +342,12 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp < 8) {
-    regs_inc<200>();
+  if (warp < kFwdStatWarps) {
+    regs_inc<kFwdRegsStat>();
     // --------------------------------------------------- statistics warpgroups
-    const int q = warp >> 2;          // query tile of this warpgroup
-    const int quarter = warp & 3;     // TMEM lane quarter of this warp
+    const int q = warp / (4 * kFwdHalves);           // query tile of this warp
+    const int half = (warp >> 2) & (kFwdHalves - 1);  // key half of every tile (split)
+    const int quarter = warp & 3;                     // TMEM lane quarter of this warp
     const int row = q0 + q * C::BM + quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float cT = args.cT, cS = args.cS;
@@ -299,13 +371,48 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       if (need_mask) {
         int last = seq.nk - 1;
         if (args.causal) last = min(last, row + seq.off);
+#if SKL_FWD_SPLIT
+        fold_half<true>(st, ta + 32 * half, ta + 64 + 32 * half, cT, cS, last - k0 - 32 * half,
+                        fr, lane);
+#else
         fold_tile<true>(st, ta, cT, cS, last - k0, fr, lane);
+#endif
       } else {
+#if SKL_FWD_SPLIT
+        fold_half<false>(st, ta + 32 * half, ta + 64 + 32 * half, cT, cS, 31, fr, lane);
+#else
         fold_tile<false>(st, ta, cT, cS, C::BN - 1, fr, lane);
+#endif
       }
     }
 
-    if (ok && row < seq.nq) {
+#if SKL_FWD_SPLIT
+    // Half 1 hands its row state to half 0 through this query tile's shared memory: it is
+    // no longer read once the tile's MMAs have completed (the last s_full), and its TMA
+    // load has landed (q_full; also covers a tile with no keys, never read by an MMA).
+    float* xfer = reinterpret_cast<float*>(smem + q * C::QT_TILE);
+    const int r = quarter * 32 + lane;
+    if (half == 1) {
+      if (!mbar_wait(smem_u32(&bars->q_full), 0)) {
+        skl_fail(abort_flag);
+        ok = false;
+      }
+      xfer[r] = st.mT;
+      xfer[128 + r] = st.mS;
+      xfer[256 + r] = st.lT;
+      xfer[384 + r] = st.lS;
+      xfer[512 + r] = st.A;
+      xfer[640 + r] = ok ? 1.f : 0.f;
+    }
+    named_bar_sync(1 + q, 8 * 32);  // the 8 warps of query tile q
+    if (half == 0) {
+      const RowState other{xfer[r], xfer[128 + r], xfer[256 + r], xfer[384 + r], xfer[512 + r]};
+      ok = ok && xfer[640 + r] != 0.f;
+      merge_state(st, other);
+    }
+#endif
+
+    if (ok && row < seq.nq && half == 0) {
       const size_t o = (size_t)(seq.ob + row);
       if (args.state) {
         float* p = args.state + o;
@@ -323,8 +430,8 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       }
     }
   } else {
-    regs_dec<104>();
-    if (warp == 8) {
+    regs_dec<kFwdRegsCtrl>();
+    if (warp == kFwdTmaWarp) {
       // ------------------------------------------------------------ TMA producer
       if (elect_one()) {
         tma_prefetch_desc(&map_qt);
@@ -368,7 +475,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
             mbar_wait(smem_u32(&bars->full[j % C::NST]), (j / C::NST) & 1);
         }
       }
-    } else if (warp == 9) {
+    } else if (warp == kFwdMmaWarp) {
       // ------------------------------------------------------------- MMA issuer
       if (elect_one()) {
         bool ok = mbar_wait(smem_u32(&bars->q_full), 0);
@@ -423,7 +530,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kFwdMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
