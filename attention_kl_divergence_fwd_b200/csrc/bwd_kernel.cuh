@@ -62,6 +62,13 @@ struct BwdArgs {
   float* dk;        // dK of the differentiated side (fp32, the layout of K)
 };
 
+// SKL_BWD_KTMEM: the K tiles are also copied into tensor memory (one key row per lane),
+// where the score MMAs read them as their A operand instead of re-reading them from
+// shared memory every step; the score tile is then single-buffered to make room.
+#ifndef SKL_BWD_KTMEM
+#define SKL_BWD_KTMEM 0
+#endif
+
 // TEACHER = false: gradients of the student (dQ_S, dK_S), d_G = d_S.
 // TEACHER = true: gradients of a trainable teacher (dQ_T, dK_T), d_G = d_T.
 template <int DT, int DS, bool TEACHER = false>
@@ -90,11 +97,14 @@ struct BwdCfg {
   static constexpr int SMEM = OFF_BAR + BAR_BYTES;  // the dynamic base is 1024-byte aligned
   static constexpr int THREADS = 384;
   // TMEM columns: S_T^T / S_S^T per buffer, dK, dQ^T per buffer.
+  static constexpr int NSB = SKL_BWD_KTMEM ? 1 : 2;  // score-tile buffers
   static constexpr int TM_S = 0;          // buffer b: [128b, 128b+64) S_T, [+64, +128) S_S
-  static constexpr int TM_DK = 256;       // d_G columns
-  static constexpr int TM_DQ = 256 + DG;  // buffer b: + 64 b
+  static constexpr int TM_DK = 128 * NSB; // d_G columns
+  static constexpr int TM_DQ = TM_DK + DG;  // buffer b: + 64 b
+  static constexpr int TM_KT = TM_DQ + 2 * BM;  // SKL_BWD_KTMEM: K_T rows, d_T/2 columns
+  static constexpr int TM_KS = TM_KT + DT / 2;  //                K_S rows, d_S/2 columns
   static constexpr int DQ_M = DG;         // M of the dQ^T MMA (64 uses half the lanes)
-  static_assert(TM_DQ + 2 * BM <= 512, "TMEM budget");
+  static_assert((SKL_BWD_KTMEM ? TM_KS + DS / 2 : TM_DQ + 2 * BM) <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -106,6 +116,7 @@ struct BwdBars {
   uint64_t ds_full[2], ds_empty[2];
   uint64_t dq_full[2], dq_free[2];
   uint64_t dk_full;
+  uint64_t k_tmem;  // SKL_BWD_KTMEM: the K rows are in tensor memory (8 warps arrive)
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -186,6 +197,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       mbar_init(smem_u32(&bars->stg_free[b]), 1);
     }
     mbar_init(smem_u32(&bars->dk_full), 1);
+    mbar_init(smem_u32(&bars->k_tmem), 8);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -332,6 +344,42 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     if (elect_one()) {
       const uint32_t s_kt = sb + C::OFF_KT, s_ks = sb + C::OFF_KS;
       bool ok = mbar_wait(smem_u32(&bars->k_full), 0);
+#if SKL_BWD_KTMEM
+      // The dS warps copy the K rows into tensor memory first.
+      if (ok) ok = mbar_wait(smem_u32(&bars->k_tmem), 0);
+      // S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T of step s into the single score buffer,
+      // A (the K rows) from tensor memory; the buffer is free once step s-1 has been read.
+      // Barriers stay per step parity (each warpgroup waits only on its own steps' phases).
+      auto issue_scores = [&](int s) -> bool {
+        const int st = s % C::NQST;
+        if (!mbar_wait(smem_u32(&bars->q_full[st]), (s / C::NQST) & 1)) return false;
+        if (s > 0 && !mbar_wait(smem_u32(&bars->s_free[(s - 1) & 1]), ((s - 1) >> 1) & 1))
+          return false;
+        tc_fence_after();
+        const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
+        const uint32_t d_t = tmem + C::TM_S, d_s = d_t + 64;
+#pragma unroll
+        for (int kk = 0; kk < DT / 16; ++kk) {
+          const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
+          umma_bf16_ts(d_t, tmem + C::TM_KT + kk * 8, sdesc_sw128(q_base + qa, 16, 1024),
+                       idesc_st, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < DS / 16; ++kk) {
+          const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
+          umma_bf16_ts(d_s, tmem + C::TM_KS + kk * 8,
+                       sdesc_sw128(q_base + C::QT_TILE + qa, 16, 1024), idesc_ss, kk > 0);
+        }
+        umma_commit(smem_u32(&bars->s_full[s & 1]));
+        return true;
+      };
+      if (ok && n_steps > 0) ok = issue_scores(0);
+      for (int p = 0; ok && p < n_steps; ++p) {
+        const int pb = p & 1, pst = p % C::NQST;
+        // Scores of step p+1 as soon as the warpgroup of step p has read its scores.
+        if (p + 1 < n_steps && !issue_scores(p + 1)) { ok = false; break; }
+        constexpr bool early = true;
+#else
       // S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T of step s into TMEM buffer s&1.
       auto issue_scores = [&](int s) -> bool {
         const int st = s % C::NQST, b = s & 1;
@@ -370,6 +418,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           if (!issue_scores(p + 2)) { ok = false; break; }
           early = true;
         }
+#endif
         if (!mbar_wait(smem_u32(&bars->ds_full[pb]), (p >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s_ds = sb + C::OFF_DS + pb * C::DS_TILE;
@@ -446,17 +495,40 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     };
 
     bool ok = true;
+#if SKL_BWD_KTMEM
+    {
+      // K rows into tensor memory (A operand of the score MMAs): warpgroup 0 copies K_T,
+      // warpgroup 1 copies K_S, one key row per thread.
+      if (mbar_wait(smem_u32(&bars->k_full), 0)) {
+        if (wg == 0)
+          row_to_tmem<DT>(sb + C::OFF_KT + kl * 128, tmem + lane_off + C::TM_KT, kl);
+        else
+          row_to_tmem<DS>(sb + C::OFF_KS + kl * 128, tmem + lane_off + C::TM_KS, kl);
+      } else {
+        ok = false;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->k_tmem));
+    }
+    constexpr int sbuf = 0;  // TMEM score buffer (single)
+#else
+    const int sbuf = wg;
+#endif
     int last = -1;
-    for (int s = wg; s < n_steps; s += 2) {
+    for (int s = wg; ok && s < n_steps; s += 2) {
       const int st = s % C::NQST;
       const int i0 = (jq_begin + s) * C::BM;  // first query column of this step
-      if (!mbar_wait(smem_u32(&bars->s_full[wg]), (s >> 1) & 1)) { ok = false; break; }
+      if (!mbar_wait(smem_u32(&bars->s_full[wg]), (s >> 1) & 1)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       uint32_t vt[64], vs[64];  // raw teacher / student scores of this key, 64 query columns
-      tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + wg * 128,
-                        tmem + lane_off + C::TM_S + wg * 128 + 32, vt);
-      tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + wg * 128 + 64,
-                        tmem + lane_off + C::TM_S + wg * 128 + 96, vs);
+      tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + sbuf * 128,
+                        tmem + lane_off + C::TM_S + sbuf * 128 + 32, vt);
+      tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + sbuf * 128 + 64,
+                        tmem + lane_off + C::TM_S + sbuf * 128 + 96, vs);
       // The score buffer can take step s+2 as soon as every lane has read it.
       tc_fence_before();
       __syncwarp();

@@ -59,6 +59,14 @@ constexpr int kFwdTmaWarp = kFwdStatWarps;               // TMA producer
 constexpr int kFwdMmaWarp = kFwdStatWarps + 1;           // TMEM owner + MMA issuer
 constexpr int kFwdThreads = 32 * (kFwdStatWarps + 4);    // + TMA, MMA and two idle warps
 // Registers after setmaxnreg: statistics / control warps (sum within the launch's pool).
+// SKL_FWD_QTMEM: the query tiles are also copied into tensor memory, where the score MMAs
+// read them as their A operand (an N = 64 MMA with both operands in shared memory is
+// bound by shared-memory bandwidth); each query tile's score buffer is then single.
+#ifndef SKL_FWD_QTMEM
+#define SKL_FWD_QTMEM 1
+#endif
+static_assert(!SKL_FWD_QTMEM || SKL_FWD_SPLIT, "the Q copy into TMEM assumes split warps");
+
 #ifndef SKL_FWD_RS
 #define SKL_FWD_RS (SKL_FWD_SPLIT ? 104 : 200)
 #endif
@@ -88,6 +96,14 @@ struct FwdCfg {
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
   static constexpr int SMEM = QBYTES + NST * STAGE + BAR_BYTES;  // base is 1024-aligned
   static constexpr int THREADS = kFwdThreads;
+  // TMEM columns: score buffers (query tile q, buffer b), and with SKL_FWD_QTMEM the
+  // query rows (Q_T: d_T/2 columns, Q_S: d_S/2 columns per query tile).
+  static constexpr int NSB = SKL_FWD_QTMEM ? 1 : 2;
+  static __device__ __forceinline__ int tm_s(int q, int b) { return (q * NSB + b % NSB) * 128; }
+  static constexpr int TM_Q = NQ * NSB * 128;
+  static __device__ __forceinline__ int tm_qt(int q) { return TM_Q + q * (DT + DS) / 2; }
+  static __device__ __forceinline__ int tm_qs(int q) { return tm_qt(q) + DT / 2; }
+  static_assert(!SKL_FWD_QTMEM || TM_Q + NQ * (DT + DS) / 2 <= 512, "TMEM budget");
   static_assert(NST >= 2, "key ring needs two stages");
   static_assert(SMEM <= SMEM_MAX, "shared memory budget");
 };
@@ -98,6 +114,7 @@ struct FwdBars {
   uint64_t empty[4];
   uint64_t s_full[2][2];
   uint64_t s_free[2][2];
+  uint64_t q_tmem;  // SKL_FWD_QTMEM: the query rows are in tensor memory
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -329,6 +346,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         mbar_init(smem_u32(&bars->s_full[q][b]), 1);
         mbar_init(smem_u32(&bars->s_free[q][b]), 4 * kFwdHalves);
       }
+    mbar_init(smem_u32(&bars->q_tmem), kFwdStatWarps);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -355,7 +373,26 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
 
     RowState st{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
     bool ok = true;
-    for (int j = 0; j < nk[q]; ++j) {
+#if SKL_FWD_QTMEM
+    {
+      // Query rows into tensor memory (A operand of the score MMAs): half 0 copies the
+      // row of Q_T, half 1 the row of Q_S.
+      const int r = quarter * 32 + lane;
+      if (mbar_wait(smem_u32(&bars->q_full), 0)) {
+        if (half == 0)
+          row_to_tmem<DT>(s_qt + q * C::QT_TILE + r * 128, tmem + lane_off + C::tm_qt(q), r);
+        else
+          row_to_tmem<DS>(s_qs + q * C::QS_TILE + r * 128, tmem + lane_off + C::tm_qs(q), r);
+      } else {
+        skl_fail(abort_flag);
+        ok = false;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->q_tmem));
+    }
+#endif
+    for (int j = 0; ok && j < nk[q]; ++j) {
       const int b = j & 1;
       if (!mbar_wait(smem_u32(&bars->s_full[q][b]), (j >> 1) & 1)) {
         skl_fail(abort_flag);
@@ -366,7 +403,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       const int k0 = j * C::BN;
       const bool need_mask =
           (k0 + C::BN > seq.nk) || (args.causal && k0 + C::BN - 1 > first_row + seq.off);
-      const uint32_t ta = tmem + lane_off + q * 256 + b * 128;
+      const uint32_t ta = tmem + lane_off + C::tm_s(q, b);
       const uint32_t fr = smem_u32(&bars->s_free[q][b]);
       if (need_mask) {
         int last = seq.nk - 1;
@@ -479,6 +516,9 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       // ------------------------------------------------------------- MMA issuer
       if (elect_one()) {
         bool ok = mbar_wait(smem_u32(&bars->q_full), 0);
+#if SKL_FWD_QTMEM
+        if (ok) ok = mbar_wait(smem_u32(&bars->q_tmem), 0);
+#endif
         if (!ok) skl_fail(abort_flag);
         for (int j = 0; ok && j < nk_max; ++j) {
           const int s = j % C::NST;
@@ -492,14 +532,34 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           for (int q = 0; q < C::NQ; ++q) {
             if (j >= nk[q]) continue;
             const int b = j & 1;
+#if SKL_FWD_QTMEM
+            // Single score buffer: free once tile j-1 has been read (per-parity barriers,
+            // so every waiter sees each phase of its barrier in order).
+            if (j > 0 && !mbar_wait(smem_u32(&bars->s_free[q][(j - 1) & 1]), ((j - 1) >> 1) & 1)) {
+#else
             if (!mbar_wait(smem_u32(&bars->s_free[q][b]), ((j >> 1) & 1) ^ 1)) {
+#endif
               skl_fail(abort_flag);
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t d_t = tmem + q * 256 + b * 128;
+            const uint32_t d_t = tmem + C::tm_s(q, b);
             const uint32_t d_s = d_t + 64;
+#if SKL_FWD_QTMEM
+  #pragma unroll
+            for (int kk = 0; kk < DT / 16; ++kk) {
+              const uint64_t bd =
+                  sdesc_sw128(st + (kk >> 2) * (C::BN * 128) + (kk & 3) * 32, 16, 1024);
+              umma_bf16_ts(d_t, tmem + C::tm_qt(q) + kk * 8, bd, idesc_t, kk > 0);
+            }
+  #pragma unroll
+            for (int kk = 0; kk < DS / 16; ++kk) {
+              const uint64_t bd = sdesc_sw128(
+                  st + C::KT_TILE + (kk >> 2) * (C::BN * 128) + (kk & 3) * 32, 16, 1024);
+              umma_bf16_ts(d_s, tmem + C::tm_qs(q) + kk * 8, bd, idesc_s, kk > 0);
+            }
+#else
   #pragma unroll
             for (int kk = 0; kk < DT / 16; ++kk) {
               const uint32_t off = (kk & 3) * 32;
@@ -517,6 +577,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                   sdesc_sw128(st + C::KT_TILE + (kk >> 2) * (C::BN * 128) + off, 16, 1024);
               umma_bf16_ss(d_s, a, bd, idesc_s, kk > 0);
             }
+#endif
             umma_commit(smem_u32(&bars->s_full[q][b]));
           }
           umma_commit(smem_u32(&bars->empty[s]));
