@@ -69,6 +69,30 @@ struct BwdArgs {
 #define SKL_BWD_KTMEM 0
 #endif
 
+// Warp layout. Default (SKL_BWD_SPLIT): 16 dS warps; warp w takes the steps of parity
+// (w >> 2) & 1, query columns 32 (w >> 3) .. +31 of each step and key rows
+// 32 (w & 3) .. +31 (its TMEM lane quarter). SKL_BWD_SPLIT = 0: 8 dS warps, all 64 columns.
+#ifndef SKL_BWD_SPLIT
+#define SKL_BWD_SPLIT 0
+#endif
+constexpr int kBwdHalves = SKL_BWD_SPLIT ? 2 : 1;      // query-column halves per step
+constexpr int kBwdDsWarps = 8 * kBwdHalves;            // warps 0 .. kBwdDsWarps-1
+constexpr int kBwdTmaWarp = kBwdDsWarps;               // TMA producer
+constexpr int kBwdMmaWarp = kBwdDsWarps + 1;           // TMEM owner + MMA issuer
+constexpr int kBwdStatWarp = kBwdDsWarps + 2;          // row-statistics loader
+constexpr int kBwdRedWarp = kBwdDsWarps + 3;           // dQ / dK reduce issuer
+constexpr int kBwdThreads = 32 * (kBwdDsWarps + 4);
+constexpr int kBwdArrive = 4 * kBwdHalves;             // dS warps working on one step
+#ifndef SKL_BWD_RS
+#define SKL_BWD_RS 96
+#endif
+#ifndef SKL_BWD_RC
+#define SKL_BWD_RC 88
+#endif
+static_assert(!SKL_BWD_SPLIT || kBwdDsWarps * SKL_BWD_RS + 4 * SKL_BWD_RC <=
+                                    (kBwdDsWarps + 4) * ((65536 / kBwdThreads) & ~7),
+              "register split exceeds the launch's register pool");
+
 // TEACHER = false: gradients of the student (dQ_S, dK_S), d_G = d_S.
 // TEACHER = true: gradients of a trainable teacher (dQ_T, dK_T), d_G = d_T.
 template <int DT, int DS, bool TEACHER = false>
@@ -95,7 +119,7 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_ST + NSTS * STATS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES;  // the dynamic base is 1024-byte aligned
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = kBwdThreads;
   // TMEM columns: S_T^T / S_S^T per buffer, dK, dQ^T per buffer.
   static constexpr int NSB = SKL_BWD_KTMEM ? 1 : 2;  // score-tile buffers
   static constexpr int TM_S = 0;          // buffer b: [128b, 128b+64) S_T, [+64, +128) S_S
@@ -128,7 +152,7 @@ __device__ __forceinline__ void skl_fail_b(volatile int* abort_flag) {
 }
 
 template <int DT, int DS, bool TEACHER>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
 streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
                     const __grid_constant__ CUtensorMap map_kt,
                     const __grid_constant__ CUtensorMap map_qs,
@@ -182,27 +206,27 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     }
     for (int i = 0; i < C::NSTS; ++i) {
       mbar_init(smem_u32(&bars->st_full[i]), 32);
-      mbar_init(smem_u32(&bars->st_empty[i]), 4);
+      mbar_init(smem_u32(&bars->st_empty[i]), kBwdArrive);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&bars->s_full[b]), 1);
-      mbar_init(smem_u32(&bars->s_free[b]), 4);
-      mbar_init(smem_u32(&bars->ds_full[b]), 4);
+      mbar_init(smem_u32(&bars->s_free[b]), kBwdArrive);
+      mbar_init(smem_u32(&bars->ds_full[b]), kBwdArrive);
       mbar_init(smem_u32(&bars->ds_empty[b]), 1);
       mbar_init(smem_u32(&bars->dq_full[b]), 1);
-      mbar_init(smem_u32(&bars->dq_free[b]), 4);
+      mbar_init(smem_u32(&bars->dq_free[b]), kBwdArrive);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&bars->stg_full[b]), 4);
+      mbar_init(smem_u32(&bars->stg_full[b]), kBwdArrive);
       mbar_init(smem_u32(&bars->stg_free[b]), 1);
     }
     mbar_init(smem_u32(&bars->dk_full), 1);
-    mbar_init(smem_u32(&bars->k_tmem), 8);
+    mbar_init(smem_u32(&bars->k_tmem), kBwdDsWarps);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kBwdMmaWarp) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
   }
@@ -211,249 +235,260 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 8) {
-    // ----------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      const uint64_t keep = l2_policy_evict_last();
-      int issued = 0;
-      tma_prefetch_desc(&map_qt);
-      tma_prefetch_desc(&map_kt);
-      tma_prefetch_desc(&map_qs);
-      tma_prefetch_desc(&map_ks);
-      const uint32_t kb = smem_u32(&bars->k_full);
-      mbar_arrive_expect_tx(kb, C::KT_TILE + C::KS_TILE);
-      for (int blk = 0; blk < DT / 64; ++blk)
-        tma_load_3d(sb + C::OFF_KT + blk * (C::BN * 128), &map_kt, kb, blk * 64, seq.kr + k0,
-                    seq.zkt, keep);
-      for (int blk = 0; blk < DS / 64; ++blk)
-        tma_load_3d(sb + C::OFF_KS + blk * (C::BN * 128), &map_ks, kb, blk * 64, seq.kr + k0,
-                    seq.zks, keep);
-      for (int s = 0; s < n_steps; ++s) {
-        const int st = s % C::NQST;
-        const int i0 = seq.qr + (jq_begin + s) * C::BM;
-        if (!mbar_wait(smem_u32(&bars->q_empty[st]), ((s / C::NQST) & 1) ^ 1)) {
-          skl_fail_b(abort_flag);
-          break;
-        }
-        const uint32_t fb = smem_u32(&bars->q_full[st]);
-        const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
-        mbar_arrive_expect_tx(fb, C::Q_STAGE);
-        for (int blk = 0; blk < DT / 64; ++blk)
-          tma_load_3d(q_base + blk * (C::BM * 128), &map_qt, fb, blk * 64, i0, seq.zq, keep);
-        for (int blk = 0; blk < DS / 64; ++blk)
-          tma_load_3d(q_base + C::QT_TILE + blk * (C::BM * 128), &map_qs, fb, blk * 64, i0,
-                      seq.zq, keep);
-        issued = s + 1;
-      }
-      if (*abort_flag) {
-        // Let every copy this thread started land before the CTA can exit.
-        mbar_wait(smem_u32(&bars->k_full), 0);
-        for (int s = max(0, issued - C::NQST); s < issued; ++s)
-          mbar_wait(smem_u32(&bars->q_full[s % C::NQST]), (s / C::NQST) & 1);
-      }
-    }
-  } else if (warp == 10) {
-    // ------------------------------------------------ row-statistics loader
-    // Each lane owns query rows lane and lane+32 of every step. Raw LSE_T, LSE_S, g (and
-    // KL for the teacher gradient) are loaded kStatAhead steps before they are needed and
-    // kept in registers.
-    constexpr int kStatAhead = 3;
-    const float LOG2E = 1.4426950408889634f;
-    float r_lt[kStatAhead][2], r_ls[kStatAhead][2], r_g[kStatAhead][2], r_kl[kStatAhead][2];
-    auto load_step = [&](int s, float (&lt)[2], float (&ls)[2], float (&gg)[2], float (&kv)[2]) {
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int row = (jq_begin + s) * C::BM + r * 32 + lane;
-        lt[r] = -INFINITY;
-        ls[r] = -INFINITY;
-        gg[r] = 0.f;
-        kv[r] = 0.f;
-        if (s < n_steps && row < seq.nq) {
-          const size_t o = (size_t)(seq.ob + row);
-          lt[r] = __ldg(args.lse_t + o);
-          ls[r] = __ldg(args.lse_s + o);
-          gg[r] = __ldg(args.g + o);
-          if (TEACHER) kv[r] = __ldg(args.kl + o);
-        }
-      }
-    };
-#pragma unroll
-    for (int k = 0; k < kStatAhead; ++k) load_step(k, r_lt[k], r_ls[k], r_g[k], r_kl[k]);
-    bool ok = true;
-    for (int s = 0; s < n_steps; ++s) {
-      if (lane == 0 && !mbar_wait(smem_u32(&bars->st_empty[s & 1]), ((s >> 1) & 1) ^ 1)) {
-        ok = false;
-        skl_fail_b(abort_flag);
-      }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      // Slot s&1: -LSE_T*log2e, -LSE_S*log2e, g*scale_G, E = KL + LSE_T - LSE_S
-      // (rows without keys: -inf, -inf, 0, 0).
-      float* sts = stats + (s & 1) * (4 * C::BM);
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const float lt = r_lt[0][r], ls = r_ls[0][r];
-        const bool live = lt != -INFINITY && ls != -INFINITY;
-        sts[r * 32 + lane] = live ? -lt * LOG2E : -INFINITY;
-        sts[C::BM + r * 32 + lane] = live ? -ls * LOG2E : -INFINITY;
-        sts[2 * C::BM + r * 32 + lane] = live ? r_g[0][r] * args.scale_G : 0.f;
-        sts[3 * C::BM + r * 32 + lane] = live ? r_kl[0][r] + (lt - ls) : 0.f;
-      }
-      mbar_arrive(smem_u32(&bars->st_full[s & 1]));
-#pragma unroll
-      for (int k = 0; k + 1 < kStatAhead; ++k)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          r_lt[k][r] = r_lt[k + 1][r];
-          r_ls[k][r] = r_ls[k + 1][r];
-          r_g[k][r] = r_g[k + 1][r];
-          r_kl[k][r] = r_kl[k + 1][r];
-        }
-      load_step(s + kStatAhead, r_lt[kStatAhead - 1], r_ls[kStatAhead - 1], r_g[kStatAhead - 1],
-                r_kl[kStatAhead - 1]);
-    }
-  } else if (warp == 11) {
-    // ------------------------------------------- dQ (and shared-K dK) reduce issuer
-    if (lane == 0) {
-      tma_prefetch_desc(&map_dq);
-      if (dk_rounds) tma_prefetch_desc(&map_dk);
-      for (int p = 0; p < n_steps + dk_rounds; ++p) {
-        if (!mbar_wait(smem_u32(&bars->stg_full[p & 1]), (p >> 1) & 1)) {
-          skl_fail_b(abort_flag);
-          break;
-        }
-        if (p < n_steps) {  // dQ part of step p: 64 query rows
-          const int i0 = seq.qr + (jq_begin + p) * C::BM;
-#pragma unroll
-          for (int db = 0; db < DG / 32; ++db)
-            tma_reduce_add_3d(&map_dq, sb + C::OFF_STG + db * (C::BM * 128), db * 32, i0, seq.zq);
-        } else {  // dK tile of this CTA, 64 key rows per round
-          const int r0 = seq.kr + k0 + (p - n_steps) * 64;
-#pragma unroll
-          for (int db = 0; db < DG / 32; ++db)
-            tma_reduce_add_3d(&map_dk, sb + C::OFF_STG + db * (C::BM * 128), db * 32, r0, bkg);
-        }
-        bulk_commit_group();
-        bulk_wait_group_read0();
-        mbar_arrive(smem_u32(&bars->stg_free[p & 1]));
-      }
-      bulk_wait_group0();
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------- MMA issuer
-    if (elect_one()) {
-      const uint32_t s_kt = sb + C::OFF_KT, s_ks = sb + C::OFF_KS;
-      bool ok = mbar_wait(smem_u32(&bars->k_full), 0);
-#if SKL_BWD_KTMEM
-      // The dS warps copy the K rows into tensor memory first.
-      if (ok) ok = mbar_wait(smem_u32(&bars->k_tmem), 0);
-      // S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T of step s into the single score buffer,
-      // A (the K rows) from tensor memory; the buffer is free once step s-1 has been read.
-      // Barriers stay per step parity (each warpgroup waits only on its own steps' phases).
-      auto issue_scores = [&](int s) -> bool {
-        const int st = s % C::NQST;
-        if (!mbar_wait(smem_u32(&bars->q_full[st]), (s / C::NQST) & 1)) return false;
-        if (s > 0 && !mbar_wait(smem_u32(&bars->s_free[(s - 1) & 1]), ((s - 1) >> 1) & 1))
-          return false;
-        tc_fence_after();
-        const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
-        const uint32_t d_t = tmem + C::TM_S, d_s = d_t + 64;
-#pragma unroll
-        for (int kk = 0; kk < DT / 16; ++kk) {
-          const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
-          umma_bf16_ts(d_t, tmem + C::TM_KT + kk * 8, sdesc_sw128(q_base + qa, 16, 1024),
-                       idesc_st, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < DS / 16; ++kk) {
-          const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
-          umma_bf16_ts(d_s, tmem + C::TM_KS + kk * 8,
-                       sdesc_sw128(q_base + C::QT_TILE + qa, 16, 1024), idesc_ss, kk > 0);
-        }
-        umma_commit(smem_u32(&bars->s_full[s & 1]));
-        return true;
-      };
-      if (ok && n_steps > 0) ok = issue_scores(0);
-      for (int p = 0; ok && p < n_steps; ++p) {
-        const int pb = p & 1, pst = p % C::NQST;
-        // Scores of step p+1 as soon as the warpgroup of step p has read its scores.
-        if (p + 1 < n_steps && !issue_scores(p + 1)) { ok = false; break; }
-        constexpr bool early = true;
-#else
-      // S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T of step s into TMEM buffer s&1.
-      auto issue_scores = [&](int s) -> bool {
-        const int st = s % C::NQST, b = s & 1;
-        if (!mbar_wait(smem_u32(&bars->q_full[st]), (s / C::NQST) & 1)) return false;
-        if (!mbar_wait(smem_u32(&bars->s_free[b]), ((s >> 1) & 1) ^ 1)) return false;
-        tc_fence_after();
-        const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
-        const uint32_t d_t = tmem + C::TM_S + b * 128, d_s = d_t + 64;
-#pragma unroll
-        for (int kk = 0; kk < DT / 16; ++kk) {
-          const uint32_t ka = (kk >> 2) * (C::BN * 128) + (kk & 3) * 32;
-          const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
-          umma_bf16_ss(d_t, sdesc_sw128(s_kt + ka, 16, 1024), sdesc_sw128(q_base + qa, 16, 1024),
-                       idesc_st, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < DS / 16; ++kk) {
-          const uint32_t ka = (kk >> 2) * (C::BN * 128) + (kk & 3) * 32;
-          const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
-          umma_bf16_ss(d_s, sdesc_sw128(s_ks + ka, 16, 1024),
-                       sdesc_sw128(q_base + C::QT_TILE + qa, 16, 1024), idesc_ss, kk > 0);
-        }
-        umma_commit(smem_u32(&bars->s_full[b]));
-        return true;
-      };
-      if (ok && n_steps > 0) ok = issue_scores(0);
-      if (ok && n_steps > 1) ok = issue_scores(1);
-      for (int p = 0; ok && p < n_steps; ++p) {
-        const int pb = p & 1, pst = p % C::NQST;
-        // The score tiles of step p+2 reuse buffer pb, which the warpgroup frees as soon as
-        // it has read step p's scores; issue them ahead of dK/dQ(p) when their query tile
-        // has landed, so the warpgroup finds them ready when it finishes step p.
-        bool early = false;
-        if (p + 2 < n_steps && mbar_try_wait(smem_u32(&bars->q_full[(p + 2) % C::NQST]),
-                                             ((p + 2) / C::NQST) & 1)) {
-          if (!issue_scores(p + 2)) { ok = false; break; }
-          early = true;
-        }
+  if (warp >= kBwdDsWarps) {
+#if SKL_BWD_SPLIT
+    regs_dec<SKL_BWD_RC>();
 #endif
-        if (!mbar_wait(smem_u32(&bars->ds_full[pb]), (p >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t s_ds = sb + C::OFF_DS + pb * C::DS_TILE;
-        // Q tile of the differentiated side (student Q_S, or teacher Q_T).
-        const uint32_t s_qg = sb + C::OFF_Q + pst * C::Q_STAGE + (TEACHER ? 0 : C::QT_TILE);
-        // dK += dS^T Q : A = dS^T [keys][queries] K-major, B = Q [queries][d] MN-major.
-#pragma unroll
-        for (int kk = 0; kk < C::BM / 16; ++kk) {
-          umma_bf16_ss(tmem + C::TM_DK, sdesc_sw128(s_ds + kk * 32, 16, 1024),
-                       sdesc_sw128(s_qg + kk * 2048, C::BM * 128, 1024), idesc_dk,
-                       (p > 0 || kk > 0) ? 1u : 0u);
+    if (warp == kBwdTmaWarp) {
+      // ----------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        const uint64_t keep = l2_policy_evict_last();
+        int issued = 0;
+        tma_prefetch_desc(&map_qt);
+        tma_prefetch_desc(&map_kt);
+        tma_prefetch_desc(&map_qs);
+        tma_prefetch_desc(&map_ks);
+        const uint32_t kb = smem_u32(&bars->k_full);
+        mbar_arrive_expect_tx(kb, C::KT_TILE + C::KS_TILE);
+        for (int blk = 0; blk < DT / 64; ++blk)
+          tma_load_3d(sb + C::OFF_KT + blk * (C::BN * 128), &map_kt, kb, blk * 64, seq.kr + k0,
+                      seq.zkt, keep);
+        for (int blk = 0; blk < DS / 64; ++blk)
+          tma_load_3d(sb + C::OFF_KS + blk * (C::BN * 128), &map_ks, kb, blk * 64, seq.kr + k0,
+                      seq.zks, keep);
+        for (int s = 0; s < n_steps; ++s) {
+          const int st = s % C::NQST;
+          const int i0 = seq.qr + (jq_begin + s) * C::BM;
+          if (!mbar_wait(smem_u32(&bars->q_empty[st]), ((s / C::NQST) & 1) ^ 1)) {
+            skl_fail_b(abort_flag);
+            break;
+          }
+          const uint32_t fb = smem_u32(&bars->q_full[st]);
+          const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
+          mbar_arrive_expect_tx(fb, C::Q_STAGE);
+          for (int blk = 0; blk < DT / 64; ++blk)
+            tma_load_3d(q_base + blk * (C::BM * 128), &map_qt, fb, blk * 64, i0, seq.zq, keep);
+          for (int blk = 0; blk < DS / 64; ++blk)
+            tma_load_3d(q_base + C::QT_TILE + blk * (C::BM * 128), &map_qs, fb, blk * 64, i0,
+                        seq.zq, keep);
+          issued = s + 1;
         }
-        umma_commit(smem_u32(&bars->q_empty[pst]));
-        if (!mbar_wait(smem_u32(&bars->dq_free[pb]), ((p >> 1) & 1) ^ 1)) { ok = false; break; }
-        tc_fence_after();
-        // dQ^T = K^T dS^T : A = K [keys][d] MN-major, B = dS^T [keys][queries] MN-major.
-        const uint32_t s_kg = TEACHER ? s_kt : s_ks;
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          umma_bf16_ss(tmem + C::TM_DQ + pb * C::BM,
-                       sdesc_sw128(s_kg + kk * 2048, C::BN * 128, 1024),
-                       sdesc_sw128(s_ds + kk * 2048, C::BN * 128, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+        if (*abort_flag) {
+          // Let every copy this thread started land before the CTA can exit.
+          mbar_wait(smem_u32(&bars->k_full), 0);
+          for (int s = max(0, issued - C::NQST); s < issued; ++s)
+            mbar_wait(smem_u32(&bars->q_full[s % C::NQST]), (s / C::NQST) & 1);
         }
-        umma_commit(smem_u32(&bars->ds_empty[pb]));
-        umma_commit(smem_u32(&bars->dq_full[pb]));
-        if (!early && p + 2 < n_steps && !issue_scores(p + 2)) { ok = false; break; }
       }
-      if (!ok) skl_fail_b(abort_flag);
-      umma_commit(smem_u32(&bars->dk_full));
-      umma_commit(smem_u32(&bars->drain));
-      if (!mbar_wait(smem_u32(&bars->drain), 0)) skl_fail_b(abort_flag);
+    } else if (warp == kBwdStatWarp) {
+      // ------------------------------------------------ row-statistics loader
+      // Each lane owns query rows lane and lane+32 of every step. Raw LSE_T, LSE_S, g (and
+      // KL for the teacher gradient) are loaded kStatAhead steps before they are needed and
+      // kept in registers.
+      constexpr int kStatAhead = 3;
+      const float LOG2E = 1.4426950408889634f;
+      float r_lt[kStatAhead][2], r_ls[kStatAhead][2], r_g[kStatAhead][2], r_kl[kStatAhead][2];
+      auto load_step = [&](int s, float (&lt)[2], float (&ls)[2], float (&gg)[2], float (&kv)[2]) {
+    #pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int row = (jq_begin + s) * C::BM + r * 32 + lane;
+          lt[r] = -INFINITY;
+          ls[r] = -INFINITY;
+          gg[r] = 0.f;
+          kv[r] = 0.f;
+          if (s < n_steps && row < seq.nq) {
+            const size_t o = (size_t)(seq.ob + row);
+            lt[r] = __ldg(args.lse_t + o);
+            ls[r] = __ldg(args.lse_s + o);
+            gg[r] = __ldg(args.g + o);
+            if (TEACHER) kv[r] = __ldg(args.kl + o);
+          }
+        }
+      };
+    #pragma unroll
+      for (int k = 0; k < kStatAhead; ++k) load_step(k, r_lt[k], r_ls[k], r_g[k], r_kl[k]);
+      bool ok = true;
+      for (int s = 0; s < n_steps; ++s) {
+        if (lane == 0 && !mbar_wait(smem_u32(&bars->st_empty[s & 1]), ((s >> 1) & 1) ^ 1)) {
+          ok = false;
+          skl_fail_b(abort_flag);
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        // Slot s&1: -LSE_T*log2e, -LSE_S*log2e, g*scale_G, E = KL + LSE_T - LSE_S
+        // (rows without keys: -inf, -inf, 0, 0).
+        float* sts = stats + (s & 1) * (4 * C::BM);
+    #pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float lt = r_lt[0][r], ls = r_ls[0][r];
+          const bool live = lt != -INFINITY && ls != -INFINITY;
+          sts[r * 32 + lane] = live ? -lt * LOG2E : -INFINITY;
+          sts[C::BM + r * 32 + lane] = live ? -ls * LOG2E : -INFINITY;
+          sts[2 * C::BM + r * 32 + lane] = live ? r_g[0][r] * args.scale_G : 0.f;
+          sts[3 * C::BM + r * 32 + lane] = live ? r_kl[0][r] + (lt - ls) : 0.f;
+        }
+        mbar_arrive(smem_u32(&bars->st_full[s & 1]));
+    #pragma unroll
+        for (int k = 0; k + 1 < kStatAhead; ++k)
+    #pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            r_lt[k][r] = r_lt[k + 1][r];
+            r_ls[k][r] = r_ls[k + 1][r];
+            r_g[k][r] = r_g[k + 1][r];
+            r_kl[k][r] = r_kl[k + 1][r];
+          }
+        load_step(s + kStatAhead, r_lt[kStatAhead - 1], r_ls[kStatAhead - 1], r_g[kStatAhead - 1],
+                  r_kl[kStatAhead - 1]);
+      }
+    } else if (warp == kBwdRedWarp) {
+      // ------------------------------------------- dQ (and shared-K dK) reduce issuer
+      if (lane == 0) {
+        tma_prefetch_desc(&map_dq);
+        if (dk_rounds) tma_prefetch_desc(&map_dk);
+        for (int p = 0; p < n_steps + dk_rounds; ++p) {
+          if (!mbar_wait(smem_u32(&bars->stg_full[p & 1]), (p >> 1) & 1)) {
+            skl_fail_b(abort_flag);
+            break;
+          }
+          if (p < n_steps) {  // dQ part of step p: 64 query rows
+            const int i0 = seq.qr + (jq_begin + p) * C::BM;
+    #pragma unroll
+            for (int db = 0; db < DG / 32; ++db)
+              tma_reduce_add_3d(&map_dq, sb + C::OFF_STG + db * (C::BM * 128), db * 32, i0, seq.zq);
+          } else {  // dK tile of this CTA, 64 key rows per round
+            const int r0 = seq.kr + k0 + (p - n_steps) * 64;
+    #pragma unroll
+            for (int db = 0; db < DG / 32; ++db)
+              tma_reduce_add_3d(&map_dk, sb + C::OFF_STG + db * (C::BM * 128), db * 32, r0, bkg);
+          }
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(smem_u32(&bars->stg_free[p & 1]));
+        }
+        bulk_wait_group0();
+      }
+    } else if (warp == kBwdMmaWarp) {
+      // ------------------------------------------------------------- MMA issuer
+      if (elect_one()) {
+        const uint32_t s_kt = sb + C::OFF_KT, s_ks = sb + C::OFF_KS;
+        bool ok = mbar_wait(smem_u32(&bars->k_full), 0);
+    #if SKL_BWD_KTMEM
+        // The dS warps copy the K rows into tensor memory first.
+        if (ok) ok = mbar_wait(smem_u32(&bars->k_tmem), 0);
+        // S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T of step s into the single score buffer,
+        // A (the K rows) from tensor memory; the buffer is free once step s-1 has been read.
+        // Barriers stay per step parity (each warpgroup waits only on its own steps' phases).
+        auto issue_scores = [&](int s) -> bool {
+          const int st = s % C::NQST;
+          if (!mbar_wait(smem_u32(&bars->q_full[st]), (s / C::NQST) & 1)) return false;
+          if (s > 0 && !mbar_wait(smem_u32(&bars->s_free[(s - 1) & 1]), ((s - 1) >> 1) & 1))
+            return false;
+          tc_fence_after();
+          const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
+          const uint32_t d_t = tmem + C::TM_S, d_s = d_t + 64;
+    #pragma unroll
+          for (int kk = 0; kk < DT / 16; ++kk) {
+            const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
+            umma_bf16_ts(d_t, tmem + C::TM_KT + kk * 8, sdesc_sw128(q_base + qa, 16, 1024),
+                         idesc_st, kk > 0);
+          }
+    #pragma unroll
+          for (int kk = 0; kk < DS / 16; ++kk) {
+            const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
+            umma_bf16_ts(d_s, tmem + C::TM_KS + kk * 8,
+                         sdesc_sw128(q_base + C::QT_TILE + qa, 16, 1024), idesc_ss, kk > 0);
+          }
+          umma_commit(smem_u32(&bars->s_full[s & 1]));
+          return true;
+        };
+        if (ok && n_steps > 0) ok = issue_scores(0);
+        for (int p = 0; ok && p < n_steps; ++p) {
+          const int pb = p & 1, pst = p % C::NQST;
+          // Scores of step p+1 as soon as the warpgroup of step p has read its scores.
+          if (p + 1 < n_steps && !issue_scores(p + 1)) { ok = false; break; }
+          constexpr bool early = true;
+    #else
+        // S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T of step s into TMEM buffer s&1.
+        auto issue_scores = [&](int s) -> bool {
+          const int st = s % C::NQST, b = s & 1;
+          if (!mbar_wait(smem_u32(&bars->q_full[st]), (s / C::NQST) & 1)) return false;
+          if (!mbar_wait(smem_u32(&bars->s_free[b]), ((s >> 1) & 1) ^ 1)) return false;
+          tc_fence_after();
+          const uint32_t q_base = sb + C::OFF_Q + st * C::Q_STAGE;
+          const uint32_t d_t = tmem + C::TM_S + b * 128, d_s = d_t + 64;
+    #pragma unroll
+          for (int kk = 0; kk < DT / 16; ++kk) {
+            const uint32_t ka = (kk >> 2) * (C::BN * 128) + (kk & 3) * 32;
+            const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
+            umma_bf16_ss(d_t, sdesc_sw128(s_kt + ka, 16, 1024), sdesc_sw128(q_base + qa, 16, 1024),
+                         idesc_st, kk > 0);
+          }
+    #pragma unroll
+          for (int kk = 0; kk < DS / 16; ++kk) {
+            const uint32_t ka = (kk >> 2) * (C::BN * 128) + (kk & 3) * 32;
+            const uint32_t qa = (kk >> 2) * (C::BM * 128) + (kk & 3) * 32;
+            umma_bf16_ss(d_s, sdesc_sw128(s_ks + ka, 16, 1024),
+                         sdesc_sw128(q_base + C::QT_TILE + qa, 16, 1024), idesc_ss, kk > 0);
+          }
+          umma_commit(smem_u32(&bars->s_full[b]));
+          return true;
+        };
+        if (ok && n_steps > 0) ok = issue_scores(0);
+        if (ok && n_steps > 1) ok = issue_scores(1);
+        for (int p = 0; ok && p < n_steps; ++p) {
+          const int pb = p & 1, pst = p % C::NQST;
+          // The score tiles of step p+2 reuse buffer pb, which the warpgroup frees as soon as
+          // it has read step p's scores; issue them ahead of dK/dQ(p) when their query tile
+          // has landed, so the warpgroup finds them ready when it finishes step p.
+          bool early = false;
+          if (p + 2 < n_steps && mbar_try_wait(smem_u32(&bars->q_full[(p + 2) % C::NQST]),
+                                               ((p + 2) / C::NQST) & 1)) {
+            if (!issue_scores(p + 2)) { ok = false; break; }
+            early = true;
+          }
+    #endif
+          if (!mbar_wait(smem_u32(&bars->ds_full[pb]), (p >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t s_ds = sb + C::OFF_DS + pb * C::DS_TILE;
+          // Q tile of the differentiated side (student Q_S, or teacher Q_T).
+          const uint32_t s_qg = sb + C::OFF_Q + pst * C::Q_STAGE + (TEACHER ? 0 : C::QT_TILE);
+          // dK += dS^T Q : A = dS^T [keys][queries] K-major, B = Q [queries][d] MN-major.
+    #pragma unroll
+          for (int kk = 0; kk < C::BM / 16; ++kk) {
+            umma_bf16_ss(tmem + C::TM_DK, sdesc_sw128(s_ds + kk * 32, 16, 1024),
+                         sdesc_sw128(s_qg + kk * 2048, C::BM * 128, 1024), idesc_dk,
+                         (p > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&bars->q_empty[pst]));
+          if (!mbar_wait(smem_u32(&bars->dq_free[pb]), ((p >> 1) & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          // dQ^T = K^T dS^T : A = K [keys][d] MN-major, B = dS^T [keys][queries] MN-major.
+          const uint32_t s_kg = TEACHER ? s_kt : s_ks;
+    #pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk) {
+            umma_bf16_ss(tmem + C::TM_DQ + pb * C::BM,
+                         sdesc_sw128(s_kg + kk * 2048, C::BN * 128, 1024),
+                         sdesc_sw128(s_ds + kk * 2048, C::BN * 128, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&bars->ds_empty[pb]));
+          umma_commit(smem_u32(&bars->dq_full[pb]));
+          if (!early && p + 2 < n_steps && !issue_scores(p + 2)) { ok = false; break; }
+        }
+        if (!ok) skl_fail_b(abort_flag);
+        umma_commit(smem_u32(&bars->dk_full));
+        umma_commit(smem_u32(&bars->drain));
+        if (!mbar_wait(smem_u32(&bars->drain), 0)) skl_fail_b(abort_flag);
+      }
     }
   } else {
     // ------------------------------------------------- dS / reduction warpgroups
-    const int wg = warp >> 2;            // steps s with s&1 == wg
+#if SKL_BWD_SPLIT
+    regs_inc<SKL_BWD_RS>();
+#endif
+    const int wg = (warp >> 2) & 1;      // steps s with s&1 == wg
+    const int hh = warp >> 3;            // query-column half (split), else 0
+    constexpr int NC = C::BM / kBwdHalves;  // query columns of a step handled by this warp
+    const int c0 = hh * NC;
     const int quarter = warp & 3;
     const int kl = quarter * 32 + lane;  // key row within the tile = TMEM lane
     const int key = k0 + kl;
@@ -470,9 +505,13 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     auto drain_dq = [&](int p) -> bool {
       if (!mbar_wait(smem_u32(&bars->dq_full[wg]), (p >> 1) & 1)) return false;
       tc_fence_after();
-      uint32_t v[64];
-      tmem_ld_2x32_wait(tmem + lane_off + C::TM_DQ + wg * C::BM,
-                        tmem + lane_off + C::TM_DQ + wg * C::BM + 32, v);
+      uint32_t v[NC];  // this warp's query columns c0 .. c0+NC-1 of the dQ^T part
+      if constexpr (NC == 64) {
+        tmem_ld_2x32_wait(tmem + lane_off + C::TM_DQ + wg * C::BM,
+                          tmem + lane_off + C::TM_DQ + wg * C::BM + 32, v);
+      } else {
+        tmem_ld_32_wait(tmem + lane_off + C::TM_DQ + wg * C::BM + c0, v);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->dq_free[wg]));
@@ -485,8 +524,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         const uint32_t col = sb + C::OFF_STG + (dq_d >> 5) * (C::BM * 128) + ((dq_d & 3) << 2);
         const uint32_t chunk = (dq_d & 31) >> 2;
 #pragma unroll
-        for (int c = 0; c < C::BM; ++c)
-          st_shared_f32(col + c * 128 + ((chunk ^ (c & 7)) << 4), __uint_as_float(v[c]));
+        for (int i = 0; i < NC; ++i) {
+          const int c = c0 + i;
+          st_shared_f32(col + c * 128 + ((chunk ^ (c & 7)) << 4), __uint_as_float(v[i]));
+        }
       }
       fence_async_smem();
       __syncwarp();
@@ -499,7 +540,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     {
       // K rows into tensor memory (A operand of the score MMAs): warpgroup 0 copies K_T,
       // warpgroup 1 copies K_S, one key row per thread.
-      if (mbar_wait(smem_u32(&bars->k_full), 0)) {
+      if (hh > 0) {
+        // the first column half copies
+      } else if (mbar_wait(smem_u32(&bars->k_full), 0)) {
         if (wg == 0)
           row_to_tmem<DT>(sb + C::OFF_KT + kl * 128, tmem + lane_off + C::TM_KT, kl);
         else
@@ -524,11 +567,17 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         break;
       }
       tc_fence_after();
-      uint32_t vt[64], vs[64];  // raw teacher / student scores of this key, 64 query columns
-      tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + sbuf * 128,
-                        tmem + lane_off + C::TM_S + sbuf * 128 + 32, vt);
-      tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + sbuf * 128 + 64,
-                        tmem + lane_off + C::TM_S + sbuf * 128 + 96, vs);
+      // Raw teacher / student scores of this key for this warp's query columns.
+      uint32_t vt[NC], vs[NC];
+      if constexpr (NC == 64) {
+        tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + sbuf * 128,
+                          tmem + lane_off + C::TM_S + sbuf * 128 + 32, vt);
+        tmem_ld_2x32_wait(tmem + lane_off + C::TM_S + sbuf * 128 + 64,
+                          tmem + lane_off + C::TM_S + sbuf * 128 + 96, vs);
+      } else {
+        tmem_ld_32_wait(tmem + lane_off + C::TM_S + sbuf * 128 + c0, vt);
+        tmem_ld_32_wait(tmem + lane_off + C::TM_S + sbuf * 128 + 64 + c0, vs);
+      }
       // The score buffer can take step s+2 as soon as every lane has read it.
       tc_fence_before();
       __syncwarp();
@@ -546,7 +595,8 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       const bool need_mask = causal_mask || (k0 + C::BN > seq.nk);
       const int cmin = key >= seq.nk ? C::BM : (causal_mask ? (key - seq.off - i0) : -1);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {  // 8 query columns = one 16-byte chunk of dS^T
+      for (int uu = 0; uu < NC / 8; ++uu) {  // 8 query columns = one 16-byte chunk of dS^T
+        const int u = c0 / 8 + uu;
         const float4 nlt0 = *reinterpret_cast<const float4*>(sts + u * 8);
         const float4 nlt1 = *reinterpret_cast<const float4*>(sts + u * 8 + 4);
         const float4 nls0 = *reinterpret_cast<const float4*>(sts + C::BM + u * 8);
@@ -566,17 +616,18 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         float d[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int c = u * 8 + e;
-          const float pT = ex2_approx(fmaf(__uint_as_float(vt[c]), cT, nlt[e]));
+          const int c = u * 8 + e;   // query column within the step
+          const int ci = uu * 8 + e;  // its register index
+          const float pT = ex2_approx(fmaf(__uint_as_float(vt[ci]), cT, nlt[e]));
           float ds;
           if (TEACHER) {
             // g*scale_T * P_T * ((s_T - s_S) - E), scores in natural units; both products
             // rounded alike so that identical teacher and student scores cancel exactly.
-            const float w = __fsub_rn(__fmul_rn(__uint_as_float(vt[c]), aT),
-                                      __fmul_rn(__uint_as_float(vs[c]), aS)) - ee[e];
+            const float w = __fsub_rn(__fmul_rn(__uint_as_float(vt[ci]), aT),
+                                      __fmul_rn(__uint_as_float(vs[ci]), aS)) - ee[e];
             ds = gg[e] * pT * w;
           } else {
-            const float pS = ex2_approx(fmaf(__uint_as_float(vs[c]), cS, nls[e]));
+            const float pS = ex2_approx(fmaf(__uint_as_float(vs[ci]), cS, nls[e]));
             ds = gg[e] * (pS - pT);
           }
           if (need_mask && c < cmin) ds = 0.f;
@@ -598,7 +649,8 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     // dK rows of this key tile (TMEM lanes = keys); zero when no query sees them. With a
     // K head shared by several query heads (dk_reduce) the tile is added into the zeroed
     // dk through the staging tile in two 64-row rounds, continuing the staging sequence.
-    constexpr int DKH = DG / 2;  // dK columns handled by this warpgroup
+    constexpr int DKH = DG / (2 * kBwdHalves);  // dK columns handled by this warp
+    const int col0 = (hh * 2 + wg) * DKH;
     uint32_t v[DKH];
 #pragma unroll
     for (int c = 0; c < DKH; ++c) v[c] = 0u;
@@ -608,16 +660,18 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       } else {
         tc_fence_after();
         if constexpr (DKH == 64) {
-          tmem_ld_2x32_wait(tmem + lane_off + C::TM_DK + wg * DKH,
-                            tmem + lane_off + C::TM_DK + wg * DKH + 32, v);
+          tmem_ld_2x32_wait(tmem + lane_off + C::TM_DK + col0,
+                            tmem + lane_off + C::TM_DK + col0 + 32, v);
+        } else if constexpr (DKH == 32) {
+          tmem_ld_32_wait(tmem + lane_off + C::TM_DK + col0, v);
         } else {
-          tmem_ld_32_wait(tmem + lane_off + C::TM_DK + wg * DKH, v);
+          tmem_ld_16_wait(tmem + lane_off + C::TM_DK + col0, v);
         }
       }
     }
     if (ok && !dk_rounds && key < seq.nk) {
       float4* dst = reinterpret_cast<float4*>(args.dk + bkg * args.dk_hs +
-                                              (long long)(seq.kr + key) * args.dk_rs + wg * DKH);
+                                              (long long)(seq.kr + key) * args.dk_rs + col0);
 #pragma unroll
       for (int c = 0; c < DKH; c += 4)
         dst[c / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
@@ -626,7 +680,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     if (dk_rounds) {
       // Every dS warp reaches this barrier (dk_rounds is uniform over the CTA), after its
       // last dQ drain, so each staging wait below is at most one phase ahead of its barrier.
-      named_bar_sync(1, 256);
+      named_bar_sync(1, 32 * kBwdDsWarps);
       ok = __all_sync(0xffffffffu, ok);
       for (int r = 0; ok && r < 2; ++r) {
         const int p = n_steps + r;
@@ -637,7 +691,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           const int row = kl - 64 * r;
 #pragma unroll
           for (int c = 0; c < DKH; c += 4) {
-            const int dcol = wg * DKH + c;
+            const int dcol = col0 + c;
             const uint32_t addr = sb + C::OFF_STG + (dcol >> 5) * (C::BM * 128) + row * 128 +
                                   ((((dcol & 31) >> 2) ^ (row & 7)) << 4);
             st_shared_v4(addr, v[c], v[c + 1], v[c + 2], v[c + 3]);
@@ -653,7 +707,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kBwdMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -18,9 +18,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -47,61 +45,73 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """SM clock, power and clock-event reasons of this process's GPU, sampled through NVML
+    every few milliseconds from a background thread while the timed region runs. The GPU
+    is found by its PCI bus id (NVML does not follow CUDA_VISIBLE_DEVICES); read-only."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    def __init__(self, cuda_index: int, period_s: float = 0.005):
+        self.cuda_index = cuda_index
+        self.period = period_s
+        self.samples = []
+        self.error = None
+        self.thread = None
+        self.stop_flag = False
+
+    def _handle(self, nv):
+        prop = torch.cuda.get_device_properties(self.cuda_index)
+        bus = f"{prop.pci_domain_id:08X}:{prop.pci_bus_id:02X}:{prop.pci_device_id:02X}.0"
+        return nv.nvmlDeviceGetHandleByPciBusId(bus.encode()), bus
+
+    def _run(self, nv, h):
+        while not self.stop_flag:
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except Exception as e:  # keep whatever was sampled
+                self.error = repr(e)
+                return
+            time.sleep(self.period)
 
     def start(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
-        time.sleep(0.3)
+            import pynvml as nv
+            nv.nvmlInit()
+            h, self.bus = self._handle(nv)
+            self.nv = nv
+        except Exception as e:
+            self.error = f"NVML unavailable: {e!r}"
+            return
+        self.thread = threading.Thread(target=self._run, args=(self.nv, h), daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.samples and self.error is None and time.time() - t0 < 2.0:
+            time.sleep(0.001)
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
+        if self.thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "no sampler"]}
+        self.stop_flag = True
+        self.thread.join(timeout=2.0)
+        rows = list(self.samples)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
-        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "power_w_max": max(pw) if pw else None,
-                "samples": len(rows), "reasons": reasons}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "no samples"]}
+        masks = {name: getattr(self.nv, attr, 0) for name, attr in self.REASONS}
+        reasons = sorted({name for r in rows for name, m in masks.items() if m and (r[3] & m)})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_median": statistics.median(r[2] for r in rows),
+                "power_w_max": max(r[2] for r in rows),
+                "samples": len(rows), "gpu_pci_bus_id": self.bus, "source": "NVML",
+                "reasons": reasons}
 
 
 def dist_setup():
@@ -461,37 +471,53 @@ def run_context_parallel(skl, w, d, dev, stream, steps, world, shards=4):
 
 
 def run_e2e(skl, w, x, dev, stream, steps, world):
-    """Same metric through the public API from pinned host buffers: every step copies
-    the inputs host->device, runs forward + backward, and reads the KL rows back."""
+    """Same metric through the public API from pinned host buffers: every step copies its
+    inputs host->device, runs forward + backward, and reads its KL rows back to the host.
+    The copies run on a second stream into one of two device input buffers, so step k's
+    host->device copy overlaps step k-1's kernels (a double-buffered input pipeline)."""
     host = {k: v.pin_memory() for k, v in x.items()}
-    d = {k: torch.empty_like(v, device=dev) for k, v in x.items()}
-    kl_h = torch.empty(w.B, w.H, w.N_Q, dtype=torch.float32).pin_memory()
+    bufs = [{k: torch.empty_like(v, device=dev) for k, v in x.items()} for _ in range(2)]
+    kl_h = [torch.empty(w.B, w.H, w.N_Q, dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = kl_h.numel() * 4
+    d2h = kl_h[0].numel() * 4
+    copy_stream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event() for _ in range(2)]
+    freed = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        for k in d:
-            d[k].copy_(host[k], non_blocking=True)
+    def one(k):
+        b = k & 1
+        d = bufs[b]
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(freed[b])  # step k-2's kernels are done with buffer b
+            for name in d:
+                d[name].copy_(host[name], non_blocking=True)
+            copied[b].record(copy_stream)
+        stream.wait_event(copied[b])
         kl, lt, ls = skl.streamkl_fwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T,
-                                      w.scale_S, w.causal)
+                                      w.scale_S, w.causal, stream=stream)
         skl.streamkl_bwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S,
-                         w.causal, lt, ls, d["g"])
-        kl_h.copy_(kl, non_blocking=True)
+                         w.causal, lt, ls, d["g"], stream=stream)
+        freed[b].record(stream)
+        kl_h[b].copy_(kl, non_blocking=True)
 
-    for _ in range(2):
-        one()
+    for b in range(2):
+        freed[b].record(stream)
+    for k in range(2):
+        one(k)
     torch.cuda.synchronize()
     barrier(world)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    copy_stream.wait_event(a)  # the first timed copy starts inside the timed region
+    for k in range(steps):
+        one(k)
+    e.record(stream)
     torch.cuda.synchronize()
-    ms = max_over_ranks(a.elapsed_time(b), world)
+    ms = max_over_ranks(a.elapsed_time(e), world)
     value = world * (flops_fwd(w) + flops_bwd(w)) * steps / (ms * 1e-3) / 1e12
     return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps}
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps,
+            "pipeline": "host->device copies on a second stream, double-buffered"}
 
 
 def load_traffic(workload: str, which: str):
