@@ -66,14 +66,14 @@ struct BwdArgs {
 // where the score MMAs read them as their A operand instead of re-reading them from
 // shared memory every step; the score tile is then single-buffered to make room.
 #ifndef SKL_BWD_KTMEM
-#define SKL_BWD_KTMEM 0
+#define SKL_BWD_KTMEM 1
 #endif
 
 // Warp layout. Default (SKL_BWD_SPLIT): 16 dS warps; warp w takes the steps of parity
 // (w >> 2) & 1, query columns 32 (w >> 3) .. +31 of each step and key rows
 // 32 (w & 3) .. +31 (its TMEM lane quarter). SKL_BWD_SPLIT = 0: 8 dS warps, all 64 columns.
 #ifndef SKL_BWD_SPLIT
-#define SKL_BWD_SPLIT 0
+#define SKL_BWD_SPLIT 1
 #endif
 constexpr int kBwdHalves = SKL_BWD_SPLIT ? 2 : 1;      // query-column halves per step
 constexpr int kBwdDsWarps = 8 * kBwdHalves;            // warps 0 .. kBwdDsWarps-1
@@ -584,9 +584,6 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[wg]));
       if (!mbar_wait(smem_u32(&bars->st_full[s & 1]), (s >> 1) & 1)) { ok = false; break; }
       const float* sts = stats + (s & 1) * (4 * C::BM);
-      // The dS buffer is free once the dK/dQ MMAs of step s-2 have read it (they were
-      // issued before this step's scores, so this wait normally returns at once).
-      if (!mbar_wait(smem_u32(&bars->ds_empty[wg]), ((s >> 1) & 1) ^ 1)) { ok = false; break; }
 
       // Query column c is allowed for this key iff i0 + c >= key - off; keys past the end
       // of the sequence (the next sequence's keys in the packed layout, zero fill in the
@@ -594,6 +591,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       const bool causal_mask = args.causal && (i0 + seq.off < k0 + C::BN - 1);
       const bool need_mask = causal_mask || (k0 + C::BN > seq.nk);
       const int cmin = key >= seq.nk ? C::BM : (causal_mask ? (key - seq.off - i0) : -1);
+      // dS of this step into registers (bf16 pairs) first; it is stored once the dK/dQ MMAs
+      // of step s-2 have read the dS buffer, so this arithmetic overlaps those MMAs.
+      uint32_t pk[NC / 8][4];
 #pragma unroll
       for (int uu = 0; uu < NC / 8; ++uu) {  // 8 query columns = one 16-byte chunk of dS^T
         const int u = c0 / 8 + uu;
@@ -633,11 +633,21 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           if (need_mask && c < cmin) ds = 0.f;
           d[e] = ds;
         }
-        st_shared_v4(s_ds_row + ((u ^ (kl & 7)) << 4), pack_bf16x2(d[0], d[1]),
-                     pack_bf16x2(d[2], d[3]), pack_bf16x2(d[4], d[5]), pack_bf16x2(d[6], d[7]));
+        pk[uu][0] = pack_bf16x2(d[0], d[1]);
+        pk[uu][1] = pack_bf16x2(d[2], d[3]);
+        pk[uu][2] = pack_bf16x2(d[4], d[5]);
+        pk[uu][3] = pack_bf16x2(d[6], d[7]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->st_empty[s & 1]));
+      // The dS buffer is free once the dK/dQ MMAs of step s-2 have read it.
+      if (!mbar_wait(smem_u32(&bars->ds_empty[wg]), ((s >> 1) & 1) ^ 1)) { ok = false; break; }
+#pragma unroll
+      for (int uu = 0; uu < NC / 8; ++uu) {
+        const int u = c0 / 8 + uu;
+        st_shared_v4(s_ds_row + ((u ^ (kl & 7)) << 4), pk[uu][0], pk[uu][1], pk[uu][2],
+                     pk[uu][3]);
+      }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->ds_full[wg]));
