@@ -182,7 +182,8 @@ def run_reference(args, world, rank):
     w = WORKLOADS[args.workload]
     if rank != 0:
         return
-    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    # The whole run (warm-up and timed steps) spends about args.ref_seconds on the host.
+    per_step = max(0.5, args.ref_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         cpu_baseline(w, budget_s=min(per_step, 3.0), seed=11)
     vals, secs = [], 0.0
@@ -220,7 +221,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="host time of the cpu_baseline leg of this arm")
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="total host time of the --impl reference arm")
     args = ap.parse_args()
 
     if args.impl == "reference":
