@@ -93,6 +93,15 @@ static_assert(!SKL_BWD_SPLIT || kBwdDsWarps * SKL_BWD_RS + 4 * SKL_BWD_RC <=
                                     (kBwdDsWarps + 4) * ((65536 / kBwdThreads) & ~7),
               "register split exceeds the launch's register pool");
 
+// SKL_BWD_NSTG = 2: two fp32 staging tiles for the dQ reduce-adds, one per step parity (each
+// dS warpgroup drains into its own tile while the previous reduce is still reading the
+// other). The second tile is the shared K tile of the side that is not differentiated: with
+// SKL_BWD_KTMEM it is only read by the copy into tensor memory, which completes before the
+// first score MMA and so before any drain. Used where that tile is large enough.
+#ifndef SKL_BWD_NSTG
+#define SKL_BWD_NSTG 2
+#endif
+
 // TEACHER = false: gradients of the student (dQ_S, dK_S), d_G = d_S.
 // TEACHER = true: gradients of a trainable teacher (dQ_T, dK_T), d_G = d_T.
 template <int DT, int DS, bool TEACHER = false>
@@ -116,6 +125,15 @@ struct BwdCfg {
   static constexpr int STG_TILE = BM * DG * 4;             // fp32 dQ staging tile
   static constexpr int OFF_STG = OFF_DS + 2 * DS_TILE;
   static constexpr int OFF_ST = OFF_STG + STG_TILE;        // NSTS statistics slots
+  // K tile of the side that is not differentiated (second staging tile, see SKL_BWD_NSTG).
+  static constexpr int OFF_KX = TEACHER ? OFF_KS : OFF_KT;
+  static constexpr int KX_TILE = TEACHER ? KS_TILE : KT_TILE;
+  static constexpr int NSTG =
+      (SKL_BWD_NSTG == 2 && SKL_BWD_KTMEM && KX_TILE >= STG_TILE) ? 2 : 1;  // staging tiles
+  // Staging tile of use p (dQ part of step p, or dK round p - n_steps).
+  static __device__ __forceinline__ uint32_t stg_off(int p) {
+    return (NSTG == 2 && (p & 1)) ? OFF_KX : OFF_STG;
+  }
   static constexpr int OFF_BAR = OFF_ST + NSTS * STATS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES;  // the dynamic base is 1024-byte aligned
@@ -345,25 +363,38 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       if (lane == 0) {
         tma_prefetch_desc(&map_dq);
         if (dk_rounds) tma_prefetch_desc(&map_dk);
+        int issued = 0;
         for (int p = 0; p < n_steps + dk_rounds; ++p) {
           if (!mbar_wait(smem_u32(&bars->stg_full[p & 1]), (p >> 1) & 1)) {
             skl_fail_b(abort_flag);
             break;
           }
+          const uint32_t src = sb + C::stg_off(p);
           if (p < n_steps) {  // dQ part of step p: 64 query rows
             const int i0 = seq.qr + (jq_begin + p) * C::BM;
     #pragma unroll
             for (int db = 0; db < DG / 32; ++db)
-              tma_reduce_add_3d(&map_dq, sb + C::OFF_STG + db * (C::BM * 128), db * 32, i0, seq.zq);
+              tma_reduce_add_3d(&map_dq, src + db * (C::BM * 128), db * 32, i0, seq.zq);
           } else {  // dK tile of this CTA, 64 key rows per round
             const int r0 = seq.kr + k0 + (p - n_steps) * 64;
     #pragma unroll
             for (int db = 0; db < DG / 32; ++db)
-              tma_reduce_add_3d(&map_dk, sb + C::OFF_STG + db * (C::BM * 128), db * 32, r0, bkg);
+              tma_reduce_add_3d(&map_dk, src + db * (C::BM * 128), db * 32, r0, bkg);
           }
           bulk_commit_group();
+          issued = p + 1;
+          if (C::NSTG == 2) {
+            // The reduce of use p may still be reading its tile; use p-1's tile is free.
+            bulk_wait_group_read1();
+            if (p > 0) mbar_arrive(smem_u32(&bars->stg_free[(p - 1) & 1]));
+          } else {
+            bulk_wait_group_read0();
+            mbar_arrive(smem_u32(&bars->stg_free[p & 1]));
+          }
+        }
+        if (C::NSTG == 2 && issued > 0) {
           bulk_wait_group_read0();
-          mbar_arrive(smem_u32(&bars->stg_free[p & 1]));
+          mbar_arrive(smem_u32(&bars->stg_free[(issued - 1) & 1]));
         }
         bulk_wait_group0();
       }
@@ -500,6 +531,15 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     const bool dq_lane_ok = (C::DQ_M == 128) || lane < 16;
     const int dq_d = (C::DQ_M == 128) ? kl : quarter * 16 + lane;
 
+    // The staging tile of use p is free once the reduce of its previous use has read it:
+    // use p-2 with a tile per step parity, use p-1 with a single tile. Barriers are split
+    // by step parity so no wait is ever more than one phase ahead.
+    auto stg_wait = [&](int p) -> bool {
+      if (C::NSTG == 2)
+        return p < 2 || mbar_wait(smem_u32(&bars->stg_free[p & 1]), ((p - 2) >> 1) & 1);
+      return p < 1 || mbar_wait(smem_u32(&bars->stg_free[(p - 1) & 1]), ((p - 1) >> 1) & 1);
+    };
+
     // dQ^T part of step p (TMEM) -> staging tile (dQ row layout: 32-column boxes of
     // 64 rows x 128 bytes, 128-byte swizzle) -> one bulk reduce-add by warp 11.
     auto drain_dq = [&](int p) -> bool {
@@ -515,13 +555,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->dq_free[wg]));
-      // The staging tile is free once the reduce of step p-1 has read it. Barriers are
-      // split by step parity so this wait is never more than one phase ahead: the
-      // previous wait of this warpgroup (step p-2) already covered step p-3.
-      if (p > 0 && !mbar_wait(smem_u32(&bars->stg_free[(p - 1) & 1]), ((p - 1) >> 1) & 1))
-        return false;
+      if (!stg_wait(p)) return false;
       if (dq_lane_ok) {
-        const uint32_t col = sb + C::OFF_STG + (dq_d >> 5) * (C::BM * 128) + ((dq_d & 3) << 2);
+        const uint32_t col = sb + C::stg_off(p) + (dq_d >> 5) * (C::BM * 128) + ((dq_d & 3) << 2);
         const uint32_t chunk = (dq_d & 31) >> 2;
 #pragma unroll
         for (int i = 0; i < NC; ++i) {
@@ -694,15 +730,14 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       ok = __all_sync(0xffffffffu, ok);
       for (int r = 0; ok && r < 2; ++r) {
         const int p = n_steps + r;
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(smem_u32(&bars->stg_free[(p - 1) & 1]), ((p - 1) >> 1) & 1));
+        ok = __all_sync(0xffffffffu, stg_wait(p));
         if (!ok) break;
         if ((quarter >> 1) == r) {  // this warp's lanes are rows 64r .. 64r+63 of the tile
           const int row = kl - 64 * r;
 #pragma unroll
           for (int c = 0; c < DKH; c += 4) {
             const int dcol = col0 + c;
-            const uint32_t addr = sb + C::OFF_STG + (dcol >> 5) * (C::BM * 128) + row * 128 +
+            const uint32_t addr = sb + C::stg_off(p) + (dcol >> 5) * (C::BM * 128) + row * 128 +
                                   ((((dcol & 31) >> 2) ^ (row & 7)) << 4);
             st_shared_v4(addr, v[c], v[c + 1], v[c + 2], v[c + 3]);
           }
