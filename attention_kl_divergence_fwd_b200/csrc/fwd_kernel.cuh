@@ -132,9 +132,9 @@ struct RowState {
 
 // Which column pairs (c, c+1) send their second exponential of both distributions to the
 // FMA pipe: the first SKL_FWD_POLY entries of the order 1, 5, 3, 7, 6, 2, 4, 0 over every 8
-// consecutive pairs, i.e. SKL_FWD_POLY/16 of all exponentials (2: 12.5 %).
+// consecutive pairs, i.e. SKL_FWD_POLY/16 of all exponentials (1: 6.25 %).
 #ifndef SKL_FWD_POLY
-#define SKL_FWD_POLY 2
+#define SKL_FWD_POLY 1
 #endif
 __host__ __device__ constexpr int poly_rank(int p) {
   return p == 1 ? 0 : p == 5 ? 1 : p == 3 ? 2 : p == 7 ? 3 : p == 6 ? 4 : p == 2 ? 5 : p == 4 ? 6 : 7;
