@@ -31,7 +31,8 @@ EXPORTS = ("streamkl_fwd", "streamkl_bwd", "streamkl_bwd_teacher", "streamkl_fwd
            "streamkl_bwd_gqa", "streamkl_bwd_teacher_gqa", "streamkl_fwd_varlen",
            "streamkl_bwd_varlen", "streamkl_bwd_teacher_varlen", "streamkl_fwd_partial",
            "streamkl_merge_partial", "streamkl_bwd_shard", "streamkl_bwd_teacher_shard",
-           "streamkl_status_string", "streamkl_device_status", "streamkl_version")
+           "streamkl_watchdog_selftest", "streamkl_status_string", "streamkl_device_status",
+           "streamkl_version")
 
 
 class StreamKLError(RuntimeError):
@@ -89,6 +90,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.streamkl_bwd_shard.restype = i
     lib.streamkl_bwd_teacher_shard.argtypes = shead + [vp, vp, vp, vp, vp, vp, vp]
     lib.streamkl_bwd_teacher_shard.restype = i
+    lib.streamkl_watchdog_selftest.argtypes = [vp]
+    lib.streamkl_watchdog_selftest.restype = i
     lib.streamkl_status_string.argtypes = [i]
     lib.streamkl_status_string.restype = ctypes.c_char_p
     lib.streamkl_device_status.argtypes = [vp]
@@ -468,6 +471,13 @@ def streamkl_bwd_teacher_shard(q_t, k_t, q_s, k_s, scale_T: float, scale_S: floa
         dq_t.data_ptr(), dk_t.data_ptr(), _stream_ptr(stream))
     _check(st, "streamkl_bwd_teacher_shard")
     return dq_t, dk_t
+
+
+def watchdog_selftest(stream=None) -> None:
+    """Let one bounded pipeline wait expire on purpose (about 2 s); device_status() then
+    reports STREAMKL_ERR_TIMEOUT (5)."""
+    _check(load_library().streamkl_watchdog_selftest(_stream_ptr(stream)),
+           "streamkl_watchdog_selftest")
 
 
 def device_status(stream=None) -> int:

@@ -47,4 +47,16 @@ streamkl_merge_kernel(const float* __restrict__ states, int R, long long rows,
   }
 }
 
+// Watchdog self-test: one thread waits, through the same bounded wait as every pipeline
+// wait of the library, on an mbarrier that nothing arrives on. The wait gives up after its
+// time limit and the error word records it, exactly as a stalled pipeline would.
+__global__ void streamkl_watchdog_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+    if (!mbar_wait(smem_u32(&bar), 0)) atomicOr(&g_skl_error, 16u);
+  }
+}
+
 }  // namespace skl

@@ -15,8 +15,9 @@ namespace skl {
 // Device-side error word of this library (one per device, in the library's module):
 // bit 0 = a forward watchdog fired, bit 1 = a backward watchdog fired, bit 2 = the
 // dynamic shared memory was not 1024-byte aligned, bit 3 = malformed packed-sequence
-// offsets. Read and cleared by streamkl_device_status(). The library is built as one
-// translation unit, so this is the only definition.
+// offsets, bit 4 = the watchdog self-test's wait expired. Read and cleared by
+// streamkl_device_status(). The library is built as one translation unit, so this is the
+// only definition.
 __device__ unsigned int g_skl_error = 0;
 
 // ----------------------------------------------------------------- misc

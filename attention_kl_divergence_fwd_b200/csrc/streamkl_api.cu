@@ -501,6 +501,11 @@ streamkl_status streamkl_bwd_teacher_shard(const void* q_t, const void* k_t, con
                           lse_s, g, dq_t, dk_t, stream);
 }
 
+streamkl_status streamkl_watchdog_selftest(cudaStream_t stream) {
+  skl::streamkl_watchdog_kernel<<<1, 32, 0, stream>>>();
+  return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
+}
+
 const char* streamkl_status_string(streamkl_status s) {
   switch (s) {
     case STREAMKL_OK: return "ok";

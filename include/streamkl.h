@@ -235,6 +235,14 @@ streamkl_status streamkl_bwd_teacher_shard(const void* q_t, const void* k_t, con
                                            const float* g, float* dq_t, float* dk_t,
                                            cudaStream_t stream);
 
+/*
+ * Diagnostic: launches one thread that waits, with the library's bounded pipeline wait
+ * (2 s), on a barrier nothing arrives on. After it gives up, streamkl_device_status(stream)
+ * returns STREAMKL_ERR_TIMEOUT, exactly as for a kernel whose pipeline stalled, and the
+ * context stays usable. Returns STREAMKL_OK when the launch succeeded.
+ */
+streamkl_status streamkl_watchdog_selftest(cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char* streamkl_status_string(streamkl_status status);
 

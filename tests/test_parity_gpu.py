@@ -490,3 +490,19 @@ def test_context_parallel_autograd_single_rank():
     assert torch.equal(grads[0][0], grads[1][0])
     assert torch.equal(grads[0][2], grads[1][2])
     assert rel_fro(grads[1][1].cpu().double(), grads[0][1].cpu().double()) < 1e-2
+
+
+# ------------------------------------------------ failure detection
+
+def test_watchdog_expiry_is_reported_and_the_context_survives():
+    """A bounded pipeline wait that runs out (a barrier nothing arrives on) sets the error
+    word; the host reads STREAMKL_ERR_TIMEOUT, the word is cleared, and later calls work."""
+    import time
+    assert skl.device_status() == 0
+    t0 = time.time()
+    skl.watchdog_selftest()
+    assert skl.device_status() == 5  # STREAMKL_ERR_TIMEOUT
+    assert time.time() - t0 >= 1.0   # the wait ran to its limit
+    assert skl.device_status() == 0  # cleared by the read
+    w = WORKLOADS["tiny_n256_d64"]
+    check_full(w, make_inputs(w))    # the context is still usable
