@@ -13,24 +13,28 @@
 //                              dQ_T = dS K_T,   dK_T = dS^T Q_T.
 // Both recompute both score tiles; the teacher variant needs one exponential per pair.
 //
-// CTA = one tile of 128 keys of one (batch, head), resident in shared memory. It walks
-// the 64-row query tiles ("steps") that can see those keys. Per step s:
-//   1. tensor core: S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T into TMEM buffer s&1
-//      (keys on the 128 lanes, 64 query columns);
-//   2. warpgroup s&1 (one thread per key) recomputes P_T, P_S, forms dS^T in registers
-//      and stores it as bf16 into shared-memory buffer s&1;
-//   3. tensor core: dK_S += dS^T Q_S (TMEM accumulator over all steps) and
-//      dQ^T_part = K_S^T dS^T into TMEM buffer s&1 (d_S on the lanes, queries on columns);
-//   4. the same warpgroup copies dQ^T_part from TMEM into a shared-memory staging tile
+// CTA = one tile of 128 keys of one (batch, head), resident in shared memory (and, by
+// default, copied into TMEM). It walks the 64-row query tiles ("steps") that can see those
+// keys. Per step s:
+//   1. tensor core: S_T^T = K_T Q_T^T and S_S^T = K_S Q_S^T into TMEM (keys on the 128
+//      lanes, 64 query columns), K read from TMEM as the A operand;
+//   2. the dS warps of step parity s&1 (one thread per key row, each warp 32 of the 64
+//      query columns) recompute P_T, P_S, form dS^T in registers and store it as bf16
+//      into shared-memory buffer s&1;
+//   3. tensor core: dK += dS^T Q (TMEM accumulator over all steps) and
+//      dQ^T_part = K^T dS^T into TMEM buffer s&1 (d on the lanes, queries on columns);
+//   4. the same warps copy dQ^T_part from TMEM into the fp32 staging tile of parity s&1,
 //      laid out as dQ rows, and one thread adds the tile into dQ with a bulk tensor
 //      reduce-add (the fp32 adds happen in L2).
-// Score tiles, dS tiles and dQ parts are double-buffered, so the two warpgroups work on
-// alternate steps while the tensor core computes the next ones.
+// dS tiles, dQ parts and staging tiles are double-buffered by step parity, so the two
+// groups of dS warps work on alternate steps while the tensor core computes the next.
 //
-// Warp roles (384 threads): warps 0-3 even steps, warps 4-7 odd steps, warp 8 TMA
-// producer, warp 9 TMEM allocator + MMA issuer, warp 10 row-statistics loader (global
-// loads issued several steps ahead so their latency never reaches the pipeline), warp 11
-// issues the dQ reduce-adds.
+// Warp roles (640 threads, the default switches): warps 0-15 dS (warp w: step parity
+// (w >> 2) & 1, query columns 32 (w >> 3) .. +31, key rows 32 (w & 3) .. +31), warp 16 TMA
+// producer, warp 17 TMEM allocator + MMA issuer, warp 18 row-statistics loader (global
+// loads issued several steps ahead so their latency never reaches the pipeline), warp 19
+// issues the dQ (and shared-K dK) reduce-adds. The switches below select the measured
+// alternatives (8 dS warps, K only in shared memory, one staging tile).
 #pragma once
 
 #include "ptx.cuh"
@@ -541,7 +545,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     };
 
     // dQ^T part of step p (TMEM) -> staging tile (dQ row layout: 32-column boxes of
-    // 64 rows x 128 bytes, 128-byte swizzle) -> one bulk reduce-add by warp 11.
+    // 64 rows x 128 bytes, 128-byte swizzle) -> one bulk reduce-add by the reduce warp.
     auto drain_dq = [&](int p) -> bool {
       if (!mbar_wait(smem_u32(&bars->dq_full[wg]), (p >> 1) & 1)) return false;
       tc_fence_after();

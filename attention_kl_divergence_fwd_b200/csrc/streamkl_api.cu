@@ -3,7 +3,8 @@
 // The planner picks the kernel instantiation from (d_T, d_S), encodes the TMA tensor
 // maps (dense [B*H, N, d] or packed [total, heads, d] bf16, 128-byte swizzle, zero fill
 // out of bounds so ragged N needs no padding), orders the grid so causal work is
-// scheduled heaviest-first, and launches on the caller's stream. See include/streamkl.h for the contract.
+// scheduled heaviest-first, and launches on the caller's stream. include/streamkl.h
+// states the contract.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
