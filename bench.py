@@ -425,6 +425,9 @@ def run_context_parallel(skl, w, d, dev, stream, steps, world, shards=4):
     side by side: partial forwards, the merge of their states, shard backwards. The
     all-gather / all-reduce between ranks is not part of it (one GPU)."""
     from attention_kl_divergence_fwd_b200.context_parallel import even_shards
+    shards = min(shards, -(-w.N_K // 128))  # at least one 128-key tile per shard
+    if shards < 2:
+        return None
     cuts = even_shards(w.N_K, shards)
     ks = [(d["k_t"][:, :, a:a + n].contiguous(), d["k_s"][:, :, a:a + n].contiguous(), a)
           for a, n in cuts]
