@@ -506,3 +506,37 @@ def test_watchdog_expiry_is_reported_and_the_context_survives():
     assert skl.device_status() == 0  # cleared by the read
     w = WORKLOADS["tiny_n256_d64"]
     check_full(w, make_inputs(w))    # the context is still usable
+
+
+def test_gqa_full_size_sampled():
+    """Grouped-query attention at a full configuration size (B=2, H=16, N=4096, causal):
+    teacher K with 8 heads, student K with 4 heads (groups of 2 and 4). Sampled query rows
+    against the per-row oracle; dK of two shared student heads against the sum of the
+    oracle's per-query-head dK over each group."""
+    from oracle.streamkl_oracle import expand_kv
+    w = WORKLOADS["b2h16_n4096_d128_causal"]
+    x = make_inputs(w)
+    x["k_t"] = x["k_t"][:, :8].contiguous()
+    x["k_s"] = x["k_s"][:, :4].contiguous()
+    d = to_dev(x)
+    a = (d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal)
+    kl, lt, ls = skl.streamkl_fwd_gqa(*a)
+    dq, dk = skl.streamkl_bwd_gqa(*a, lt, ls, d["g"])
+    assert skl.device_status() == 0
+    kl, lt, ls, dq, dk = (t.cpu().double() for t in (kl, lt, ls, dq, dk))
+    ex = (x["q_t"], expand_kv(x["k_t"], w.H), x["q_s"], expand_kv(x["k_s"], w.H), w.scale_T,
+          w.scale_S, w.causal, x["g"])
+    rows = sample_rows(w, 256)
+    kl_r, lt_r, ls_r, dq_r = oracle_rows(*ex, rows)
+    idx = torch.tensor([bh * w.N_Q + i for bh, i in rows])
+    check_kl(kl.reshape(-1)[idx], kl_r)
+    check_lse(lt.reshape(-1)[idx], lt_r)
+    check_lse(ls.reshape(-1)[idx], ls_r)
+    assert rel_fro(dq.reshape(-1, w.d_S)[idx], dq_r) <= GRAD_REL
+    keys = sorted(set([0, w.N_K - 1] + torch.randperm(w.N_K, generator=torch.Generator()
+                                                       .manual_seed(5))[:62].tolist()))
+    for b, hk in [(0, 1), (1, 3)]:
+        ref = sum(oracle_dk_rows(*ex, b * w.H + h, keys, row_block=1024)
+                  for h in range(hk * 4, hk * 4 + 4))
+        assert rel_fro(dk[b, hk, keys], ref) <= GRAD_REL, rel_fro(dk[b, hk, keys], ref)
+    assert torch.isfinite(kl).all() and kl.min().item() >= -1e-5
