@@ -540,3 +540,22 @@ def test_gqa_full_size_sampled():
                   for h in range(hk * 4, hk * 4 + 4))
         assert rel_fro(dk[b, hk, keys], ref) <= GRAD_REL, rel_fro(dk[b, hk, keys], ref)
     assert torch.isfinite(kl).all() and kl.min().item() >= -1e-5
+
+
+def test_teacher_grads_full_size_two_heads():
+    """Trainable-teacher gradients at a full configuration size (B=2, H=16, N=4096,
+    causal). Heads are independent, so two of them are checked element by element against
+    the oracle run on those heads alone."""
+    w = WORKLOADS["b2h16_n4096_d128_causal"]
+    x = make_inputs(w)
+    d = to_dev(x)
+    a = (d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal)
+    kl, lt, ls = skl.streamkl_fwd(*a)
+    dq_t, dk_t = skl.streamkl_bwd_teacher(*a, kl, lt, ls, d["g"])
+    assert skl.device_status() == 0
+    for b, h in [(0, 0), (1, 15)]:
+        one = {k: v[b:b + 1, h:h + 1] for k, v in x.items()}
+        dq_r, dk_r = oracle_bwd_teacher(one["q_t"], one["k_t"], one["q_s"], one["k_s"], w.scale_T,
+                                        w.scale_S, w.causal, one["g"])
+        assert rel_fro(dq_t[b, h].cpu().double(), dq_r[0, 0]) <= GRAD_REL
+        assert rel_fro(dk_t[b, h].cpu().double(), dk_r[0, 0]) <= GRAD_REL
