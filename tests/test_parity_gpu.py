@@ -559,3 +559,25 @@ def test_teacher_grads_full_size_two_heads():
                                         w.scale_S, w.causal, one["g"])
         assert rel_fro(dq_t[b, h].cpu().double(), dq_r[0, 0]) <= GRAD_REL
         assert rel_fro(dk_t[b, h].cpu().double(), dk_r[0, 0]) <= GRAD_REL
+
+
+def test_config2_full_oracle():
+    """Config 2 (B=2, H=16, N=4096, d=128, causal) compared in full: every KL and LSE row
+    and the whole dQ_S and dK_S against the fp64 oracle (about 0.4 TFLOP of fp64 on the
+    host)."""
+    w = WORKLOADS["b2h16_n4096_d128_causal"]
+    x = make_inputs(w)
+    g = run_gpu(w, x)
+    args = (x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S, w.causal)
+    kl, lt, ls = oracle_fwd(*args)
+    check_kl(g["kl"], kl)
+    check_lse(g["lse_t"], lt)
+    check_lse(g["lse_s"], ls)
+    dq, dk = oracle_bwd(*args, x["g"])
+    assert rel_fro(g["dq"], dq) <= GRAD_REL, rel_fro(g["dq"], dq)
+    assert rel_fro(g["dk"], dk) <= GRAD_REL, rel_fro(g["dk"], dk)
+    # per head as well, so that one bad head cannot hide in the global norm
+    for bh in range(w.bh):
+        b, h = divmod(bh, w.H)
+        assert rel_fro(g["dq"][b, h], dq[b, h]) <= GRAD_REL
+        assert rel_fro(g["dk"][b, h], dk[b, h]) <= GRAD_REL
