@@ -31,8 +31,8 @@ EXPORTS = ("streamkl_fwd", "streamkl_bwd", "streamkl_bwd_teacher", "streamkl_fwd
            "streamkl_bwd_gqa", "streamkl_bwd_teacher_gqa", "streamkl_fwd_varlen",
            "streamkl_bwd_varlen", "streamkl_bwd_teacher_varlen", "streamkl_fwd_partial",
            "streamkl_merge_partial", "streamkl_bwd_shard", "streamkl_bwd_teacher_shard",
-           "streamkl_watchdog_selftest", "streamkl_status_string", "streamkl_device_status",
-           "streamkl_version")
+           "streamkl_watchdog_selftest", "streamkl_exp2_eval", "streamkl_status_string",
+           "streamkl_device_status", "streamkl_version")
 
 
 class StreamKLError(RuntimeError):
@@ -90,6 +90,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.streamkl_bwd_shard.restype = i
     lib.streamkl_bwd_teacher_shard.argtypes = shead + [vp, vp, vp, vp, vp, vp, vp]
     lib.streamkl_bwd_teacher_shard.restype = i
+    lib.streamkl_exp2_eval.argtypes = [vp, vp, vp, ctypes.c_longlong, vp]
+    lib.streamkl_exp2_eval.restype = i
     lib.streamkl_watchdog_selftest.argtypes = [vp]
     lib.streamkl_watchdog_selftest.restype = i
     lib.streamkl_status_string.argtypes = [i]
@@ -478,6 +480,18 @@ def watchdog_selftest(stream=None) -> None:
     reports STREAMKL_ERR_TIMEOUT (5)."""
     _check(load_library().streamkl_watchdog_selftest(_stream_ptr(stream)),
            "streamkl_watchdog_selftest")
+
+
+def exp2_eval(x, stream=None):
+    """The forward's FMA-pipe 2^x on a float32 CUDA tensor with an even number of elements:
+    (scalar form, packed-pair form)."""
+    import torch
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous() or x.numel() % 2:
+        raise ValueError("x must be a contiguous float32 CUDA tensor with an even size")
+    y1, y2 = torch.empty_like(x), torch.empty_like(x)
+    _check(load_library().streamkl_exp2_eval(x.data_ptr(), y1.data_ptr(), y2.data_ptr(),
+                                             x.numel(), _stream_ptr(stream)), "streamkl_exp2_eval")
+    return y1, y2
 
 
 def device_status(stream=None) -> int:

@@ -59,4 +59,20 @@ __global__ void streamkl_watchdog_kernel() {
   }
 }
 
+// Evaluates the FMA-pipe exp2 (scalar and packed-pair forms) on n inputs, for checking it
+// against the exact 2^x and CUDA's exp2f. n is even; one thread per pair.
+__global__ void streamkl_exp2_kernel(const float* __restrict__ x, float* __restrict__ y1,
+                                     float* __restrict__ y2, long long n) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x; 2 * k < n; k += stride) {
+    const float a = x[2 * k], b = x[2 * k + 1];
+    y1[2 * k] = exp2_fma(a);
+    y1[2 * k + 1] = exp2_fma(b);
+    float p, q;
+    f2_unpack(exp2_fma2(f2_pack(a, b)), p, q);
+    y2[2 * k] = p;
+    y2[2 * k + 1] = q;
+  }
+}
+
 }  // namespace skl

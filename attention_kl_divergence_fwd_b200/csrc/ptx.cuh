@@ -32,8 +32,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
-
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;
   asm volatile(
@@ -280,19 +278,6 @@ __device__ __forceinline__ void tmem_ld_4x32_wait(uint32_t ta, uint32_t tb, uint
       : "memory");
 }
 
-// Two 16-column loads (lanes = this warp's quarter) followed by the wait.
-__device__ __forceinline__ void tmem_ld_2x16_wait(uint32_t ta, uint32_t tb, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n"
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n"
-      "tcgen05.wait::ld.sync.aligned;\n"
-      : SKL_R8(0), SKL_R8(8), SKL_R8(16), SKL_R8(24)
-      : "r"(ta), "r"(tb)
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_ld_16_wait(uint32_t ta, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -516,32 +501,6 @@ __device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
                  __int_as_float(__float_as_int(p1) + (__float_as_int(y1) << 23)));
 }
 
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
-// Lower-accuracy pair variant for values that are rounded to bf16 afterwards: degree-3
-// polynomial from the same fit (fit_exp2_poly.py), max relative error 7.5e-5.
-__device__ __forceinline__ uint64_t exp2_fma2_d3(uint64_t x) {
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t kShift = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t y = f2_add(x, kShift);
-  const uint64_t f = f2_sub(x, f2_sub(y, kShift));
-  uint64_t p = f2_pack(0.055171750485897064f, 0.055171750485897064f);
-  p = f2_fma(p, f, f2_pack(0.24261131882667542f, 0.24261131882667542f));
-  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-  float p0, p1, y0, y1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(y, y0, y1);
-  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(y0) << 23)),
-                 __int_as_float(__float_as_int(p1) + (__float_as_int(y1) << 23)));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -560,12 +519,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void red_add_v4(float* gaddr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(gaddr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
                : "memory");
 }
 
@@ -601,10 +554,6 @@ __device__ __forceinline__ void bulk_wait_group0() {
 
 __device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-
-__device__ __forceinline__ void red_add_f32(float* gaddr, float a) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(gaddr), "f"(a) : "memory");
 }
 
 // Per-warpgroup register budget changes (every warp of the warpgroup executes them).

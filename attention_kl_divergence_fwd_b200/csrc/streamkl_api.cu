@@ -507,6 +507,16 @@ streamkl_status streamkl_watchdog_selftest(cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
 }
 
+streamkl_status streamkl_exp2_eval(const float* x, float* y_scalar, float* y_pair, long long n,
+                                   cudaStream_t stream) {
+  if (!x || !y_scalar || !y_pair || n < 2 || (n & 1)) return STREAMKL_ERR_INVALID_ARG;
+  const long long pairs = n / 2;
+  const long long need = (pairs + 255) / 256;
+  const unsigned grid = (unsigned)(need < 148 * 16 ? need : 148 * 16);
+  skl::streamkl_exp2_kernel<<<grid, 256, 0, stream>>>(x, y_scalar, y_pair, n);
+  return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
+}
+
 const char* streamkl_status_string(streamkl_status s) {
   switch (s) {
     case STREAMKL_OK: return "ok";

@@ -243,6 +243,16 @@ streamkl_status streamkl_bwd_teacher_shard(const void* q_t, const void* k_t, con
  */
 streamkl_status streamkl_watchdog_selftest(cudaStream_t stream);
 
+/*
+ * Diagnostic: the forward's FMA-pipe 2^x (range reduction with the 1.5*2^23 shifter, a
+ * degree-5 minimax polynomial fitted for this library, the integer part added into the
+ * exponent field) evaluated on n device floats x (n even), scalar form into y_scalar and
+ * packed-pair form into y_pair. Inputs below -125 give 2^-125. INVALID_ARG for null pointers
+ * or odd n.
+ */
+streamkl_status streamkl_exp2_eval(const float* x, float* y_scalar, float* y_pair, long long n,
+                                   cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char* streamkl_status_string(streamkl_status status);
 

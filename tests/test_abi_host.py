@@ -26,7 +26,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(streamkl_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(streamkl_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_exports():
@@ -36,7 +36,7 @@ def test_header_declares_the_exports():
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", skl.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\bT (streamkl_[a-z_]+)\b", out))
+    exported = set(re.findall(r"\bT (streamkl_[a-z0-9_]+)\b", out))
     for name in declared_functions():
         assert name in exported, name
         assert hasattr(lib, name)

@@ -581,3 +581,24 @@ def test_config2_full_oracle():
         b, h = divmod(bh, w.H)
         assert rel_fro(g["dq"][b, h], dq[b, h]) <= GRAD_REL
         assert rel_fro(g["dk"][b, h], dk[b, h]) <= GRAD_REL
+
+
+def test_fma_pipe_exp2_accuracy():
+    """The forward's polynomial 2^x against the exact value (fp64) and against CUDA's exp2f:
+    relative error within the fitted bound (1.9e-7) plus fp32 rounding of the evaluation."""
+    gen = torch.Generator().manual_seed(3)
+    x = torch.cat([torch.linspace(-124.0, 0.0, 1 << 20),
+                   -124.0 * torch.rand(1 << 20, generator=gen),
+                   torch.tensor([0.0, -0.5, 0.5 - 1.0, -1.0, -2.5, -124.0])])
+    y1, y2 = skl.exp2_eval(x.cuda())
+    exact = torch.exp2(x.double())
+    for y in (y1, y2):
+        rel = ((y.cpu().double() - exact) / exact).abs()
+        assert rel.max().item() <= 4e-7, rel.max().item()
+    cuda = torch.exp2(x.cuda()).cpu().double()  # CUDA's exp2f
+    assert ((y1.cpu().double() - cuda) / cuda).abs().max().item() <= 5e-7
+    assert torch.equal(y1, y2)  # the packed form computes the same values
+    # below the clamp: 2^-125
+    lo, _ = skl.exp2_eval(torch.tensor([-200.0, -125.0], device="cuda"))
+    assert torch.allclose(lo.cpu().double(), torch.full((2,), 2.0 ** -125, dtype=torch.float64),
+                          rtol=4e-7, atol=0)
