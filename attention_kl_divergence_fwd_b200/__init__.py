@@ -20,6 +20,7 @@ int32 offsets cu_seqlens_q / cu_seqlens_k [B+1] on the device, row statistics an
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 from typing import Optional, Tuple
 
@@ -114,6 +115,29 @@ def _check(status: int, where: str) -> None:
         raise StreamKLError(status, where)
 
 
+def _on_device(fn):
+    """Runs a tensor-level entry point on the CUDA device of its tensor arguments: all of
+    them (and a given stream) must be on one device, which is made current for the call so
+    that the default stream and the launch are on that device."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        import torch
+        ts = [a for a in list(args) + list(kwargs.values()) if isinstance(a, torch.Tensor)]
+        devs = {t.device for t in ts}
+        if len(devs) > 1:
+            raise ValueError(f"{fn.__name__}: tensors on different devices: "
+                             f"{sorted(str(d) for d in devs)}")
+        if not ts or next(iter(devs)).type != "cuda":
+            return fn(*args, **kwargs)  # the entry point's own checks reject non-CUDA input
+        dev = next(iter(devs))
+        stream = kwargs.get("stream")
+        if stream is not None and stream.device != dev:
+            raise ValueError(f"{fn.__name__}: stream on {stream.device}, tensors on {dev}")
+        with torch.cuda.device(dev):
+            return fn(*args, **kwargs)
+    return wrapper
+
+
 def _stream_ptr(stream) -> int:
     import torch
     s = torch.cuda.current_stream() if stream is None else stream
@@ -161,6 +185,7 @@ def streamkl_bwd_teacher_raw(q_t: int, k_t: int, q_s: int, k_s: int, B: int, H: 
                                                dk_t, stream)
 
 
+@_on_device
 def streamkl_fwd(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
                  kl=None, lse_t=None, lse_s=None, stream=None):
     """Per-row KL(P_T || P_S), LSE_T, LSE_S (fp32 [B,H,N_Q]) on the current stream."""
@@ -178,6 +203,7 @@ def streamkl_fwd(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: boo
     return kl, lse_t, lse_s
 
 
+@_on_device
 def streamkl_bwd(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
                  lse_t, lse_s, g, dq_s=None, dk_s=None, stream=None):
     """dQ_S [B,H,N_Q,d_S] and dK_S [B,H,N_K,d_S] (fp32) of sum_i g_i KL_i."""
@@ -199,6 +225,7 @@ def streamkl_bwd(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: boo
     return dq_s, dk_s
 
 
+@_on_device
 def streamkl_bwd_teacher(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
                          kl, lse_t, lse_s, g, dq_t=None, dk_t=None, stream=None):
     """dQ_T [B,H,N_Q,d_T] and dK_T [B,H,N_K,d_T] (fp32) of sum_i g_i KL_i (trainable teacher)."""
@@ -236,6 +263,7 @@ def _shape_gqa(q_t, k_t, q_s, k_s):
     return B, H, h_kt, h_ks, n_q, n_k, d_t, d_s
 
 
+@_on_device
 def streamkl_fwd_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
                      kl=None, lse_t=None, lse_s=None, stream=None):
     """streamkl_fwd with grouped K heads (k_* may have fewer heads than q_*)."""
@@ -254,6 +282,7 @@ def streamkl_fwd_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal:
     return kl, lse_t, lse_s
 
 
+@_on_device
 def streamkl_bwd_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
                      lse_t, lse_s, g, dq_s=None, dk_s=None, stream=None):
     """streamkl_bwd with grouped K heads; dk_s has the student's K-head count."""
@@ -273,6 +302,7 @@ def streamkl_bwd_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal:
     return dq_s, dk_s
 
 
+@_on_device
 def streamkl_bwd_teacher_gqa(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
                              kl, lse_t, lse_s, g, dq_t=None, dk_t=None, stream=None):
     """streamkl_bwd_teacher with grouped K heads; dk_t has the teacher's K-head count."""
@@ -329,6 +359,7 @@ def _shape_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k):
     return cu_q.numel() - 1, H, h_kt, h_ks, total_q, total_k, d_t, d_s
 
 
+@_on_device
 def streamkl_fwd_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                         max_seqlen_k: int, scale_T: float, scale_S: float, causal: bool,
                         kl=None, lse_t=None, lse_s=None, stream=None):
@@ -351,6 +382,7 @@ def streamkl_fwd_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k, max_seql
     return kl, lse_t, lse_s
 
 
+@_on_device
 def streamkl_bwd_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                         max_seqlen_k: int, scale_T: float, scale_S: float, causal: bool,
                         lse_t, lse_s, g, dq_s=None, dk_s=None, stream=None):
@@ -373,6 +405,7 @@ def streamkl_bwd_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k, max_seql
     return dq_s, dk_s
 
 
+@_on_device
 def streamkl_bwd_teacher_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k,
                                 max_seqlen_q: int, max_seqlen_k: int, scale_T: float,
                                 scale_S: float, causal: bool, kl, lse_t, lse_s, g, dq_t=None,
@@ -398,6 +431,7 @@ def streamkl_bwd_teacher_varlen(q_t, k_t, q_s, k_s, cu_seqlens_q, cu_seqlens_k,
     return dq_t, dk_t
 
 
+@_on_device
 def streamkl_fwd_partial(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
                          k_offset: int, n_k_total: int, state=None, stream=None):
     """Row state of one key shard (k_* hold the shard's keys): fp32 [5, B, H, N_Q], planes
@@ -414,6 +448,7 @@ def streamkl_fwd_partial(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, cau
     return state
 
 
+@_on_device
 def streamkl_merge_partial(states, kl=None, lse_t=None, lse_s=None, stream=None):
     """Merge gathered shard states [R, 5, B, H, N_Q] into KL, LSE_T, LSE_S [B, H, N_Q]."""
     import torch
@@ -432,6 +467,7 @@ def streamkl_merge_partial(states, kl=None, lse_t=None, lse_s=None, stream=None)
     return kl, lse_t, lse_s
 
 
+@_on_device
 def streamkl_bwd_shard(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causal: bool,
                        k_offset: int, n_k_total: int, lse_t, lse_s, g, dq_s=None, dk_s=None,
                        stream=None):
@@ -454,6 +490,7 @@ def streamkl_bwd_shard(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float, causa
     return dq_s, dk_s
 
 
+@_on_device
 def streamkl_bwd_teacher_shard(q_t, k_t, q_s, k_s, scale_T: float, scale_S: float,
                                causal: bool, k_offset: int, n_k_total: int, kl, lse_t, lse_s, g,
                                dq_t=None, dk_t=None, stream=None):
@@ -482,6 +519,7 @@ def watchdog_selftest(stream=None) -> None:
            "streamkl_watchdog_selftest")
 
 
+@_on_device
 def exp2_eval(x, stream=None):
     """The forward's FMA-pipe 2^x on a float32 CUDA tensor with an even number of elements:
     (scalar form, packed-pair form)."""

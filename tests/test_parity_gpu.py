@@ -602,3 +602,15 @@ def test_fma_pipe_exp2_accuracy():
     lo, _ = skl.exp2_eval(torch.tensor([-200.0, -125.0], device="cuda"))
     assert torch.allclose(lo.cpu().double(), torch.full((2,), 2.0 ** -125, dtype=torch.float64),
                           rtol=4e-7, atol=0)
+
+
+def test_mixed_devices_rejected_before_any_launch():
+    w = WORKLOADS["tiny_n256_d64"]
+    x = make_inputs(w)
+    d = to_dev(x)
+    with pytest.raises(ValueError):
+        skl.streamkl_fwd(d["q_t"], x["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, False)
+    with pytest.raises(ValueError):
+        skl.streamkl_bwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, False,
+                         torch.zeros(1, 1, 256, device="cuda"), torch.zeros(1, 1, 256), d["g"])
+    assert skl.device_status() == 0
