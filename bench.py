@@ -299,12 +299,15 @@ def main():
     bwd_tf = fb / (bwd_ms * 1e-3) / 1e12
     dominant = "bwd" if bwd_ms >= fwd_ms else "fwd"
     traffic = load_traffic(w.name, dominant)
+    # The timed region is tens of milliseconds and the clocks stay at their maximum (see
+    # "clocks"), so the denominator is the burst cuBLAS figure; the fraction of the
+    # sustained (power-capped, seconds-long loop) figure is reported beside it.
+    achieved = bwd_tf if dominant == "bwd" else fwd_tf
     roof = {"kernel": f"streamkl_{dominant}_kernel", "bound": "tensor",
-            "achieved": bwd_tf if dominant == "bwd" else fwd_tf,
-            "peak": peak_sus, "unit": "TFLOP/s",
-            "frac": (bwd_tf if dominant == "bwd" else fwd_tf) / peak_sus,
-            "traffic": traffic,
-            "peak_kind": f"{peak_kind} bf16 dense, sustained (kernel timed inside a long loop)"}
+            "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
+            "frac": achieved / peak_burst, "traffic": traffic,
+            "peak_kind": f"{peak_kind} bf16 dense, burst (short timed region at full clocks)",
+            "frac_of_sustained_peak": achieved / peak_sus}
 
     # Trainable-teacher backward (streamkl_bwd_teacher), timed on its own: not part of the
     # step (the teacher is frozen in the measured workload), reported beside it.
@@ -367,9 +370,9 @@ def main():
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                "dtype": "bf16", "data": "synthetic", "config": config_of(w, world),
                "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
-               "fwd_frac_peak": fwd_tf / peak_sus, "bwd_frac_peak": bwd_tf / peak_sus,
-               "fwd_frac_burst_peak": fwd_tf / peak_burst,
-               "bwd_frac_burst_peak": bwd_tf / peak_burst,
+               "fwd_frac_peak": fwd_tf / peak_burst, "bwd_frac_peak": bwd_tf / peak_burst,
+               "fwd_frac_sustained_peak": fwd_tf / peak_sus,
+               "bwd_frac_sustained_peak": bwd_tf / peak_sus,
                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
                "gqa": gqa, "varlen": varlen, "context_parallel": cp,
                "bwd_teacher_ms": bwd_t_ms,
