@@ -221,6 +221,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-eager", action="store_true",
+                    help="skip the PyTorch eager materialising comparator")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="host time of the cpu_baseline leg of this arm")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
@@ -356,6 +358,12 @@ def main():
     varlen = run_varlen(skl, w, dev, stream, args.steps, world) if w.d_T == w.d_S else None
     cp = run_context_parallel(skl, w, d, dev, stream, args.steps, world)
 
+    eager = None
+    if rank == 0 and not args.no_eager:
+        skl.streamkl_fwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal,
+                         kl=kl, lse_t=lt, lse_s=ls)  # the buffers held the variants' rows
+        eager = run_eager(w, d, kl, dev, stream, fwd_ms, bwd_ms)
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(skl, w, x, dev, stream, args.steps, world)
@@ -374,7 +382,7 @@ def main():
                "fwd_frac_sustained_peak": fwd_tf / peak_sus,
                "bwd_frac_sustained_peak": bwd_tf / peak_sus,
                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-               "gqa": gqa, "varlen": varlen, "context_parallel": cp,
+               "gqa": gqa, "varlen": varlen, "context_parallel": cp, "eager_baseline": eager,
                "bwd_teacher_ms": bwd_t_ms,
                "bwd_teacher_tflops": flops_bwd_teacher(w) / (bwd_t_ms * 1e-3) / 1e12,
                "gpu_launches": 2 * args.steps,
@@ -528,6 +536,81 @@ def run_e2e(skl, w, x, dev, stream, steps, world):
     return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps,
             "pipeline": "host->device copies on a second stream, double-buffered"}
+
+
+def run_eager(w, d, kl_fused, dev, stream, fwd_ms, bwd_ms, steps=2, budget_bytes=24 << 30):
+    """The materialising comparator the pages measure against, timed on the same GPU:
+    plain PyTorch eager ops that form both N_Q x N_K score matrices (bf16 matmul as under
+    autocast, then fp32), both log-softmaxes and the row-wise KL, and differentiate
+    sum_i g_i KL_i with autograd for dQ_S and dK_S. Heads are processed in chunks sized
+    to the memory budget (the whole batch at once does not fit for long sequences).
+    Returns times per step, the speedups of the fused kernels over it and the peak extra
+    memory of one chunk, and the largest difference of its per-row KL from the fused
+    forward's (its scores are rounded to bf16, the fused kernels keep them in fp32); a
+    "skipped" note when a single head would not fit the budget."""
+    nq, nk = w.N_Q, w.N_K
+    per_head = 36 * nq * nk  # fp32 N_Q x N_K tensors live at the peak (measured ~32 B/pair)
+    if per_head > budget_bytes:
+        return {"skipped": f"one head needs about {per_head / 2**30:.0f} GiB of score matrices"}
+    hc = max(1, min(w.bh, budget_bytes // per_head))
+    qt, kt = d["q_t"].flatten(0, 1), d["k_t"].flatten(0, 1)
+    qs, ks = d["q_s"].flatten(0, 1), d["k_s"].flatten(0, 1)
+    g = d["g"].flatten(0, 1)
+    allowed = None
+    if w.causal:  # bottom-right aligned: key j is visible to query i iff j <= i + N_K - N_Q
+        i = torch.arange(nq, device=dev)[:, None]
+        j = torch.arange(nk, device=dev)[None, :]
+        allowed = j <= i + (nk - nq)
+
+    def chunk(a, b, ev):
+        q_s = qs[a:b].detach().requires_grad_(True)
+        k_s = ks[a:b].detach().requires_grad_(True)
+        ev[0].record(stream)
+        s_t = torch.matmul(qt[a:b], kt[a:b].transpose(-1, -2)).float() * w.scale_T
+        s_s = torch.matmul(q_s, k_s.transpose(-1, -2)).float() * w.scale_S
+        if allowed is not None:
+            s_t = s_t.masked_fill(~allowed, float("-inf"))
+            s_s = s_s.masked_fill(~allowed, float("-inf"))
+        lp_t = torch.log_softmax(s_t, dim=-1)
+        lp_s = torch.log_softmax(s_s, dim=-1)
+        terms = lp_t.exp() * (lp_t - lp_s)
+        if allowed is not None:
+            terms = torch.where(allowed, terms, 0.0)
+        kl = terms.sum(-1)
+        ev[1].record(stream)
+        (kl * g[a:b]).sum().backward()
+        ev[2].record(stream)
+        return kl
+
+    def one_step(evs):
+        diff = 0.0
+        for n, a in enumerate(range(0, w.bh, hc)):
+            b = min(w.bh, a + hc)
+            kl = chunk(a, b, evs[n] if evs else [torch.cuda.Event() for _ in range(3)])
+            if not evs:
+                ref = kl_fused.flatten(0, 1)[a:b]
+                diff = max(diff, (kl.detach() - ref).abs().max().item())
+        return diff
+
+    n_chunks = (w.bh + hc - 1) // hc
+    torch.cuda.synchronize()
+    base = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    diff = one_step(None)  # warm-up, compared with the fused forward
+    torch.cuda.synchronize()
+    peak = torch.cuda.max_memory_allocated(dev) - base
+    f_ms = b_ms = 0.0
+    for _ in range(steps):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_chunks)]
+        one_step(evs)
+        torch.cuda.synchronize()
+        f_ms += sum(e[0].elapsed_time(e[1]) for e in evs)
+        b_ms += sum(e[1].elapsed_time(e[2]) for e in evs)
+    f_ms, b_ms = f_ms / steps, b_ms / steps
+    return {"kind": "torch eager, both softmaxes materialised (bf16 scores, fp32 softmax/KL)",
+            "heads_per_chunk": hc, "fwd_ms": f_ms, "bwd_ms": b_ms,
+            "speedup_fwd": f_ms / fwd_ms, "speedup_bwd": b_ms / bwd_ms,
+            "peak_extra_bytes": peak, "max_abs_kl_diff_vs_fused": diff}
 
 
 def load_traffic(workload: str, which: str):

@@ -117,6 +117,21 @@ def test_negative_and_zero_scales():
     check_full(w, make_inputs(w, seed=6))
 
 
+def test_mixed_sign_upstream_weights():
+    """g of both signs: 64-row query steps whose weights are all >= 0, steps with a negative
+    weight, zero weights and a step of negative weights only, in one call."""
+    w = BASE.with_sizes(B=1, H=2, N_Q=384, N_K=384, causal=True)
+    x = make_inputs(w, seed=12)
+    gen = torch.Generator().manual_seed(13)
+    g = torch.rand(1, 2, 384, generator=gen)
+    g[:, :, 64:128] -= 0.5                      # mixed signs inside a step
+    g[:, :, 200] = -1.0                         # one negative row
+    g[:, :, 256:320] = -torch.rand(1, 2, 64, generator=gen)  # negative only
+    g[:, 1, 320:] = 0.0                         # zero weights
+    x["g"] = g
+    check_full(w, x)
+
+
 def test_large_scores():
     """Peaked distributions (|s| up to ~50): exercises the online max and rescaling."""
     w = BASE.with_sizes(B=1, H=2, N_Q=384, N_K=384, scale_T=0.5, scale_S=0.4, causal=True,
