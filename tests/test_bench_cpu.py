@@ -28,3 +28,44 @@ def test_reference_arm_prints_the_contract_line():
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == "tiny_n256_d64"
+
+
+def test_eager_comparator_computes_the_kl(monkeypatch):
+    """The materialising comparator of bench.py (run here on CPU tensors with the CUDA event
+    and memory calls stubbed) forms the same per-row KL as the oracle, up to the bf16
+    rounding of its scores, for causal and full attention."""
+    import dataclasses
+
+    import torch
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from oracle import oracle_fwd
+    from workloads import WORKLOADS, make_inputs
+
+    class Ev:
+        def __init__(self, **kw):
+            pass
+
+        def record(self, stream=None):
+            pass
+
+        def elapsed_time(self, other):
+            return 1.0
+
+    monkeypatch.setattr(torch.cuda, "Event", Ev)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a: None)
+    monkeypatch.setattr(torch.cuda, "memory_allocated", lambda *a: 0)
+    monkeypatch.setattr(torch.cuda, "reset_peak_memory_stats", lambda *a: None)
+    monkeypatch.setattr(torch.cuda, "max_memory_allocated", lambda *a: 0)
+    for causal in (False, True):
+        w = dataclasses.replace(WORKLOADS["tiny_n256_d64"], causal=causal)
+        x = make_inputs(w)
+        kl, _, _ = oracle_fwd(x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S,
+                              causal)
+        r = bench.run_eager(w, x, kl.float(), torch.device("cpu"), None, 2.0, 4.0, steps=1)
+        assert r["max_abs_kl_diff_vs_fused"] < 0.02, r
+        assert r["speedup_fwd"] == 0.5 and r["speedup_bwd"] == 0.25
+        assert r["heads_per_chunk"] == 1
+    big = dataclasses.replace(WORKLOADS["extreme_b1h8_n65536_d128_causal"])
+    assert "skipped" in bench.run_eager(big, {}, None, torch.device("cpu"), None, 1.0, 1.0)
