@@ -97,6 +97,12 @@ static_assert(!SKL_BWD_SPLIT || kBwdDsWarps * SKL_BWD_RS + 4 * SKL_BWD_RC <=
                                     (kBwdDsWarps + 4) * ((65536 / kBwdThreads) & ~7),
               "register split exceeds the launch's register pool");
 
+// SKL_BWD_LEANMMA (with SKL_BWD_KTMEM): the MMA thread's per-step work reduced to adds of
+// compile-time constants to precomputed descriptor halves and addresses.
+#ifndef SKL_BWD_LEANMMA
+#define SKL_BWD_LEANMMA 1
+#endif
+
 // SKL_BWD_NSTG = 2: two fp32 staging tiles for the dQ reduce-adds, one per step parity (each
 // dS warpgroup drains into its own tile while the previous reduce is still reading the
 // other). The second tile is the shared K tile of the side that is not differentiated: with
@@ -407,6 +413,75 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       if (elect_one()) {
         const uint32_t s_kt = sb + C::OFF_KT, s_ks = sb + C::OFF_KS;
         bool ok = mbar_wait(smem_u32(&bars->k_full), 0);
+    #if SKL_BWD_KTMEM && SKL_BWD_LEANMMA
+        // The dS warps copy the K rows into tensor memory first.
+        if (ok) ok = mbar_wait(smem_u32(&bars->k_tmem), 0);
+        // This thread's instruction stream is on the step's critical path, so every
+        // per-MMA quantity is a precomputed base plus a compile-time constant: descriptor
+        // low halves (one shared high half), TMEM column addresses, stage indices and
+        // phases tracked incrementally (no divisions).
+        const uint32_t hi = sdesc_hi(1024);
+        const uint32_t lq0 = sdesc_lo(sb + C::OFF_Q, 16);  // Q_T of stage 0, K-major
+        const uint32_t lqg0 =                               // Q of the differentiated side
+            sdesc_lo(sb + C::OFF_Q + (TEACHER ? 0 : C::QT_TILE), C::BM * 128);
+        const uint32_t lds_k0 = sdesc_lo(sb + C::OFF_DS, 16);           // dS^T buffer 0 as A
+        const uint32_t lds_n0 = sdesc_lo(sb + C::OFF_DS, C::BN * 128);  // dS^T buffer 0 as B
+        const uint32_t lkg = sdesc_lo(TEACHER ? s_kt : s_ks, C::BN * 128);  // K^T as A
+        constexpr uint32_t kQ16 = C::Q_STAGE >> 4, kDs16 = C::DS_TILE >> 4;
+        const uint32_t t_st = tmem + C::TM_S, t_ss = t_st + 64, t_dk = tmem + C::TM_DK;
+        const uint32_t t_kt = tmem + C::TM_KT, t_ks = tmem + C::TM_KS, t_dq = tmem + C::TM_DQ;
+        int s_st = 0;      // query stage of the next score step
+        uint32_t s_ph = 0;  // and the phase of its q_full barrier
+        auto issue_scores = [&](int s) -> bool {
+          if (!mbar_wait(smem_u32(&bars->q_full[s_st]), s_ph)) return false;
+          if (s > 0 && !mbar_wait(smem_u32(&bars->s_free[(s - 1) & 1]), ((s - 1) >> 1) & 1))
+            return false;
+          tc_fence_after();
+          const uint32_t lq = lq0 + (uint32_t)s_st * kQ16;
+    #pragma unroll
+          for (int kk = 0; kk < DT / 16; ++kk) {
+            const uint32_t qa = ((kk >> 2) * (C::BM * 128) + (kk & 3) * 32) >> 4;
+            umma_bf16_ts_lh(t_st, t_kt + kk * 8, lq + qa, hi, idesc_st, kk > 0);
+          }
+    #pragma unroll
+          for (int kk = 0; kk < DS / 16; ++kk) {
+            const uint32_t qa = (C::QT_TILE + (kk >> 2) * (C::BM * 128) + (kk & 3) * 32) >> 4;
+            umma_bf16_ts_lh(t_ss, t_ks + kk * 8, lq + qa, hi, idesc_ss, kk > 0);
+          }
+          umma_commit(smem_u32(&bars->s_full[s & 1]));
+          if (++s_st == C::NQST) {
+            s_st = 0;
+            s_ph ^= 1u;
+          }
+          return true;
+        };
+        int pst = 0;  // query stage of step p
+        if (ok && n_steps > 0) ok = issue_scores(0);
+        for (int p = 0; ok && p < n_steps; ++p) {
+          const int pb = p & 1;
+          // Scores of step p+1 as soon as the warpgroup of step p has read its scores.
+          if (p + 1 < n_steps && !issue_scores(p + 1)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&bars->ds_full[pb]), (p >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          // dK += dS^T Q : A = dS^T [keys][queries] K-major, B = Q [queries][d] MN-major.
+          const uint32_t la = lds_k0 + (pb ? kDs16 : 0u), lb = lqg0 + (uint32_t)pst * kQ16;
+    #pragma unroll
+          for (int kk = 0; kk < C::BM / 16; ++kk)
+            umma_bf16_ss_lh(t_dk, la + kk * 2, lb + kk * 128, hi, idesc_dk,
+                            (p > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&bars->q_empty[pst]));
+          if (!mbar_wait(smem_u32(&bars->dq_free[pb]), ((p >> 1) & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          // dQ^T = K^T dS^T : A = K [keys][d] MN-major, B = dS^T [keys][queries] MN-major.
+          const uint32_t lbq = lds_n0 + (pb ? kDs16 : 0u), t_dqb = t_dq + (pb ? C::BM : 0);
+    #pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk)
+            umma_bf16_ss_lh(t_dqb, lkg + kk * 128, lbq + kk * 128, hi, idesc_dq, kk > 0);
+          umma_commit(smem_u32(&bars->ds_empty[pb]));
+          umma_commit(smem_u32(&bars->dq_full[pb]));
+          if (++pst == C::NQST) pst = 0;
+        }
+    #else
     #if SKL_BWD_KTMEM
         // The dS warps copy the K rows into tensor memory first.
         if (ok) ok = mbar_wait(smem_u32(&bars->k_tmem), 0);
@@ -509,6 +584,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           umma_commit(smem_u32(&bars->dq_full[pb]));
           if (!early && p + 2 < n_steps && !issue_scores(p + 2)) { ok = false; break; }
         }
+    #endif
         if (!ok) skl_fail_b(abort_flag);
         umma_commit(smem_u32(&bars->dk_full));
         umma_commit(smem_u32(&bars->drain));
