@@ -144,11 +144,32 @@ streamkl_status check_common(const void* q_t, const void* k_t, const void* q_s, 
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Streaming multiprocessors of the current device (queried once per device).
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 // Heads per scheduling group: small enough that a group's tiles stay in the 126 MB L2,
-// large enough to fill the 148 SMs with a heaviest-first mix. Overridable for tuning
+// large enough to fill the SMs with a heaviest-first mix. The base size is raised (up to
+// twice) until one group holds at least a wave of CTAs, so that short sequences, with few
+// CTAs per head, do not leave a tail of heavy causal tiles (measured at N = 4096:
+// +16 % forward, +7 % backward; unchanged for long sequences). Overridable for tuning
 // through STREAMKL_FWD_GROUP / STREAMKL_BWD_GROUP.
-int head_group(const char* env, int fallback, int bh) {
-  int g = fallback;
+int head_group(const char* env, int base, int bh, int units_per_head) {
+  int g = base;
+  if (units_per_head > 0) {
+    const int wave = (sm_count() + units_per_head - 1) / units_per_head;
+    g = wave > g ? (wave < 2 * base ? wave : 2 * base) : g;
+  }
   if (const char* v = std::getenv(env)) {
     const int x = std::atoi(v);
     if (x > 0) g = x;
@@ -224,7 +245,7 @@ streamkl_status fwd_common(const void* q_t, const void* k_t, const void* q_s, co
   a.cT = std::fabs(scale_T) * kLog2e;
   a.cS = std::fabs(scale_S) * kLog2e;
   a.n_ctas_per_bh = (P.N_Q + 255) / 256;
-  a.group = head_group("STREAMKL_FWD_GROUP", 4, bh);
+  a.group = head_group("STREAMKL_FWD_GROUP", 4, bh, a.n_ctas_per_bh);
   a.H = P.H;
   a.gT = P.H / P.H_kv_T;
   a.gS = P.H / P.H_kv_S;
@@ -295,7 +316,7 @@ streamkl_status bwd_common(const void* q_t, const void* k_t, const void* q_s, co
   a.aS = std::fabs(scale_S);
   a.scale_G = TEACHER ? scale_T : scale_S;
   a.n_ktiles = (P.N_K + 127) / 128;
-  a.group = head_group("STREAMKL_BWD_GROUP", 2, bh);
+  a.group = head_group("STREAMKL_BWD_GROUP", 2, bh, a.n_ktiles);
   a.H = P.H;
   a.gT = P.H / P.H_kv_T;
   a.gS = P.H / P.H_kv_S;
