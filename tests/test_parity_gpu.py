@@ -132,6 +132,28 @@ def test_mixed_sign_upstream_weights():
     check_full(w, x)
 
 
+def test_head_group_sizes_cover_every_unit(monkeypatch):
+    """The grid is ordered in groups of heads (a tuning knob with a rule-based default): group
+    sizes that do not divide B*H (the remainder path), a group of one head and a group larger
+    than B*H must each give the same results, against the oracle, as the default."""
+    w = BASE.with_sizes(B=1, H=7, N_Q=700, N_K=700, causal=True)
+    x = make_inputs(w, seed=21)
+    ref = None
+    for fg, bg in ((None, None), ("3", "3"), ("1", "1"), ("5", "2"), ("64", "64")):
+        for key, v in (("STREAMKL_FWD_GROUP", fg), ("STREAMKL_BWD_GROUP", bg)):
+            if v is None:
+                monkeypatch.delenv(key, raising=False)
+            else:
+                monkeypatch.setenv(key, v)
+        got = check_full(w, x) if ref is None else run_gpu(w, x)
+        if ref is None:
+            ref = got
+            continue
+        for k in ("kl", "lse_t", "lse_s", "dk"):  # no cross-CTA accumulation: bitwise equal
+            assert torch.equal(got[k], ref[k]), (fg, bg, k)
+        assert rel_fro(got["dq"], ref["dq"]) <= 1e-6, (fg, bg)  # reduce-add order only
+
+
 def test_large_scores():
     """Peaked distributions (|s| up to ~50): exercises the online max and rescaling."""
     w = BASE.with_sizes(B=1, H=2, N_Q=384, N_K=384, scale_T=0.5, scale_S=0.4, causal=True,
