@@ -309,6 +309,15 @@ def test_full_size_workload(name):
     _sampled(w, dk_heads=1 if w.N_K > 20000 else 2)
 
 
+def test_beyond_config_sizes_one_head_n262144():
+    """One head of 262144 causal queries and keys (four times the longest configured
+    sequence): large TMA row coordinates and 4096-step causal walks. Sampled rows against
+    the oracle (KL, both LSEs, the dQ_S row) and the any-size properties; no dK sample (its
+    reference needs every row's probabilities)."""
+    w = BASE.with_sizes(B=1, H=1, N_Q=262144, N_K=262144, causal=True)
+    _sampled(w, rows_n=64, dk_heads=0)
+
+
 # ------------------------------------------------ packed variable-length sequences
 
 from oracle import oracle_bwd_teacher_varlen, oracle_bwd_varlen, oracle_fwd_varlen  # noqa: E402
