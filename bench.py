@@ -32,6 +32,18 @@ from workloads import (WORKLOADS, flops_bwd, flops_bwd_teacher, flops_fwd, make_
 
 METRIC = "fwd/bwd TFLOP/s and % of B200 bf16 peak at N=16K,d=128; ms per fwd+bwd"
 DEFAULT_WORKLOAD = "long_b1h32_n16384_d128_causal"
+FWD_FMA_EXP_SHARE = 1.0 / 16.0  # share of the forward's exponentials computed on the FMA pipe
+
+
+def clocks_mhz_or(clk, default=1965.0):
+    """Median SM clock sampled during the timed region (MHz), else the B200's maximum."""
+    try:
+        v = float(clk["sm_mhz"]) if clk else 0.0
+    except (KeyError, TypeError, ValueError):
+        v = 0.0
+    return v if v > 0 else default
+
+
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -324,6 +336,19 @@ def main():
             "peak_kind": f"{peak_kind} bf16 dense, burst (short timed region at full clocks)",
             "frac_of_sustained_peak": achieved / peak_sus}
 
+    # Second roofline of the forward: its statistics warps are bound by the exponential unit
+    # (MUFU), two exponentials per (row, key) pair, of which the kernel sends 1/16 to the
+    # FMA pipe as a polynomial. Peak: 16 ex2 per clock per SM at the sampled SM clock.
+    pairs = ff / (2.0 * (w.d_T + w.d_S))
+    mufu_ex2 = 2.0 * pairs * (1.0 - FWD_FMA_EXP_SHARE)
+    sm_hz = (clocks_mhz_or(clk) * 1e6)
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    mufu_peak = 16.0 * n_sm * sm_hz
+    fwd_mufu = {"bound": "mufu", "achieved": mufu_ex2 / (fwd_ms * 1e-3) / 1e12,
+                "peak": mufu_peak / 1e12, "unit": "Tex2/s",
+                "frac": (mufu_ex2 / (fwd_ms * 1e-3)) / mufu_peak,
+                "peak_kind": f"16 ex2/clock/SM x {n_sm} SMs x {sm_hz / 1e6:.0f} MHz (sampled)"}
+
     # Trainable-teacher backward (streamkl_bwd_teacher), timed on its own: not part of the
     # step (the teacher is frozen in the measured workload), reported beside it.
     dq_t = torch.empty(B, H, nq, w.d_T, device=dev)
@@ -394,7 +419,8 @@ def main():
                "fwd_frac_peak": fwd_tf / peak_burst, "bwd_frac_peak": bwd_tf / peak_burst,
                "fwd_frac_sustained_peak": fwd_tf / peak_sus,
                "bwd_frac_sustained_peak": bwd_tf / peak_sus,
-               "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+               "roofline": roof, "fwd_mufu": fwd_mufu, "cpu_baseline": cpu, "e2e": e2e,
+               "clocks": clk,
                "gqa": gqa, "varlen": varlen, "context_parallel": cp, "eager_baseline": eager,
                "bwd_teacher_ms": bwd_t_ms,
                "bwd_teacher_tflops": flops_bwd_teacher(w) / (bwd_t_ms * 1e-3) / 1e12,
