@@ -69,3 +69,16 @@ def test_eager_comparator_computes_the_kl(monkeypatch):
         assert r["heads_per_chunk"] == 1
     big = dataclasses.replace(WORKLOADS["extreme_b1h8_n65536_d128_causal"])
     assert "skipped" in bench.run_eager(big, {}, None, torch.device("cpu"), None, 1.0, 1.0)
+
+
+def test_bench_helpers():
+    """The config's L2 note and the clock used for the exponential-unit roofline."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from workloads import WORKLOADS
+
+    assert "fit in the 126 MB L2" in bench.l2_note(WORKLOADS["tiny_n256_d64"])
+    assert "537 MB" in bench.l2_note(WORKLOADS["long_b1h32_n16384_d128_causal"])
+    assert bench.clocks_mhz_or(None) == 1965.0
+    assert bench.clocks_mhz_or({"sm_mhz": 1804.0}) == 1804.0
+    assert bench.clocks_mhz_or({"sm_mhz": None}) == 1965.0
