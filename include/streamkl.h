@@ -37,6 +37,12 @@
  *   streamkl_device_status(); it never traps.
  * - Rows with an empty J(i) (only causal with N_Q > N_K) get KL = 0, LSE = -inf and a
  *   zero gradient. KL is reported unclamped (rounding can make it slightly negative).
+ * - Scheduling: CTAs are ordered in groups of heads (L2 locality, heaviest causal tiles
+ *   first). The environment variables STREAMKL_FWD_GROUP and STREAMKL_BWD_GROUP (positive
+ *   integers, read at every call) override the group sizes, which otherwise follow a rule
+ *   (4 heads forward, 2 backward, raised up to twice that until a group holds one wave of
+ *   CTAs). They change only the speed: results are the same for any group size, except
+ *   that dQ is summed in a different order (fp32 reduce-adds across CTAs).
  */
 #ifndef STREAMKL_H
 #define STREAMKL_H
