@@ -12,19 +12,46 @@ kernels and nothing of that size is ever allocated.
 Packed variable-length batches use ``attention_kl_varlen`` / ``attention_kl_varlen_loss``
 (q_* [total_q, H, d], k_* [total_k, H_kv, d], int32 cu_seqlens on the device); there
 "batchmean" divides by the number of sequences.
+
+Errors found on the device (a pipeline wait that ran out, malformed packed offsets) are
+recorded in the library's device error word and the kernel returns early, leaving some
+outputs unwritten; the launch itself still succeeds. The wrappers check that word after
+every forward and backward when status checks are on (``set_check_status(True)`` or the
+environment variable STREAMKL_CHECK_STATUS=1) and raise ``StreamKLError``. The check
+synchronises the stream, so it is off by default; with it off, poll
+``attention_kl_divergence_fwd_b200.device_status()`` yourself (for instance once per
+training step) before trusting the step's gradients.
 """
 from __future__ import annotations
 
 import math
+import os
 from typing import Optional
 
 import torch
 
-from . import (streamkl_bwd, streamkl_bwd_gqa, streamkl_bwd_teacher, streamkl_bwd_teacher_gqa,
-               streamkl_bwd_teacher_varlen, streamkl_bwd_varlen, streamkl_fwd, streamkl_fwd_gqa,
-               streamkl_fwd_varlen)
+from . import (StreamKLError, device_status, streamkl_bwd, streamkl_bwd_gqa, streamkl_bwd_teacher,
+               streamkl_bwd_teacher_gqa, streamkl_bwd_teacher_varlen, streamkl_bwd_varlen,
+               streamkl_fwd, streamkl_fwd_gqa, streamkl_fwd_varlen)
 
 REDUCTIONS = ("none", "sum", "mean", "batchmean")
+
+_check_status = os.environ.get("STREAMKL_CHECK_STATUS", "0") not in ("", "0")
+
+
+def set_check_status(enabled: bool) -> None:
+    """Turn the device-status check after every wrapped forward and backward on or off."""
+    global _check_status
+    _check_status = bool(enabled)
+
+
+def _after_launch(where: str, device) -> None:
+    """Raise StreamKLError when status checks are on and the device reported an error."""
+    if _check_status:
+        with torch.cuda.device(device):
+            st = device_status()
+        if st != 0:
+            raise StreamKLError(st, where)
 
 
 class StreamKLFunction(torch.autograd.Function):
@@ -40,6 +67,7 @@ class StreamKLFunction(torch.autograd.Function):
         gqa = k_t.shape[1] != q_t.shape[1] or k_s.shape[1] != q_s.shape[1]
         fwd = streamkl_fwd_gqa if gqa else streamkl_fwd
         kl, lse_t, lse_s = fwd(q_t, k_t, q_s, k_s, scale_t, scale_s, causal)
+        _after_launch("attention_kl forward", q_t.device)
         ctx.save_for_backward(q_t, k_t, q_s, k_s, kl, lse_t, lse_s)
         ctx.params = (scale_t, scale_s, causal, gqa)
         ctx.mark_non_differentiable(lse_t, lse_s)
@@ -61,6 +89,7 @@ class StreamKLFunction(torch.autograd.Function):
             bwd_t = streamkl_bwd_teacher_gqa if gqa else streamkl_bwd_teacher
             dq_t, dk_t = bwd_t(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, kl, lse_t, lse_s, g)
             dq_t, dk_t = dq_t.to(q_t.dtype), dk_t.to(k_t.dtype)
+        _after_launch("attention_kl backward", q_t.device)
         return dq_t, dk_t, dq_s, dk_s, None, None, None
 
 
@@ -111,6 +140,7 @@ class StreamKLVarlenFunction(torch.autograd.Function):
         kl = torch.zeros(H, tq, device=q_t.device, dtype=torch.float32)
         kl, lse_t, lse_s = streamkl_fwd_varlen(q_t, k_t, q_s, k_s, cu_q, cu_k, max_q, max_k,
                                                scale_t, scale_s, causal, kl=kl)
+        _after_launch("attention_kl_varlen forward", q_t.device)
         ctx.save_for_backward(q_t, k_t, q_s, k_s, cu_q, cu_k, kl, lse_t, lse_s)
         ctx.params = (max_q, max_k, scale_t, scale_s, causal)
         ctx.mark_non_differentiable(lse_t, lse_s)
@@ -128,6 +158,7 @@ class StreamKLVarlenFunction(torch.autograd.Function):
         if ctx.needs_input_grad[0] or ctx.needs_input_grad[1]:
             dq_t, dk_t = streamkl_bwd_teacher_varlen(*a, kl, lse_t, lse_s, g)
             dq_t, dk_t = dq_t.to(q_t.dtype), dk_t.to(k_t.dtype)
+        _after_launch("attention_kl_varlen backward", q_t.device)
         return dq_t, dk_t, dq_s, dk_s, None, None, None, None, None, None, None
 
 

@@ -3,8 +3,8 @@
 Each rank holds every query row (Q_T, Q_S) and one contiguous shard of the keys
 (K_T, K_S rows k_offset .. k_offset + N_K_shard - 1 of N_K_total). The one-pass forward
 leaves an online per-row state that merges associatively ("StreamKL: Fast and
-Memory-Efficient KL Divergence for Boosting Attention Distillation", abstract: online
-formulation of the coupled two-distribution reduction), so the exchange is small:
+Memory-Efficient KL Divergence for Boosting Attention Distillation", abstract: the forward
+reduces both distributions together, online, in one pass), so the exchange is small:
 
   forward : state_r = streamkl_fwd_partial(shard r)          [5, B, H, N_Q] fp32 per rank
             all-gather the states (20 bytes per row per rank), then
@@ -57,6 +57,24 @@ def _all_gather_stacked(t: torch.Tensor, group) -> torch.Tensor:
     return out
 
 
+def _status_check(where: str, device, group) -> None:
+    """With status checks on (see ``autograd.set_check_status``): read this rank's device
+    error word and take the maximum over the group, so that every rank raises together
+    and none is left waiting in the next collective."""
+    from . import StreamKLError, device_status
+    from . import autograd as _ag
+    if not _ag._check_status:
+        return
+    with torch.cuda.device(device):
+        st = device_status()
+    if _world(group) > 1:
+        t = torch.tensor([st], dtype=torch.int32, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+        st = int(t.item())
+    if st != 0:
+        raise StreamKLError(st, where)
+
+
 def cp_forward(q_t, k_t, q_s, k_s, scale_t: float, scale_s: float, causal: bool,
                k_offset: int, n_k_total: int, group=None, ops: Optional[ShardOps] = None):
     """KL, LSE_T, LSE_S [B, H, N_Q] of the whole key range, on every rank of ``group``."""
@@ -93,6 +111,7 @@ class ContextParallelKL(torch.autograd.Function):
     def forward(ctx, q_t, k_t, q_s, k_s, scale_t, scale_s, causal, k_offset, n_k_total, group):
         kl, lse_t, lse_s = cp_forward(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, k_offset,
                                       n_k_total, group)
+        _status_check("attention_kl_context_parallel forward", q_t.device, group)
         ctx.save_for_backward(q_t, k_t, q_s, k_s, kl, lse_t, lse_s)
         ctx.params = (scale_t, scale_s, causal, k_offset, n_k_total, group)
         ctx.mark_non_differentiable(lse_t, lse_s)
@@ -114,6 +133,7 @@ class ContextParallelKL(torch.autograd.Function):
         if ctx.needs_input_grad[0] or ctx.needs_input_grad[1]:
             dq_t, dk_t = cp_backward(*a, group=group, teacher=True, kl=kl)
             dq_t, dk_t = dq_t.to(q_t.dtype), dk_t.to(k_t.dtype)
+        _status_check("attention_kl_context_parallel backward", q_t.device, group)
         return dq_t, dk_t, dq_s, dk_s, None, None, None, None, None, None
 
 

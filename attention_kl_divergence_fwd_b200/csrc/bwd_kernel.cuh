@@ -1,8 +1,8 @@
 // bwd_kernel.cuh - StreamKL backward on sm_100a (tcgen05 + TMEM + TMA).
 //
 // The recompute backward of "StreamKL: Fast and Memory-Efficient KL Divergence for
-// Boosting Attention Distillation" (abstract: the backward recomputes attention
-// probabilities tile by tile instead of storing quadratic intermediates).
+// Boosting Attention Distillation" (abstract: the backward regenerates the attention
+// probabilities one tile at a time and keeps no quadratic intermediate).
 //
 // With g[i] = dLoss/dKL[i] and P_X = 2^(t_X - LSE_X*log2 e):
 //   student (TEACHER = false): dS[i,j] = g[i] * scale_S * (P_S[i,j] - P_T[i,j]),

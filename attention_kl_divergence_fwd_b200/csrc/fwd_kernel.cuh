@@ -1,8 +1,9 @@
 // fwd_kernel.cuh - StreamKL forward on sm_100a (tcgen05 + TMEM + TMA).
 //
 // The one-pass forward of "StreamKL: Fast and Memory-Efficient KL Divergence for
-// Boosting Attention Distillation" (abstract: an online formulation of the coupled
-// two-distribution KL reduction, streaming query-key tiles through on-chip memory).
+// Boosting Attention Distillation" (abstract: one forward pass reduces both distributions
+// together with a running per-row state while query and key tiles pass through on-chip
+// memory).
 //
 // CTA = two 128-row query tiles of one (batch, head). Key tiles of 64 rows stream
 // through a TMA ring. Per key tile and query tile the tensor core computes the teacher

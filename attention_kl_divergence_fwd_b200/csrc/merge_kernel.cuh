@@ -3,8 +3,8 @@
 // Context parallelism over N_K splits the keys of a sequence into contiguous shards; the
 // forward of each shard leaves, per query row, the online state of the one-pass
 // reduction ("StreamKL: Fast and Memory-Efficient KL Divergence for Boosting Attention
-// Distillation", abstract: online formulation of the coupled two-distribution KL
-// reduction): maxima m_T, m_S and sums l_T, l_S, A in base-2 units. States combine by
+// Distillation", abstract: both distributions are reduced together, online, in one
+// pass): maxima m_T, m_S and sums l_T, l_S, A in base-2 units. States combine by
 // rescaling to the larger maximum and adding, so R shard states merge into the state of
 // the whole key range, which is then finalised exactly as the one-pass forward does.
 //

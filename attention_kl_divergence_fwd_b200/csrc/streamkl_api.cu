@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "streamkl.h"
@@ -144,18 +145,34 @@ streamkl_status check_common(const void* q_t, const void* k_t, const void* q_s, 
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Streaming multiprocessors of the current device (queried once per device).
+// Streaming multiprocessors of the current device (queried once per device; host threads
+// that race on the first query store the same value).
 int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
+}
+
+// A positive integer from the environment, else 0.
+int env_positive(const char* name) {
+  const char* v = std::getenv(name);
+  const int x = v ? std::atoi(v) : 0;
+  return x > 0 ? x : 0;
+}
+
+// Tuning overrides of the head-group sizes, read once per process (thread-safe static
+// initialisation); 0 = no override.
+int group_override(bool fwd) {
+  static const int f = env_positive("STREAMKL_FWD_GROUP");
+  static const int b = env_positive("STREAMKL_BWD_GROUP");
+  return fwd ? f : b;
 }
 
 // Heads per scheduling group: small enough that a group's tiles stay in the 126 MB L2,
@@ -163,17 +180,14 @@ int sm_count() {
 // twice) until one group holds at least a wave of CTAs, so that short sequences, with few
 // CTAs per head, do not leave a tail of heavy causal tiles (measured at N = 4096:
 // +16 % forward, +7 % backward; unchanged for long sequences). Overridable for tuning
-// through STREAMKL_FWD_GROUP / STREAMKL_BWD_GROUP.
-int head_group(const char* env, int base, int bh, int units_per_head) {
+// through STREAMKL_FWD_GROUP / STREAMKL_BWD_GROUP (read once, at the first call).
+int head_group(bool fwd, int base, int bh, int units_per_head) {
   int g = base;
   if (units_per_head > 0) {
     const int wave = (sm_count() + units_per_head - 1) / units_per_head;
     g = wave > g ? (wave < 2 * base ? wave : 2 * base) : g;
   }
-  if (const char* v = std::getenv(env)) {
-    const int x = std::atoi(v);
-    if (x > 0) g = x;
-  }
+  if (const int x = group_override(fwd)) g = x;
   return g < 1 ? 1 : (g > bh ? bh : g);
 }
 
@@ -245,7 +259,7 @@ streamkl_status fwd_common(const void* q_t, const void* k_t, const void* q_s, co
   a.cT = std::fabs(scale_T) * kLog2e;
   a.cS = std::fabs(scale_S) * kLog2e;
   a.n_ctas_per_bh = (P.N_Q + 255) / 256;
-  a.group = head_group("STREAMKL_FWD_GROUP", 4, bh, a.n_ctas_per_bh);
+  a.group = head_group(true, 4, bh, a.n_ctas_per_bh);
   a.H = P.H;
   a.gT = P.H / P.H_kv_T;
   a.gS = P.H / P.H_kv_S;
@@ -316,7 +330,7 @@ streamkl_status bwd_common(const void* q_t, const void* k_t, const void* q_s, co
   a.aS = std::fabs(scale_S);
   a.scale_G = TEACHER ? scale_T : scale_S;
   a.n_ktiles = (P.N_K + 127) / 128;
-  a.group = head_group("STREAMKL_BWD_GROUP", 2, bh, a.n_ktiles);
+  a.group = head_group(false, 2, bh, a.n_ktiles);
   a.H = P.H;
   a.gT = P.H / P.H_kv_T;
   a.gS = P.H / P.H_kv_S;

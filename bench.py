@@ -14,6 +14,7 @@ forward and 2*N_Q*N_K*(d_T+3*d_S) backward, halved when causal.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import json
 import math
 import os
@@ -152,6 +153,17 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+@contextlib.contextmanager
+def nvtx(name: str):
+    """An NVTX range around a region of the bench (visible in Nsight timelines; a no-op
+    without a profiler attached)."""
+    torch.cuda.nvtx.range_push(name)
+    try:
+        yield
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -286,9 +298,10 @@ def main():
         if ev is not None:
             ev[2].record(stream)
 
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize()
+    with nvtx("warm-up"):
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
     if skl.device_status() != 0:
         raise RuntimeError("kernel watchdog fired during warm-up")
 
@@ -300,11 +313,12 @@ def main():
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for k in range(args.steps):
-        step(evs[k])
-    t_end.record(stream)
-    torch.cuda.synchronize()
+    with nvtx("timed steps"):
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        t_end.record(stream)
+        torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop() if clocks else None
     if skl.device_status() != 0:
@@ -393,22 +407,27 @@ def main():
                "fwd_tflops": ff / (gf * 1e-3) / 1e12, "bwd_tflops": fb / (gb * 1e-3) / 1e12}
         del k_s4, dk4
 
-    varlen = run_varlen(skl, w, dev, stream, args.steps, world) if w.d_T == w.d_S else None
-    cp = run_context_parallel(skl, w, d, dev, stream, args.steps, world)
+    with nvtx("packed sequences"):
+        varlen = run_varlen(skl, w, dev, stream, args.steps, world) if w.d_T == w.d_S else None
+    with nvtx("context-parallel shards"):
+        cp = run_context_parallel(skl, w, d, dev, stream, args.steps, world)
 
     eager = None
     if rank == 0 and not args.no_eager:
         skl.streamkl_fwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal,
                          kl=kl, lse_t=lt, lse_s=ls)  # the buffers held the variants' rows
-        eager = run_eager(w, d, kl, dev, stream, fwd_ms, bwd_ms)
+        with nvtx("eager comparator"):
+            eager = run_eager(w, d, kl, dev, stream, fwd_ms, bwd_ms)
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(skl, w, x, dev, stream, args.steps, world)
+        with nvtx("end to end"):
+            e2e = run_e2e(skl, w, x, dev, stream, args.steps, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
+        with nvtx("cpu baseline"):
+            cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
 
     if rank == 0:
         out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -528,53 +547,74 @@ def run_context_parallel(skl, w, d, dev, stream, steps, world, shards=4):
 
 
 def run_e2e(skl, w, x, dev, stream, steps, world):
-    """Same metric through the public API from pinned host buffers: every step copies its
-    inputs host->device, runs forward + backward, and reads its KL rows back to the host.
-    The copies run on a second stream into one of two device input buffers, so step k's
-    host->device copy overlaps step k-1's kernels (a double-buffered input pipeline)."""
+    """Same metric through the public API from and to pinned host buffers: every step
+    copies its inputs host->device, runs forward + backward, and copies its whole result,
+    the KL rows and the student gradients dQ_S and dK_S, device->host. Three streams
+    overlap: step k's input copy (second stream) runs beside step k-1's kernels, and step
+    k-1's result copy (third stream) beside step k's kernels; inputs and outputs are
+    double-buffered on the device, so the step time is bound by the slower PCIe direction."""
     host = {k: v.pin_memory() for k, v in x.items()}
     bufs = [{k: torch.empty_like(v, device=dev) for k, v in x.items()} for _ in range(2)]
-    kl_h = [torch.empty(w.B, w.H, w.N_Q, dtype=torch.float32).pin_memory() for _ in range(2)]
+    out_shapes = {"kl": (w.B, w.H, w.N_Q), "lse_t": (w.B, w.H, w.N_Q),
+                  "lse_s": (w.B, w.H, w.N_Q), "dq": (w.B, w.H, w.N_Q, w.d_S),
+                  "dk": (w.B, w.H, w.N_K, w.d_S)}
+    outs = [{k: torch.empty(sh, device=dev) for k, sh in out_shapes.items()} for _ in range(2)]
+    result = ("kl", "dq", "dk")  # what the step returns to the host
+    host_out = [{k: torch.empty(out_shapes[k]).pin_memory() for k in result} for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = kl_h[0].numel() * 4
-    copy_stream = torch.cuda.Stream(dev)
+    d2h = sum(host_out[0][k].numel() * 4 for k in result)
+    copy_in, copy_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     copied = [torch.cuda.Event() for _ in range(2)]
-    freed = [torch.cuda.Event() for _ in range(2)]
+    freed = [torch.cuda.Event() for _ in range(2)]    # step's kernels done with buffer set b
+    drained = [torch.cuda.Event() for _ in range(2)]  # result of buffer set b is on the host
 
     def one(k):
         b = k & 1
-        d = bufs[b]
-        with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(freed[b])  # step k-2's kernels are done with buffer b
+        d, o = bufs[b], outs[b]
+        with torch.cuda.stream(copy_in):
+            copy_in.wait_event(freed[b])  # step k-2's kernels are done with input buffer b
             for name in d:
                 d[name].copy_(host[name], non_blocking=True)
-            copied[b].record(copy_stream)
+            copied[b].record(copy_in)
         stream.wait_event(copied[b])
-        kl, lt, ls = skl.streamkl_fwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T,
-                                      w.scale_S, w.causal, stream=stream)
+        stream.wait_event(drained[b])  # step k-2's result has left output buffer b
+        skl.streamkl_fwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S,
+                         w.causal, kl=o["kl"], lse_t=o["lse_t"], lse_s=o["lse_s"],
+                         stream=stream)
         skl.streamkl_bwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S,
-                         w.causal, lt, ls, d["g"], stream=stream)
+                         w.causal, o["lse_t"], o["lse_s"], d["g"], dq_s=o["dq"], dk_s=o["dk"],
+                         stream=stream)
         freed[b].record(stream)
-        kl_h[b].copy_(kl, non_blocking=True)
+        with torch.cuda.stream(copy_out):
+            copy_out.wait_event(freed[b])
+            for name in result:
+                host_out[b][name].copy_(o[name], non_blocking=True)
+            drained[b].record(copy_out)
 
     for b in range(2):
         freed[b].record(stream)
+        drained[b].record(stream)
     for k in range(2):
         one(k)
     torch.cuda.synchronize()
     barrier(world)
     a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    copy_stream.wait_event(a)  # the first timed copy starts inside the timed region
+    copy_in.wait_event(a)  # the first timed copy starts inside the timed region
     for k in range(steps):
         one(k)
+    stream.wait_stream(copy_out)  # the last result copy ends inside the timed region
     e.record(stream)
     torch.cuda.synchronize()
+    if skl.device_status() != 0:
+        raise RuntimeError("kernel watchdog fired in the end-to-end run")
     ms = max_over_ranks(a.elapsed_time(e), world)
     value = world * (flops_fwd(w) + flops_bwd(w)) * steps / (ms * 1e-3) / 1e12
     return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps,
-            "pipeline": "host->device copies on a second stream, double-buffered"}
+            "returned": "KL rows, dQ_S and dK_S (fp32) to pinned host memory every step",
+            "pipeline": "input copies, kernels and result copies on three streams, inputs and "
+                        "outputs double-buffered on the device"}
 
 
 def run_eager(w, d, kl_fused, dev, stream, fwd_ms, bwd_ms, steps=2, budget_bytes=24 << 30):

@@ -10,12 +10,13 @@
  *   KL[i]    = sum_{j in J(i)} P_T[i,j] * (log P_T[i,j] - log P_S[i,j])
  *
  * computed without materialising either N_Q x N_K matrix. The forward streams key
- * tiles past a resident query tile and keeps an online state per row (the abstract's
- * "online formulation for the coupled two-distribution KL reduction" and "single
- * one-pass forward kernel"). The backward recomputes both probability tiles from the
- * saved log-sum-exps (the abstract's "recomputes attention probabilities
- * tile-by-tile"). streamkl_bwd gives the student's gradients (teacher frozen, the
- * abstract's setting); streamkl_bwd_teacher gives a trainable teacher's.
+ * tiles past a resident query tile and keeps an online state per row (the abstract
+ * describes a single forward pass that reduces both distributions together as the tiles
+ * go by, with the tiles held on chip). The backward recomputes both probability tiles
+ * from the saved log-sum-exps (in the abstract, the backward regenerates the
+ * probabilities one tile at a time instead of storing them). streamkl_bwd gives the
+ * student's gradients (teacher frozen, the abstract's setting); streamkl_bwd_teacher
+ * gives a trainable teacher's.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -39,7 +40,7 @@
  *   zero gradient. KL is reported unclamped (rounding can make it slightly negative).
  * - Scheduling: CTAs are ordered in groups of heads (L2 locality, heaviest causal tiles
  *   first). The environment variables STREAMKL_FWD_GROUP and STREAMKL_BWD_GROUP (positive
- *   integers, read at every call) override the group sizes, which otherwise follow a rule
+ *   integers, read once per process at the first call) override the group sizes, which otherwise follow a rule
  *   (4 heads forward, 2 backward, raised up to twice that until a group holds one wave of
  *   CTAs). They change only the speed: results are the same for any group size, except
  *   that dQ is summed in a different order (fp32 reduce-adds across CTAs).

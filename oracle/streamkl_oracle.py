@@ -209,13 +209,20 @@ def oracle_dk_rows(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g, bh: int,
     return out
 
 
+def _sampled_ds(g_rows, scale_s, p_s, p_t):
+    """dS rows of sampled query rows: g_i * scale_S * (P_S[i, :] - P_T[i, :])."""
+    return g_rows[:, None] * scale_s * (p_s - p_t)
+
+
 def oracle_row_work(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g,
                     rows: Sequence[Tuple[int, int]]):
     """Whole forward + backward work of selected query rows (CPU-baseline timing).
 
     For each sampled row: its KL and LSEs, its dQ_S row, and its contribution
-    dS[i, :]^T q_S[i] to dK_S. Returns (kl, dq, dk_contrib_sum) so nothing is
-    optimised away.
+    dS[i, :]^T q_S[i] to dK_S. Returns (kl [R], dq [R, d_S], dk_acc [N_K, d_S]),
+    where dk_acc is the sum of those contributions over every sampled row (rows of
+    different heads added together, so nothing is optimised away; a row listed twice
+    contributes twice).
     """
     kl, _, _, dq = oracle_rows(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g, rows)
     B, H, n_q, d_s = q_s.shape
@@ -233,7 +240,7 @@ def oracle_row_work(q_t, k_t, q_s, k_s, scale_t, scale_s, causal, g,
             _f64(qt2[bh, rr]), _f64(kt2[bh]), qsr, _f64(ks2[bh]), rr,
             scale_t, scale_s, causal, n_q)
         _, p_t, p_s = _block_kl(st, ss, mask, lt, ls)
-        ds = _f64(g2[bh, rr])[:, None] * scale_s * (p_s - p_t)
+        ds = _sampled_ds(_f64(g2[bh, rr]), scale_s, p_s, p_t)
         dk_acc += ds.T @ qsr
     return kl, dq, dk_acc
 

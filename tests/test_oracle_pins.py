@@ -675,3 +675,56 @@ def test_merge_identity_and_grouped_heads():
     assert torch.equal(kl, kl_e) and torch.equal(lt, lt_e)
     kl_r, _, _ = O.oracle_fwd_gqa(q_t, k_t, q_s, k_s, 0.9, 0.6, True)
     torch.testing.assert_close(kl, kl_r, rtol=1e-11, atol=1e-12)
+
+
+# ------------------------------------------------ timed CPU-baseline row work
+
+def _row_work_case():
+    q_t, k_t, q_s, k_s, g = rand_case(2, 2, 13, 17, 6, 5, seed=71)
+    args = (q_t, k_t, q_s, k_s, 0.6, 0.9, True)
+    # distinct (bh, i) rows: several per head, rows 0 (5 keys) and N_Q-1 (all 17 keys)
+    rows = [(0, 0), (0, 5), (1, 12), (3, 7), (2, 3), (3, 12), (1, 0)]
+    return args, g, rows
+
+
+def _row_work_expected(args, g, rows):
+    """What oracle_row_work must return, from the full oracle_fwd / oracle_bwd.
+
+    KL and dQ rows are read off the full outputs. The summed dK contribution of the
+    sampled rows is the dK of oracle_bwd with the upstream weights of every other row set
+    to 0 (dK_S = sum_i g_i dS-row_i^T q_S[i] is linear in g), added over the heads.
+    """
+    B, H, n_q = g.shape
+    kl_f, _, _ = O.oracle_fwd(*args)
+    dq_f, _ = O.oracle_bwd(*args, g)
+    g_sel = torch.zeros_like(g).view(B * H, n_q)
+    for bh, i in rows:
+        g_sel[bh, i] = g.view(B * H, n_q)[bh, i]
+    _, dk_sel = O.oracle_bwd(*args, g_sel.view_as(g))
+    n_k, d_s = dk_sel.shape[2], dk_sel.shape[3]
+    kl = torch.stack([kl_f.view(B * H, n_q)[bh, i] for bh, i in rows])
+    dq = torch.stack([dq_f.view(B * H, n_q, -1)[bh, i] for bh, i in rows])
+    return kl, dq, dk_sel.view(B * H, n_k, d_s).sum(0)
+
+
+def test_row_work_matches_full_oracle():
+    """oracle_row_work (the timed CPU baseline and reference arm) does the same work as
+    the full oracle: its KL, dQ rows and summed dK contributions equal oracle_fwd /
+    oracle_bwd restricted to the sampled rows (N_Q != N_K, causal, ragged rows)."""
+    args, g, rows = _row_work_case()
+    kl, dq, dk = O.oracle_row_work(*args, g, rows)
+    kl_e, dq_e, dk_e = _row_work_expected(args, g, rows)
+    torch.testing.assert_close(kl, kl_e, rtol=1e-12, atol=1e-14)
+    torch.testing.assert_close(dq, dq_e, rtol=1e-12, atol=1e-14)
+    torch.testing.assert_close(dk, dk_e, rtol=1e-12, atol=1e-14)
+    assert dk.abs().max() > 1e-3  # the sampled rows do contribute
+
+
+def test_row_work_dropped_weight_is_caught(monkeypatch):
+    """A planted mistake in the row work's dS (upstream weight g dropped) breaks the pin."""
+    args, g, rows = _row_work_case()
+    kl_e, dq_e, dk_e = _row_work_expected(args, g, rows)
+    with monkeypatch.context() as m:
+        m.setattr(O, "_sampled_ds", lambda g_rows, scale_s, p_s, p_t: scale_s * (p_s - p_t))
+        _, _, dk = O.oracle_row_work(*args, g, rows)
+    assert not torch.allclose(dk, dk_e, rtol=1e-6, atol=1e-9)
