@@ -260,6 +260,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-eager", action="store_true",
                     help="skip the PyTorch eager materialising comparator")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="time only the step (skip the teacher, grouped-query, packed and "
+                         "context-parallel legs), e.g. for a small profiler capture")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="host time of the cpu_baseline leg of this arm")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
@@ -363,6 +366,57 @@ def main():
                 "frac": (mufu_ex2 / (fwd_ms * 1e-3)) / mufu_peak,
                 "peak_kind": f"16 ex2/clock/SM x {n_sm} SMs x {sm_hz / 1e6:.0f} MHz (sampled)"}
 
+    bwd_t_ms, gqa, varlen, cp = None, None, None, None
+    if not args.no_variants:
+        bwd_t_ms, gqa, varlen, cp = run_variants(skl, args, w, d, dev, stream, world, kl, lt,
+                                                 ls, dq)
+
+    eager = None
+    if rank == 0 and not args.no_eager:
+        skl.streamkl_fwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal,
+                         kl=kl, lse_t=lt, lse_s=ls)  # the buffers held the variants' rows
+        with nvtx("eager comparator"):
+            eager = run_eager(w, d, kl, dev, stream, fwd_ms, bwd_ms)
+
+    e2e = None
+    if not args.no_e2e:
+        with nvtx("end to end"):
+            e2e = run_e2e(skl, w, x, dev, stream, args.steps, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        with nvtx("cpu baseline"):
+            cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+               "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+               "dtype": "bf16", "data": "synthetic", "config": config_of(w, world),
+               "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+               "fwd_frac_peak": fwd_tf / peak_burst, "bwd_frac_peak": bwd_tf / peak_burst,
+               "fwd_frac_sustained_peak": fwd_tf / peak_sus,
+               "bwd_frac_sustained_peak": bwd_tf / peak_sus,
+               "roofline": roof, "fwd_mufu": fwd_mufu, "cpu_baseline": cpu, "e2e": e2e,
+               "clocks": clk,
+               "gqa": gqa, "varlen": varlen, "context_parallel": cp, "eager_baseline": eager,
+               "bwd_teacher_ms": bwd_t_ms,
+               "bwd_teacher_tflops": (flops_bwd_teacher(w) / (bwd_t_ms * 1e-3) / 1e12
+                                      if bwd_t_ms else None),
+               "gpu_launches": 2 * args.steps,
+               "extra_hbm_bytes": 3 * 4 * w.bh * w.N_Q,
+               "impl": "ours"}
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_variants(skl, args, w, d, dev, stream, world, kl, lt, ls, dq):
+    """The legs timed beside the step: trainable-teacher backward, grouped-query variant,
+    packed variable-length batch, context-parallel key shards."""
+    B, H, nq, nk = w.B, w.H, w.N_Q, w.N_K
+    ff, fb = flops_fwd(w), flops_bwd(w)
     # Trainable-teacher backward (streamkl_bwd_teacher), timed on its own: not part of the
     # step (the teacher is frozen in the measured workload), reported beside it.
     dq_t = torch.empty(B, H, nq, w.d_T, device=dev)
@@ -411,45 +465,7 @@ def main():
         varlen = run_varlen(skl, w, dev, stream, args.steps, world) if w.d_T == w.d_S else None
     with nvtx("context-parallel shards"):
         cp = run_context_parallel(skl, w, d, dev, stream, args.steps, world)
-
-    eager = None
-    if rank == 0 and not args.no_eager:
-        skl.streamkl_fwd(d["q_t"], d["k_t"], d["q_s"], d["k_s"], w.scale_T, w.scale_S, w.causal,
-                         kl=kl, lse_t=lt, lse_s=ls)  # the buffers held the variants' rows
-        with nvtx("eager comparator"):
-            eager = run_eager(w, d, kl, dev, stream, fwd_ms, bwd_ms)
-
-    e2e = None
-    if not args.no_e2e:
-        with nvtx("end to end"):
-            e2e = run_e2e(skl, w, x, dev, stream, args.steps, world)
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        with nvtx("cpu baseline"):
-            cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
-
-    if rank == 0:
-        out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-               "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
-               "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-               "dtype": "bf16", "data": "synthetic", "config": config_of(w, world),
-               "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
-               "fwd_frac_peak": fwd_tf / peak_burst, "bwd_frac_peak": bwd_tf / peak_burst,
-               "fwd_frac_sustained_peak": fwd_tf / peak_sus,
-               "bwd_frac_sustained_peak": bwd_tf / peak_sus,
-               "roofline": roof, "fwd_mufu": fwd_mufu, "cpu_baseline": cpu, "e2e": e2e,
-               "clocks": clk,
-               "gqa": gqa, "varlen": varlen, "context_parallel": cp, "eager_baseline": eager,
-               "bwd_teacher_ms": bwd_t_ms,
-               "bwd_teacher_tflops": flops_bwd_teacher(w) / (bwd_t_ms * 1e-3) / 1e12,
-               "gpu_launches": 2 * args.steps,
-               "extra_hbm_bytes": 3 * 4 * w.bh * w.N_Q,
-               "impl": "ours"}
-        print(json.dumps(out), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    return bwd_t_ms, gqa, varlen, cp
 
 
 def run_varlen(skl, w, dev, stream, steps, world, tokens=65536, lo=512, hi=8192):
