@@ -20,7 +20,8 @@
 //      lanes, 64 query columns), K read from TMEM as the A operand;
 //   2. the dS warps of step parity s&1 (one thread per key row, each warp 32 of the 64
 //      query columns) recompute P_T, P_S, form dS^T in registers and store it as bf16
-//      into shared-memory buffer s&1;
+//      into shared-memory buffer s&1; for the student gradient the teacher score MMAs are
+//      committed on their own, so P_T is computed while the student score MMAs still run;
 //   3. tensor core: dK += dS^T Q (TMEM accumulator over all steps) and
 //      dQ^T_part = K^T dS^T into TMEM buffer s&1 (d on the lanes, queries on columns);
 //   4. the same warps copy dQ^T_part from TMEM into the fp32 staging tile of parity s&1,
@@ -108,11 +109,20 @@ static_assert(!SKL_BWD_SPLIT || kBwdDsWarps * SKL_BWD_RS_T + 4 * SKL_BWD_RC_T <=
                                     (kBwdDsWarps + 4) * ((65536 / kBwdThreads) & ~7),
               "register split exceeds the launch's register pool");
 
+// SKL_BWD_TFIRST (student gradient, lean MMA issue): the teacher score MMAs of a step are
+// committed to their own barrier, so the dS warps load S_T^T and compute P_T while the
+// student score MMAs are still running.
+#ifndef SKL_BWD_TFIRST
+#define SKL_BWD_TFIRST 1
+#endif
+
 // SKL_BWD_LEANMMA (with SKL_BWD_KTMEM): the MMA thread's per-step work reduced to adds of
 // compile-time constants to precomputed descriptor halves and addresses.
 #ifndef SKL_BWD_LEANMMA
 #define SKL_BWD_LEANMMA 1
 #endif
+static_assert(!SKL_BWD_TFIRST || (SKL_BWD_LEANMMA && SKL_BWD_KTMEM && SKL_BWD_SPLIT),
+              "teacher scores first assume the lean MMA issue, K in TMEM and 16 dS warps");
 
 // SKL_BWD_NSTG = 2: two fp32 staging tiles for the dQ reduce-adds, one per step parity (each
 // dS warpgroup drains into its own tile while the previous reduce is still reading the
@@ -156,7 +166,7 @@ struct BwdCfg {
     return (NSTG == 2 && (p & 1)) ? OFF_KX : OFF_STG;
   }
   static constexpr int OFF_BAR = OFF_ST + NSTS * STATS;
-  static constexpr int BAR_BYTES = 256;
+  static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES;  // the dynamic base is 1024-byte aligned
   static constexpr int THREADS = kBwdThreads;
   // TMEM columns: S_T^T / S_S^T per buffer, dK, dQ^T per buffer.
@@ -176,6 +186,7 @@ struct BwdBars {
   uint64_t q_full[3], q_empty[3], st_full[2], st_empty[2];
   uint64_t stg_full[2], stg_free[2];  // indexed by step parity
   uint64_t s_full[2], s_free[2];
+  uint64_t t_full[2];  // SKL_BWD_TFIRST: teacher scores of the step (parity) are ready
   uint64_t ds_full[2], ds_empty[2];
   uint64_t dq_full[2], dq_free[2];
   uint64_t dk_full;
@@ -184,6 +195,9 @@ struct BwdBars {
   uint32_t tmem_base;
   int abort_flag;
 };
+
+static_assert(sizeof(BwdBars) <= BwdCfg<128, 128, false>::BAR_BYTES,
+              "barrier block exceeds its shared-memory reservation");
 
 __device__ __forceinline__ void skl_fail_b(volatile int* abort_flag) {
   atomicOr(&g_skl_error, 2u);
@@ -249,6 +263,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&bars->s_full[b]), 1);
+      mbar_init(smem_u32(&bars->t_full[b]), 1);
       mbar_init(smem_u32(&bars->s_free[b]), kBwdArrive);
       mbar_init(smem_u32(&bars->ds_full[b]), kBwdArrive);
       mbar_init(smem_u32(&bars->ds_empty[b]), 1);
@@ -454,6 +469,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
             const uint32_t qa = ((kk >> 2) * (C::BM * 128) + (kk & 3) * 32) >> 4;
             umma_bf16_ts_lh(t_st, t_kt + kk * 8, lq + qa, hi, idesc_st, kk > 0);
           }
+          if (SKL_BWD_TFIRST && !TEACHER) umma_commit(smem_u32(&bars->t_full[s & 1]));
     #pragma unroll
           for (int kk = 0; kk < DS / 16; ++kk) {
             const uint32_t qa = (C::QT_TILE + (kk >> 2) * (C::BM * 128) + (kk & 3) * 32) >> 4;
@@ -689,6 +705,77 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     for (int s = wg; ok && s < n_steps; s += 2) {
       const int st = s % C::NQST;
       const int i0 = (jq_begin + s) * C::BM;  // first query column of this step
+#if SKL_BWD_TFIRST
+      if constexpr (!TEACHER && NC == 32) {
+        // Teacher scores first: P_T of this warp's columns while the student score MMAs of
+        // the step are still running, then the student scores.
+        if (!mbar_wait(smem_u32(&bars->t_full[wg]), (s >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t vt[NC];
+        tmem_ld_32_wait(tmem + lane_off + C::TM_S + sbuf * 128 + c0, vt);
+        if (!mbar_wait(smem_u32(&bars->st_full[s & 1]), (s >> 1) & 1)) { ok = false; break; }
+        const float* sts = stats + (s & 1) * (4 * C::BM);
+        float pt[NC];
+#pragma unroll
+        for (int u4 = 0; u4 < NC / 4; ++u4) {
+          const float4 nl = *reinterpret_cast<const float4*>(sts + c0 + 4 * u4);
+          pt[4 * u4 + 0] = ex2_approx(fmaf(__uint_as_float(vt[4 * u4 + 0]), cT, nl.x));
+          pt[4 * u4 + 1] = ex2_approx(fmaf(__uint_as_float(vt[4 * u4 + 1]), cT, nl.y));
+          pt[4 * u4 + 2] = ex2_approx(fmaf(__uint_as_float(vt[4 * u4 + 2]), cT, nl.z));
+          pt[4 * u4 + 3] = ex2_approx(fmaf(__uint_as_float(vt[4 * u4 + 3]), cT, nl.w));
+        }
+        if (!mbar_wait(smem_u32(&bars->s_full[wg]), (s >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t vs[NC];
+        tmem_ld_32_wait(tmem + lane_off + C::TM_S + sbuf * 128 + 64 + c0, vs);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[wg]));
+        const bool causal_mask = args.causal && (i0 + seq.off < k0 + C::BN - 1);
+        const bool need_mask = causal_mask || (k0 + C::BN > seq.nk);
+        const int cmin = key >= seq.nk ? C::BM : (causal_mask ? (key - seq.off - i0) : -1);
+        uint32_t pk[NC / 8][4];
+#pragma unroll
+        for (int uu = 0; uu < NC / 8; ++uu) {
+          const int u = c0 / 8 + uu;
+          const float4 nls0 = *reinterpret_cast<const float4*>(sts + C::BM + u * 8);
+          const float4 nls1 = *reinterpret_cast<const float4*>(sts + C::BM + u * 8 + 4);
+          const float4 g0 = *reinterpret_cast<const float4*>(sts + 2 * C::BM + u * 8);
+          const float4 g1 = *reinterpret_cast<const float4*>(sts + 2 * C::BM + u * 8 + 4);
+          const float nls[8] = {nls0.x, nls0.y, nls0.z, nls0.w, nls1.x, nls1.y, nls1.z, nls1.w};
+          const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+          float d[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = u * 8 + e;
+            const int ci = uu * 8 + e;
+            const float pS = ex2_approx(fmaf(__uint_as_float(vs[ci]), cS, nls[e]));
+            float ds = gg[e] * (pS - pt[ci]);
+            if (need_mask && c < cmin) ds = 0.f;
+            d[e] = ds;
+          }
+          pk[uu][0] = pack_bf16x2(d[0], d[1]);
+          pk[uu][1] = pack_bf16x2(d[2], d[3]);
+          pk[uu][2] = pack_bf16x2(d[4], d[5]);
+          pk[uu][3] = pack_bf16x2(d[6], d[7]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->st_empty[s & 1]));
+        if (!mbar_wait(smem_u32(&bars->ds_empty[wg]), ((s >> 1) & 1) ^ 1)) { ok = false; break; }
+#pragma unroll
+        for (int uu = 0; uu < NC / 8; ++uu) {
+          const int u = c0 / 8 + uu;
+          st_shared_v4(s_ds_row + ((u ^ (kl & 7)) << 4), pk[uu][0], pk[uu][1], pk[uu][2],
+                       pk[uu][3]);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->ds_full[wg]));
+        if (last >= 0 && !drain_dq(last)) { ok = false; break; }
+        last = s;
+        continue;
+      }
+#endif
       if (!mbar_wait(smem_u32(&bars->s_full[wg]), (s >> 1) & 1)) {
         ok = false;
         break;

@@ -121,6 +121,9 @@ struct FwdBars {
   int abort_flag;
 };
 
+static_assert(sizeof(FwdBars) <= FwdCfg<128, 128>::BAR_BYTES,
+              "barrier block exceeds its shared-memory reservation");
+
 __device__ __forceinline__ void skl_fail(volatile int* abort_flag) {
   atomicOr(&g_skl_error, 1u);
   *abort_flag = 1;
