@@ -202,6 +202,14 @@ __device__ __forceinline__ void tmem_st_32(uint32_t taddr, const uint32_t (&r)[3
       : "memory");
 }
 
+// 8 columns of this warp's 32 lanes: registers -> tensor memory (no wait).
+__device__ __forceinline__ void tmem_st_8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -308,6 +316,15 @@ __device__ __forceinline__ void tmem_ld_4x32_wait(uint32_t ta, uint32_t tb, uint
         SKL_R8(56), SKL_R8(64), SKL_R8(72), SKL_R8(80), SKL_R8(88), SKL_R8(96), SKL_R8(104),
         SKL_R8(112), SKL_R8(120)
       : "r"(ta), "r"(tb), "r"(tc), "r"(td)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_8_wait(uint32_t ta, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : SKL_R8(0)
+      : "r"(ta)
       : "memory");
 }
 
@@ -600,6 +617,19 @@ __device__ __forceinline__ void regs_dec() {
 template <uint32_t N>
 __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Named barrier over `count` threads that also returns to every participant whether any of
+// them passed pred = true (one uniform decision for all of them).
+__device__ __forceinline__ bool named_bar_any(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %3, 0;\n"
+      " barrier.cta.red.or.pred q, %1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"(id), "r"(count), "r"(pred ? 1u : 0u)
+      : "memory");
+  return r != 0;
 }
 
 // Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).

@@ -17,6 +17,7 @@
 
 #include "streamkl.h"
 #include "fwd_kernel.cuh"
+#include "fwd_persistent.cuh"
 #include "bwd_kernel.cuh"
 #include "merge_kernel.cuh"
 
@@ -175,6 +176,26 @@ int group_override(bool fwd) {
   return fwd ? f : b;
 }
 
+// Forward grid form for a dense problem of `units` work units: persistent (one CTA per SM
+// walking a heaviest-first snake of units) when there are at most kPersistRounds units per
+// SM. There the per-CTA prologue and the tail of a one-CTA-per-unit grid are a visible part
+// of the launch, and all of the heads' key tiles are few enough to share L2; with more units
+// per SM the head-grouped grid keeps each group's key tiles in L2. STREAMKL_FWD_PERSIST
+// (read once) overrides: 0 never, 1 always (dense problems).
+constexpr int kPersistRounds = 8;
+#ifndef SKL_FWD_PERSIST_MODE
+#define SKL_FWD_PERSIST_MODE -1  // -1: by the rule above
+#endif
+bool fwd_persistent(long long units) {
+  static const int mode = [] {
+    const char* v = std::getenv("STREAMKL_FWD_PERSIST");
+    return v ? std::atoi(v) : SKL_FWD_PERSIST_MODE;
+  }();
+  if (mode == 0) return false;
+  if (mode == 1) return true;
+  return units <= (long long)kPersistRounds * sm_count();
+}
+
 // Heads per scheduling group: small enough that a group's tiles stay in the 126 MB L2,
 // large enough to fill the SMs with a heaviest-first mix. The base size is raised (up to
 // twice) until one group holds at least a wave of CTAs, so that short sequences, with few
@@ -199,15 +220,23 @@ bool set_smem(Kern k, int bytes) {
 
 template <int DT, int DS>
 streamkl_status launch_fwd(const CUtensorMap* maps, const skl::FwdArgs& a, bool negT, bool negS,
-                           cudaStream_t stream) {
+                           bool persistent, cudaStream_t stream) {
   using C = skl::FwdCfg<DT, DS>;
-  auto kern = skl::streamkl_fwd_kernel<DT, DS>;
-  if (!set_smem(kern, C::SMEM)) return STREAMKL_ERR_LAUNCH;
   const uint32_t it = skl::idesc_bf16_f32(128, C::BN, false, false, negT);
   const uint32_t is = skl::idesc_bf16_f32(128, C::BN, false, false, negS);
-  const long long grid = (long long)a.n_ctas_per_bh * a.BH;
-  kern<<<dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream>>>(maps[0], maps[1], maps[2],
-                                                                    maps[3], a, it, is);
+  const long long units = (long long)a.n_ctas_per_bh * a.BH;
+  if (persistent) {
+    auto kern = skl::streamkl_fwd_persistent_kernel<DT, DS>;
+    if (!set_smem(kern, C::SMEM)) return STREAMKL_ERR_LAUNCH;
+    const long long grid = units < sm_count() ? units : sm_count();
+    kern<<<dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream>>>(maps[0], maps[1], maps[2],
+                                                                      maps[3], a, it, is);
+  } else {
+    auto kern = skl::streamkl_fwd_kernel<DT, DS>;
+    if (!set_smem(kern, C::SMEM)) return STREAMKL_ERR_LAUNCH;
+    kern<<<dim3((unsigned)units), dim3(C::THREADS), C::SMEM, stream>>>(maps[0], maps[1], maps[2],
+                                                                       maps[3], a, it, is);
+  }
   return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
 }
 
@@ -275,10 +304,11 @@ streamkl_status fwd_common(const void* q_t, const void* k_t, const void* q_s, co
   a.lse_s = lse_s;
   if (a.n_ctas_per_bh == 0) return STREAMKL_OK;  // packed, every sequence empty
   const bool nT = scale_T < 0.f, nS = scale_S < 0.f;
-  if (d_T == 128 && d_S == 128) return launch_fwd<128, 128>(maps, a, nT, nS, stream);
-  if (d_T == 128 && d_S == 64) return launch_fwd<128, 64>(maps, a, nT, nS, stream);
-  if (d_T == 64 && d_S == 128) return launch_fwd<64, 128>(maps, a, nT, nS, stream);
-  return launch_fwd<64, 64>(maps, a, nT, nS, stream);
+  const bool pers = !P.packed() && fwd_persistent((long long)a.n_ctas_per_bh * bh);
+  if (d_T == 128 && d_S == 128) return launch_fwd<128, 128>(maps, a, nT, nS, pers, stream);
+  if (d_T == 128 && d_S == 64) return launch_fwd<128, 64>(maps, a, nT, nS, pers, stream);
+  if (d_T == 64 && d_S == 128) return launch_fwd<64, 128>(maps, a, nT, nS, pers, stream);
+  return launch_fwd<64, 64>(maps, a, nT, nS, pers, stream);
 }
 
 // Shared body of the student and trainable-teacher backward entry points.

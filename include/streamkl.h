@@ -44,6 +44,10 @@
  *   (4 heads forward, 2 backward, raised up to twice that until a group holds one wave of
  *   CTAs). They change only the speed: results are the same for any group size, except
  *   that dQ is summed in a different order (fp32 reduce-adds across CTAs).
+ * - The dense forward runs as a persistent grid (one CTA per SM walking a heaviest-first
+ *   snake of work units) when it has at most 8 units (pairs of 128-row query tiles) per SM,
+ *   and as one CTA per unit otherwise; STREAMKL_FWD_PERSIST=0 / 1 (read once per process)
+ *   forces the per-unit / persistent form. Both give bit-identical results.
  */
 #ifndef STREAMKL_H
 #define STREAMKL_H
