@@ -16,6 +16,7 @@
 // which merge at the end, so that KL = ln2 * A / l_T - LSE_T + LSE_S. Per tile a thread
 // reads its 64 scores from TMEM in one round trip and releases the buffer at once; the
 // fp32 work is issued as packed pairs, with a share of the exponentials on the FMA pipe.
+// Unmasked tiles are folded against the running maxima as they stand (no per-tile max).
 // Nothing of size N_Q x N_K ever leaves the SM.
 //
 // Warp roles (640 threads, SKL_FWD_SPLIT): warps 0-7 query tile 0 and 8-15 query tile 1
@@ -240,20 +241,12 @@ __device__ __forceinline__ void fold_tile(RowState& st, uint32_t ta, float cT, f
   st.A += (w0 + w1) + (mT_use - mS_use) * sumT;
 }
 
-// Half a tile (32 keys: TMEM columns tT .. tT+31 teacher, tS .. tS+31 student) folded
-// into the row state of one warp of a split pair; lim as in fold_tile, relative to the
-// half's first key.
+// Sums of one half tile (32 keys) against reference maxima (mT_use, mS_use):
+// sumT = sum 2^(t - mT), sumS = sum 2^(s - mS), w = sum 2^(t - mT) * ((t - mT) - (s - mS)).
 template <bool MASK>
-__device__ __forceinline__ void fold_half(RowState& st, uint32_t tT, uint32_t tS, float cT,
-                                          float cS, int lim, uint32_t s_free, int lane) {
-  uint32_t v[64];
-  tmem_ld_2x32_wait(tT, tS, v);
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) mbar_arrive(s_free);
-  const float mxT = max_tree32<MASK>(v, 0, lim), mxS = max_tree32<MASK>(v, 32, lim);
-  float mT_use, mS_use;
-  update_max(st, mxT, mxS, cT, cS, mT_use, mS_use);
+__device__ __forceinline__ void half_sums(const uint32_t (&v)[64], float cT, float cS,
+                                          float mT_use, float mS_use, int lim, float& sumT,
+                                          float& sumS, float& w) {
   const uint64_t cT2 = f2_pack(cT, cT), cS2 = f2_pack(cS, cS);
   const uint64_t nmT2 = f2_pack(-mT_use, -mT_use), nmS2 = f2_pack(-mS_use, -mS_use);
   uint64_t sT2 = f2_pack(0.f, 0.f), sS2 = sT2, b2 = sT2;
@@ -265,10 +258,70 @@ __device__ __forceinline__ void fold_half(RowState& st, uint32_t tT, uint32_t tS
   f2_unpack(sT2, s0, s1);
   f2_unpack(sS2, u0, u1);
   f2_unpack(b2, w0, w1);
-  const float sumT = s0 + s1;
+  sumT = s0 + s1;
+  sumS = u0 + u1;
+  w = w0 + w1;
+}
+
+// SKL_FWD_LAZY: an unmasked half tile is folded against the row's running maxima as they
+// stand, without first taking the tile's maxima (the state is exact for any reference:
+// l and A are sums relative to 2^m). The result is kept when every lane's tile sums stay
+// below 2^64 (a score at most about 64 above the reference; false for inf and NaN);
+// otherwise the tile is folded again the ordinary way. With fewer than 2^26 tiles per row
+// the running sums then stay below 2^90, far from fp32 overflow. SKL_FWD_LAZY_RENORM
+// additionally raises a reference by a sum's binary exponent k once the sum passes 2^32
+// and scales the sums by 2^-k (exact).
+#ifndef SKL_FWD_LAZY
+#define SKL_FWD_LAZY 1
+#endif
+#ifndef SKL_FWD_LAZY_RENORM
+#define SKL_FWD_LAZY_RENORM 0
+#endif
+
+__device__ __forceinline__ void lazy_renorm(float& m, float& l, float* a) {
+  if (l >= 0x1p32f) {
+    const int k = ((__float_as_int(l) >> 23) & 0xff) - 127;  // 32 .. 127
+    const float sc = __int_as_float((127 - k) << 23);        // 2^-k, a normal number
+    l *= sc;
+    if (a) *a *= sc;
+    m += (float)k;
+  }
+}
+
+// Half a tile (32 keys: TMEM columns tT .. tT+31 teacher, tS .. tS+31 student) folded
+// into the row state of one warp of a split pair; lim as in fold_tile, relative to the
+// half's first key.
+template <bool MASK>
+__device__ __forceinline__ void fold_half(RowState& st, uint32_t tT, uint32_t tS, float cT,
+                                          float cS, int lim, uint32_t s_free, int lane) {
+  uint32_t v[64];
+  tmem_ld_2x32_wait(tT, tS, v);
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(s_free);
+  float sumT, sumS, w;
+#if SKL_FWD_LAZY
+  if (!MASK && __all_sync(0xffffffffu, st.mT != -INFINITY && st.mS != -INFINITY)) {
+    half_sums<false>(v, cT, cS, st.mT, st.mS, 31, sumT, sumS, w);
+    if (__all_sync(0xffffffffu, sumT < 0x1p64f && sumS < 0x1p64f)) {
+      st.lT += sumT;
+      st.lS += sumS;
+      st.A += w + (st.mT - st.mS) * sumT;
+      if (SKL_FWD_LAZY_RENORM) {
+        lazy_renorm(st.mT, st.lT, &st.A);
+        lazy_renorm(st.mS, st.lS, nullptr);
+      }
+      return;
+    }
+  }
+#endif
+  const float mxT = max_tree32<MASK>(v, 0, lim), mxS = max_tree32<MASK>(v, 32, lim);
+  float mT_use, mS_use;
+  update_max(st, mxT, mxS, cT, cS, mT_use, mS_use);
+  half_sums<MASK>(v, cT, cS, mT_use, mS_use, lim, sumT, sumS, w);
   st.lT += sumT;
-  st.lS += u0 + u1;
-  st.A += (w0 + w1) + (mT_use - mS_use) * sumT;
+  st.lS += sumS;
+  st.A += w + (mT_use - mS_use) * sumT;
 }
 
 // Merge of two row states (rescale both to the larger maxima and add).

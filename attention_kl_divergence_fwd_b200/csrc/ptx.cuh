@@ -534,7 +534,9 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
   float x0, x1;
   f2_unpack(x, x0, x1);
-  x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  // Clamped to [-125, 64]: the upper bound keeps n inside the exponent field for the
+  // positive arguments of a stale reference maximum (64 and above read as too large).
+  x = f2_pack(fminf(fmaxf(x0, -125.0f), 64.0f), fminf(fmaxf(x1, -125.0f), 64.0f));
   const uint64_t kShift = f2_pack(12582912.0f, 12582912.0f);
   const uint64_t y = f2_add(x, kShift);
   const uint64_t f = f2_sub(x, f2_sub(y, kShift));

@@ -193,6 +193,26 @@ def test_large_scores():
     check_full(w, make_inputs(w, seed=8))
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_score_jumps_past_the_running_maximum(causal):
+    """Keys planted in later tiles raise some rows' scores far above their first tiles.
+
+    The forward folds an unmasked tile against the row's running maxima as they stand and
+    folds it again from the tile's own maxima when an exponential would reach 2^64. Key 500
+    (x3 along query 600) lifts that teacher row by about 44 in log2 units (kept, sums up to
+    2^44), key 560 (x8 along query 620) by about 115 (refolded); the student side gets the
+    same at keys 450 / 530 for queries 610 / 630 of head 1. Every other row sees those keys
+    with scores spread about 8 times wider than the rest."""
+    w = BASE.with_sizes(B=1, H=2, N_Q=640, N_K=640, causal=causal)
+    x = make_inputs(w, seed=21)
+    for side, h, plants in (("t", 0, ((500, 600, 3.0), (560, 620, 8.0))),
+                            ("s", 1, ((450, 610, 3.0), (530, 630, 8.0)))):
+        k, q = x["k_" + side], x["q_" + side]
+        for key, row, gain in plants:
+            k[0, h, key] = (q[0, h, row].float() * gain).to(k.dtype)
+    check_full(w, x)
+
+
 def test_identical_inputs_exact_zero():
     w = BASE.with_sizes(B=2, H=2, N_Q=333, N_K=333, causal=True)
     x = make_inputs(w, seed=3)
