@@ -110,6 +110,12 @@ struct FwdCfg {
   static_assert(SMEM <= SMEM_MAX, "shared memory budget");
 };
 
+// SKL_FWD_QORDER (single score buffer per query tile): per key tile the MMA thread serves
+// first the query tile whose score buffer is already free, instead of always query tile 0.
+#ifndef SKL_FWD_QORDER
+#define SKL_FWD_QORDER 1
+#endif
+
 struct FwdBars {
   uint64_t q_full;
   uint64_t full[4];
@@ -585,8 +591,19 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           }
           tc_fence_after();
           const uint32_t st = s_k + s * C::STAGE;
+          int qfirst = 0;
+#if SKL_FWD_QTMEM && SKL_FWD_QORDER
+          static_assert(C::NQ == 2, "two query tiles per CTA");
+          if (j > 0 && j < nk[0] && j < nk[1]) {
+            const uint32_t par = ((j - 1) >> 1) & 1;
+            if (!mbar_test(smem_u32(&bars->s_free[0][(j - 1) & 1]), par) &&
+                mbar_test(smem_u32(&bars->s_free[1][(j - 1) & 1]), par))
+              qfirst = 1;
+          }
+#endif
   #pragma unroll
-          for (int q = 0; q < C::NQ; ++q) {
+          for (int qi = 0; qi < C::NQ; ++qi) {
+            const int q = qi ^ qfirst;
             if (j >= nk[q]) continue;
             const int b = j & 1;
 #if SKL_FWD_QTMEM
