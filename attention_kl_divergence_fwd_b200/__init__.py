@@ -32,7 +32,8 @@ EXPORTS = ("streamkl_fwd", "streamkl_bwd", "streamkl_bwd_teacher", "streamkl_fwd
            "streamkl_bwd_gqa", "streamkl_bwd_teacher_gqa", "streamkl_fwd_varlen",
            "streamkl_bwd_varlen", "streamkl_bwd_teacher_varlen", "streamkl_fwd_partial",
            "streamkl_merge_partial", "streamkl_bwd_shard", "streamkl_bwd_teacher_shard",
-           "streamkl_watchdog_selftest", "streamkl_exp2_eval", "streamkl_status_string",
+           "streamkl_watchdog_selftest", "streamkl_exp2_eval", "streamkl_sm_clock_probe",
+           "streamkl_status_string",
            "streamkl_device_status", "streamkl_version")
 
 
@@ -93,6 +94,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.streamkl_bwd_teacher_shard.restype = i
     lib.streamkl_exp2_eval.argtypes = [vp, vp, vp, ctypes.c_longlong, vp]
     lib.streamkl_exp2_eval.restype = i
+    lib.streamkl_sm_clock_probe.argtypes = [vp, ctypes.c_longlong, vp]
+    lib.streamkl_sm_clock_probe.restype = i
     lib.streamkl_watchdog_selftest.argtypes = [vp]
     lib.streamkl_watchdog_selftest.restype = i
     lib.streamkl_status_string.argtypes = [i]
@@ -530,6 +533,16 @@ def exp2_eval(x, stream=None):
     _check(load_library().streamkl_exp2_eval(x.data_ptr(), y1.data_ptr(), y2.data_ptr(),
                                              x.numel(), _stream_ptr(stream)), "streamkl_exp2_eval")
     return y1, y2
+
+
+def sm_clock_probe(out, ns: int = 20000, stream=None) -> None:
+    """Enqueue the SM clock probe on the stream: out (int64 CUDA tensor of 2) receives the
+    clock ticks and nanoseconds of a ~`ns` ns spin; out[0] / out[1] * 1000 is the SM MHz."""
+    import torch
+    if out.dtype != torch.int64 or not out.is_cuda or not out.is_contiguous() or out.numel() < 2:
+        raise ValueError("out must be a contiguous int64 CUDA tensor of at least 2 elements")
+    _check(load_library().streamkl_sm_clock_probe(out.data_ptr(), int(ns), _stream_ptr(stream)),
+           "streamkl_sm_clock_probe")
 
 
 def device_status(stream=None) -> int:

@@ -123,6 +123,13 @@ static_assert(!SKL_BWD_SPLIT || kBwdDsWarps * SKL_BWD_RS_T + 4 * SKL_BWD_RC_T <=
 #endif
 static_assert(!SKL_BWD_TFIRST || (SKL_BWD_LEANMMA && SKL_BWD_KTMEM && SKL_BWD_SPLIT),
               "teacher scores first assume the lean MMA issue, K in TMEM and 16 dS warps");
+// SKL_BWD_TFREE (with SKL_BWD_TFIRST): the teacher half of the score buffer is released as
+// soon as the dS warps have loaded it, so the next step's teacher score MMAs can start
+// while the student half is still being read.
+#ifndef SKL_BWD_TFREE
+#define SKL_BWD_TFREE 0
+#endif
+static_assert(!SKL_BWD_TFREE || SKL_BWD_TFIRST, "the early teacher release needs SKL_BWD_TFIRST");
 
 // SKL_BWD_NSTG = 2: two fp32 staging tiles for the dQ reduce-adds, one per step parity (each
 // dS warpgroup drains into its own tile while the previous reduce is still reading the
@@ -187,6 +194,7 @@ struct BwdBars {
   uint64_t stg_full[2], stg_free[2];  // indexed by step parity
   uint64_t s_full[2], s_free[2];
   uint64_t t_full[2];  // SKL_BWD_TFIRST: teacher scores of the step (parity) are ready
+  uint64_t t_free[2];  // SKL_BWD_TFREE: teacher scores of the step (parity) have been read
   uint64_t ds_full[2], ds_empty[2];
   uint64_t dq_full[2], dq_free[2];
   uint64_t dk_full;
@@ -264,6 +272,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&bars->s_full[b]), 1);
       mbar_init(smem_u32(&bars->t_full[b]), 1);
+      mbar_init(smem_u32(&bars->t_free[b]), kBwdArrive);
       mbar_init(smem_u32(&bars->s_free[b]), kBwdArrive);
       mbar_init(smem_u32(&bars->ds_full[b]), kBwdArrive);
       mbar_init(smem_u32(&bars->ds_empty[b]), 1);
@@ -458,9 +467,12 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         const uint32_t t_kt = tmem + C::TM_KT, t_ks = tmem + C::TM_KS, t_dq = tmem + C::TM_DQ;
         int s_st = 0;      // query stage of the next score step
         uint32_t s_ph = 0;  // and the phase of its q_full barrier
+        constexpr bool kTFree = SKL_BWD_TFREE && !TEACHER;
         auto issue_scores = [&](int s) -> bool {
           if (!mbar_wait(smem_u32(&bars->q_full[s_st]), s_ph)) return false;
-          if (s > 0 && !mbar_wait(smem_u32(&bars->s_free[(s - 1) & 1]), ((s - 1) >> 1) & 1))
+          if (s > 0 && !mbar_wait(smem_u32(kTFree ? &bars->t_free[(s - 1) & 1]
+                                                  : &bars->s_free[(s - 1) & 1]),
+                                  ((s - 1) >> 1) & 1))
             return false;
           tc_fence_after();
           const uint32_t lq = lq0 + (uint32_t)s_st * kQ16;
@@ -470,6 +482,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
             umma_bf16_ts_lh(t_st, t_kt + kk * 8, lq + qa, hi, idesc_st, kk > 0);
           }
           if (SKL_BWD_TFIRST && !TEACHER) umma_commit(smem_u32(&bars->t_full[s & 1]));
+          if (kTFree && s > 0) {
+            if (!mbar_wait(smem_u32(&bars->s_free[(s - 1) & 1]), ((s - 1) >> 1) & 1)) return false;
+            tc_fence_after();
+          }
     #pragma unroll
           for (int kk = 0; kk < DS / 16; ++kk) {
             const uint32_t qa = (C::QT_TILE + (kk >> 2) * (C::BM * 128) + (kk & 3) * 32) >> 4;
@@ -713,6 +729,11 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         tc_fence_after();
         uint32_t vt[NC];
         tmem_ld_32_wait(tmem + lane_off + C::TM_S + sbuf * 128 + c0, vt);
+#if SKL_BWD_TFREE
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->t_free[wg]));
+#endif
         if (!mbar_wait(smem_u32(&bars->st_full[s & 1]), (s >> 1) & 1)) { ok = false; break; }
         const float* sts = stats + (s & 1) * (4 * C::BM);
         float pt[NC];

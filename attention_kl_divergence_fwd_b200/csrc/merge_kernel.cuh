@@ -75,4 +75,19 @@ __global__ void streamkl_exp2_kernel(const float* __restrict__ x, float* __restr
   }
 }
 
+// SM clock probe: one warp spins for about `ns` nanoseconds of the global timer and
+// records the SM clock ticks (clock64) that passed meanwhile and the nanoseconds themselves;
+// ticks / ns is the clock the SM actually ran at, which NVML's sampled clock can miss.
+__global__ void streamkl_clock_kernel(long long* __restrict__ out, long long ns) {
+  const uint64_t t0 = global_timer_ns();
+  const long long c0 = clock64();
+  uint64_t t1 = t0;
+  while ((long long)(t1 - t0) < ns) t1 = global_timer_ns();
+  const long long c1 = clock64();
+  if (threadIdx.x == 0) {
+    out[0] = c1 - c0;
+    out[1] = (long long)(t1 - t0);
+  }
+}
+
 }  // namespace skl

@@ -493,14 +493,15 @@ __device__ __forceinline__ float max_tree32(const uint32_t (&v)[N], int base, in
   return fmaxf(fmax3(l2a, l2b, l2c), l2d);
 }
 
-// 2^x on the FMA pipe, for x <= 0 (inputs below -125 give 2^-125; callers only add the
-// result to sums that are at least 1). Method: Cody-Waite style range reduction
+// 2^x on the FMA pipe for x in [-125, 64] (arguments are clamped to that range: below, 2^-125,
+// which callers only add to sums that are at least 1; above, 2^64, which the forward's
+// stale-reference fold reads as too large). Method: Cody-Waite style range reduction
 // x = n + f, n = round-to-nearest(x) taken with the 1.5*2^23 shifter, f in [-1/2, 1/2];
 // 2^f from a degree-5 polynomial fitted by this project (minimax relative error on
 // [-1/2, 1/2] by linear programming, see fit_exp2_poly.py): max relative error 1.9e-7
 // in fp32 Horner form; n is added straight into the exponent field.
 __device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.0f);
+  x = fminf(fmaxf(x, -125.0f), 64.0f);
   const float kShift = 12582912.0f;
   const float y = __fadd_rn(x, kShift);
   const float f = __fsub_rn(x, __fsub_rn(y, kShift));
@@ -546,8 +547,6 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
   float x0, x1;
   f2_unpack(x, x0, x1);
-  // Clamped to [-125, 64]: the upper bound keeps n inside the exponent field for the
-  // positive arguments of a stale reference maximum (64 and above read as too large).
   x = f2_pack(fminf(fmaxf(x0, -125.0f), 64.0f), fminf(fmaxf(x1, -125.0f), 64.0f));
   const uint64_t kShift = f2_pack(12582912.0f, 12582912.0f);
   const uint64_t y = f2_add(x, kShift);

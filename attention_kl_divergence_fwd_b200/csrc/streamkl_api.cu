@@ -582,6 +582,12 @@ streamkl_status streamkl_exp2_eval(const float* x, float* y_scalar, float* y_pai
   return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
 }
 
+streamkl_status streamkl_sm_clock_probe(long long* out, long long ns, cudaStream_t stream) {
+  if (!out || ns < 1000 || ns > 10000000) return STREAMKL_ERR_INVALID_ARG;
+  skl::streamkl_clock_kernel<<<1, 32, 0, stream>>>(out, ns);
+  return cudaGetLastError() == cudaSuccess ? STREAMKL_OK : STREAMKL_ERR_LAUNCH;
+}
+
 const char* streamkl_status_string(streamkl_status s) {
   switch (s) {
     case STREAMKL_OK: return "ok";

@@ -312,18 +312,32 @@ def main():
     clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if clocks:
         clocks.start()
+    # The SM clock the kernels actually ran at, measured by the library's probe (clock64
+    # ticks over global-timer nanoseconds) just before the first and just after the last
+    # timed step, outside the timed region: NVML's sampled clock misses the fast drops a
+    # sustained load causes.
+    probe = torch.zeros(2, 2, dtype=torch.int64, device=dev)
     barrier(world)
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with nvtx("timed steps"):
+        skl.sm_clock_probe(probe[0], 20000)
         t_start.record(stream)
         for k in range(args.steps):
             step(evs[k])
         t_end.record(stream)
+        skl.sm_clock_probe(probe[1], 20000)
         torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop() if clocks else None
+    if clk is not None:
+        pr = probe.cpu().tolist()
+        clk["sm_mhz_probe"] = {"before": round(pr[0][0] / pr[0][1] * 1e3, 1),
+                               "after": round(pr[1][0] / pr[1][1] * 1e3, 1),
+                               "how": "clock64 ticks / globaltimer ns of one warp spinning "
+                                      "20 us, launched right before and right after the "
+                                      "timed steps (outside the timed region)"}
     if skl.device_status() != 0:
         raise RuntimeError("kernel watchdog fired during the timed region")
 

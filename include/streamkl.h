@@ -258,11 +258,20 @@ streamkl_status streamkl_watchdog_selftest(cudaStream_t stream);
  * Diagnostic: the forward's FMA-pipe 2^x (range reduction with the 1.5*2^23 shifter, a
  * degree-5 minimax polynomial fitted for this library, the integer part added into the
  * exponent field) evaluated on n device floats x (n even), scalar form into y_scalar and
- * packed-pair form into y_pair. Inputs below -125 give 2^-125. INVALID_ARG for null pointers
- * or odd n.
+ * packed-pair form into y_pair. Arguments are clamped to [-125, 64]: inputs below give
+ * 2^-125, inputs above give 2^64. INVALID_ARG for null pointers or odd n.
  */
 streamkl_status streamkl_exp2_eval(const float* x, float* y_scalar, float* y_pair, long long n,
                                    cudaStream_t stream);
+
+/*
+ * Diagnostic: one warp spins for about `ns` nanoseconds (1e3 .. 1e7) of the GPU's global
+ * timer and writes, to the device array out[2] (caller-owned int64), the SM clock ticks
+ * that passed (clock64) and the nanoseconds measured; out[0] / out[1] is the SM clock in
+ * GHz at that moment. Asynchronous on `stream`. INVALID_ARG for a null pointer or `ns`
+ * outside its range.
+ */
+streamkl_status streamkl_sm_clock_probe(long long* out, long long ns, cudaStream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char* streamkl_status_string(streamkl_status status);

@@ -194,3 +194,12 @@ def test_shard_host_validation(lib):
     assert lib.streamkl_merge_partial(P, 2, 0, P, P, P, 0) == 1
     assert lib.streamkl_merge_partial(P + 4, 2, 100, P, P, P, 0) == 3
     assert lib.streamkl_merge_partial(0, 2, 100, P, P, P, 0) == 1
+
+
+def test_diagnostics_host_validation(lib):
+    # Rejected on the host before any launch: null pointers, odd sizes, probe times out of range.
+    assert lib.streamkl_sm_clock_probe(0, 20000, 0) == 1
+    assert lib.streamkl_sm_clock_probe(P, 999, 0) == 1
+    assert lib.streamkl_sm_clock_probe(P, 10000001, 0) == 1
+    assert lib.streamkl_exp2_eval(0, P, P, 8, 0) == 1
+    assert lib.streamkl_exp2_eval(P, P, P, 7, 0) == 1

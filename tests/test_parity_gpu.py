@@ -683,11 +683,13 @@ def test_config2_full_oracle():
 
 def test_fma_pipe_exp2_accuracy():
     """The forward's polynomial 2^x against the exact value (fp64) and against CUDA's exp2f:
-    relative error within the fitted bound (1.9e-7) plus fp32 rounding of the evaluation."""
+    relative error within the fitted bound (1.9e-7) plus fp32 rounding of the evaluation,
+    over [-124, 63.9] (positive arguments occur when a tile is folded against a stale
+    reference maximum)."""
     gen = torch.Generator().manual_seed(3)
-    x = torch.cat([torch.linspace(-124.0, 0.0, 1 << 20),
-                   -124.0 * torch.rand(1 << 20, generator=gen),
-                   torch.tensor([0.0, -0.5, 0.5 - 1.0, -1.0, -2.5, -124.0])])
+    x = torch.cat([torch.linspace(-124.0, 63.9, 1 << 20),
+                   -124.0 + 187.9 * torch.rand(1 << 20, generator=gen),
+                   torch.tensor([0.0, -0.5, 0.5 - 1.0, -1.0, -2.5, -124.0, 0.5, 1.0, 33.25, 63.5])])
     y1, y2 = skl.exp2_eval(x.cuda())
     exact = torch.exp2(x.double())
     for y in (y1, y2):
@@ -696,10 +698,20 @@ def test_fma_pipe_exp2_accuracy():
     cuda = torch.exp2(x.cuda()).cpu().double()  # CUDA's exp2f
     assert ((y1.cpu().double() - cuda) / cuda).abs().max().item() <= 5e-7
     assert torch.equal(y1, y2)  # the packed form computes the same values
-    # below the clamp: 2^-125
-    lo, _ = skl.exp2_eval(torch.tensor([-200.0, -125.0], device="cuda"))
-    assert torch.allclose(lo.cpu().double(), torch.full((2,), 2.0 ** -125, dtype=torch.float64),
-                          rtol=4e-7, atol=0)
+    # outside the clamp: 2^-125 below, 2^64 above (both forms)
+    for y in skl.exp2_eval(torch.tensor([-200.0, -125.0, 64.0, 200.0], device="cuda")):
+        want = torch.tensor([2.0 ** -125] * 2 + [2.0 ** 64] * 2, dtype=torch.float64)
+        assert torch.allclose(y.cpu().double(), want, rtol=4e-7, atol=0)
+
+
+def test_sm_clock_probe():
+    """The probe's ticks over nanoseconds is a plausible SM clock (the B200's range)."""
+    out = torch.zeros(2, dtype=torch.int64, device="cuda")
+    skl.sm_clock_probe(out, 20000)
+    assert skl.device_status() == 0
+    ticks, ns = out.tolist()
+    assert ns >= 20000
+    assert 300.0 <= ticks / ns * 1000.0 <= 2500.0
 
 
 def test_mixed_devices_rejected_before_any_launch():
