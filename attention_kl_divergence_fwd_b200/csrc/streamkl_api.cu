@@ -196,6 +196,13 @@ bool fwd_persistent(long long units) {
   return units <= (long long)kPersistRounds * sm_count();
 }
 
+#ifndef SKL_FWD_GROUP_BASE
+#define SKL_FWD_GROUP_BASE 4
+#endif
+#ifndef SKL_BWD_GROUP_BASE
+#define SKL_BWD_GROUP_BASE 2
+#endif
+
 // Heads per scheduling group: small enough that a group's tiles stay in the 126 MB L2,
 // large enough to fill the SMs with a heaviest-first mix. The base size is raised (up to
 // twice) until one group holds at least a wave of CTAs, so that short sequences, with few
@@ -288,7 +295,7 @@ streamkl_status fwd_common(const void* q_t, const void* k_t, const void* q_s, co
   a.cT = std::fabs(scale_T) * kLog2e;
   a.cS = std::fabs(scale_S) * kLog2e;
   a.n_ctas_per_bh = (P.N_Q + 255) / 256;
-  a.group = head_group(true, 4, bh, a.n_ctas_per_bh);
+  a.group = head_group(true, SKL_FWD_GROUP_BASE, bh, a.n_ctas_per_bh);
   a.H = P.H;
   a.gT = P.H / P.H_kv_T;
   a.gS = P.H / P.H_kv_S;
@@ -360,7 +367,7 @@ streamkl_status bwd_common(const void* q_t, const void* k_t, const void* q_s, co
   a.aS = std::fabs(scale_S);
   a.scale_G = TEACHER ? scale_T : scale_S;
   a.n_ktiles = (P.N_K + 127) / 128;
-  a.group = head_group(false, 2, bh, a.n_ktiles);
+  a.group = head_group(false, SKL_BWD_GROUP_BASE, bh, a.n_ktiles);
   a.H = P.H;
   a.gT = P.H / P.H_kv_T;
   a.gS = P.H / P.H_kv_S;
