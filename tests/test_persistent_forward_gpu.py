@@ -44,6 +44,17 @@ x = {k: v.cuda() for k, v in make_inputs(w, seed=61).items()}
 kl, lt, ls = skl.streamkl_fwd_gqa(x["q_t"], x["k_t"][:, :2].contiguous(), x["q_s"],
                                   x["k_s"][:, :4].contiguous(), w.scale_T, w.scale_S, True)
 out["gqa"] = torch.stack([kl, lt, ls]).cpu()
+# planted keys lift some rows' scores far above their first tiles (the lazy fold keeps a
+# tile with sums up to 2^44 and refolds one that would reach 2^64)
+w = base.with_sizes(B=1, H=2, N_Q=640, N_K=640, causal=False)
+x = make_inputs(w, seed=21)
+for side, h, plants in (("t", 0, ((500, 600, 3.0), (560, 620, 8.0))),
+                        ("s", 1, ((450, 610, 3.0), (530, 630, 8.0)))):
+    for key, row, gain in plants:
+        x["k_" + side][0, h, key] = (x["q_" + side][0, h, row].float() * gain).to(torch.bfloat16)
+x = {k: v.cuda() for k, v in x.items()}
+kl, lt, ls = skl.streamkl_fwd(x["q_t"], x["k_t"], x["q_s"], x["k_s"], w.scale_T, w.scale_S, False)
+out["jumps"] = torch.stack([kl, lt, ls]).cpu()
 # a key shard's raw row state (context parallelism): keys 384..767 of 1000
 w = base.with_sizes(B=1, H=3, N_Q=1000, N_K=1000, causal=True)
 x = {k: v.cuda() for k, v in make_inputs(w, seed=62).items()}
