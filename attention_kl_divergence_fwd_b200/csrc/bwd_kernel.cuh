@@ -130,20 +130,16 @@ static_assert(!SKL_BWD_TFIRST || (SKL_BWD_LEANMMA && SKL_BWD_KTMEM && SKL_BWD_SP
 #define SKL_BWD_TFREE 0
 #endif
 static_assert(!SKL_BWD_TFREE || SKL_BWD_TFIRST, "the early teacher release needs SKL_BWD_TFIRST");
-// SKL_BWD_DQ3 (student gradient) / SKL_BWD_DQ3_T (trainable-teacher gradient): the S_S
-// score MMAs read K_S from shared memory instead of TMEM, and the 64 TMEM columns this
-// frees hold a third dQ^T buffer, so a step's dQ^T MMAs reuse the buffer of step s-3
-// (drained long before) instead of step s-2. Measured at N = 16384, d = 128: teacher
-// gradient +8.5 %, student gradient -1.9 % (its S_S MMAs are on the teacher-first
-// critical path); teacher gradient with d_S = 64 (mismatched heads): -1.6 to -3 %. So it
-// is used for the teacher gradient with d_S = 128 only.
+// SKL_BWD_DQ3 (student gradient only): the S_S score MMAs read K_S from shared memory
+// instead of TMEM, and the 64 TMEM columns this frees hold a third dQ^T buffer, so a
+// step's dQ^T MMAs reuse the buffer of step s-3 (drained long before) instead of step s-2.
+// Measured at N = 16384, d = 128: -1.9 % (the S_S MMAs are on the teacher-first critical
+// path), so it is off. The trainable-teacher gradient cannot use it: its second staging
+// tile is the K_S tile, which the S_S MMAs would still be reading.
 #ifndef SKL_BWD_DQ3
 #define SKL_BWD_DQ3 0
 #endif
-#ifndef SKL_BWD_DQ3_T
-#define SKL_BWD_DQ3_T 1
-#endif
-static_assert(!(SKL_BWD_DQ3 || SKL_BWD_DQ3_T) || (SKL_BWD_LEANMMA && SKL_BWD_KTMEM && SKL_BWD_SPLIT),
+static_assert(!SKL_BWD_DQ3 || (SKL_BWD_LEANMMA && SKL_BWD_KTMEM && SKL_BWD_SPLIT),
               "three dQ buffers assume the lean MMA issue, K_T in TMEM and 16 dS warps");
 
 // SKL_BWD_NSTG = 2: two fp32 staging tiles for the dQ reduce-adds, one per step parity (each
@@ -195,7 +191,7 @@ struct BwdCfg {
   static constexpr int NSB = SKL_BWD_KTMEM ? 1 : 2;  // score-tile buffers
   static constexpr int TM_S = 0;          // buffer b: [128b, 128b+64) S_T, [+64, +128) S_S
   static constexpr int TM_DK = 128 * NSB; // d_G columns
-  static constexpr bool DQ3 = TEACHER ? (SKL_BWD_DQ3_T != 0 && DS == 128) : (SKL_BWD_DQ3 != 0);
+  static constexpr bool DQ3 = !TEACHER && SKL_BWD_DQ3 != 0;
   static constexpr int NDQ = DQ3 ? 3 : 2;  // dQ^T buffers in TMEM
   static constexpr int TM_DQ = TM_DK + DG;  // buffer b: + 64 b
   static constexpr int TM_KT = TM_DQ + NDQ * BM;  // SKL_BWD_KTMEM: K_T rows, d_T/2 columns

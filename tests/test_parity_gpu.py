@@ -250,6 +250,7 @@ def test_repeatable_and_no_allocation():
 
 @pytest.mark.parametrize("nq,nk,dt,ds,causal", [
     (300, 300, 128, 128, True),
+    (1024, 1024, 128, 128, True),   # 16 query steps per key tile: every staging tile in use
     (333, 517, 128, 64, False),
     (517, 333, 64, 128, True),
     (640, 640, 64, 64, True),
@@ -651,6 +652,7 @@ def test_teacher_grads_full_size_two_heads():
     kl, lt, ls = skl.streamkl_fwd(*a)
     dq_t, dk_t = skl.streamkl_bwd_teacher(*a, kl, lt, ls, d["g"])
     assert skl.device_status() == 0
+    assert bool(torch.isfinite(dq_t).all()) and bool(torch.isfinite(dk_t).all())
     for b, h in [(0, 0), (1, 15)]:
         one = {k: v[b:b + 1, h:h + 1] for k, v in x.items()}
         dq_r, dk_r = oracle_bwd_teacher(one["q_t"], one["k_t"], one["q_s"], one["k_s"], w.scale_T,
