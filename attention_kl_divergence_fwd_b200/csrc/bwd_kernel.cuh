@@ -139,7 +139,12 @@ static_assert(!SKL_BWD_TFREE || SKL_BWD_TFIRST, "the early teacher release needs
 #ifndef SKL_BWD_DQ3
 #define SKL_BWD_DQ3 0
 #endif
-static_assert(!SKL_BWD_DQ3 || (SKL_BWD_LEANMMA && SKL_BWD_KTMEM && SKL_BWD_SPLIT),
+// SKL_BWD_DQ3_T: the same for the trainable-teacher gradient, with a single dQ staging tile
+// (its second one would be the K_S tile, which the S_S MMAs then still read).
+#ifndef SKL_BWD_DQ3_T
+#define SKL_BWD_DQ3_T 0
+#endif
+static_assert(!(SKL_BWD_DQ3 || SKL_BWD_DQ3_T) || (SKL_BWD_LEANMMA && SKL_BWD_KTMEM && SKL_BWD_SPLIT),
               "three dQ buffers assume the lean MMA issue, K_T in TMEM and 16 dS warps");
 
 // SKL_BWD_NSTG = 2: two fp32 staging tiles for the dQ reduce-adds, one per step parity (each
@@ -177,8 +182,10 @@ struct BwdCfg {
   // K tile of the side that is not differentiated (second staging tile, see SKL_BWD_NSTG).
   static constexpr int OFF_KX = TEACHER ? OFF_KS : OFF_KT;
   static constexpr int KX_TILE = TEACHER ? KS_TILE : KT_TILE;
-  static constexpr int NSTG =
-      (SKL_BWD_NSTG == 2 && SKL_BWD_KTMEM && KX_TILE >= STG_TILE) ? 2 : 1;  // staging tiles
+  // SKL_BWD_DQ3(_T): S_S reads K_S from shared memory (third dQ^T buffer in TMEM)
+  static constexpr bool DQ3 = TEACHER ? SKL_BWD_DQ3_T != 0 : SKL_BWD_DQ3 != 0;
+  static constexpr int NSTG =  // staging tiles; the K_S tile is not free with DQ3
+      (SKL_BWD_NSTG == 2 && SKL_BWD_KTMEM && KX_TILE >= STG_TILE && !(TEACHER && DQ3)) ? 2 : 1;
   // Staging tile of use p (dQ part of step p, or dK round p - n_steps).
   static __device__ __forceinline__ uint32_t stg_off(int p) {
     return (NSTG == 2 && (p & 1)) ? OFF_KX : OFF_STG;
@@ -191,7 +198,6 @@ struct BwdCfg {
   static constexpr int NSB = SKL_BWD_KTMEM ? 1 : 2;  // score-tile buffers
   static constexpr int TM_S = 0;          // buffer b: [128b, 128b+64) S_T, [+64, +128) S_S
   static constexpr int TM_DK = 128 * NSB; // d_G columns
-  static constexpr bool DQ3 = !TEACHER && SKL_BWD_DQ3 != 0;
   static constexpr int NDQ = DQ3 ? 3 : 2;  // dQ^T buffers in TMEM
   static constexpr int TM_DQ = TM_DK + DG;  // buffer b: + 64 b
   static constexpr int TM_KT = TM_DQ + NDQ * BM;  // SKL_BWD_KTMEM: K_T rows, d_T/2 columns
