@@ -123,29 +123,6 @@ static_assert(!SKL_BWD_SPLIT || kBwdDsWarps * SKL_BWD_RS_T + 4 * SKL_BWD_RC_T <=
 #endif
 static_assert(!SKL_BWD_TFIRST || (SKL_BWD_LEANMMA && SKL_BWD_KTMEM && SKL_BWD_SPLIT),
               "teacher scores first assume the lean MMA issue, K in TMEM and 16 dS warps");
-// SKL_BWD_TFREE (with SKL_BWD_TFIRST): the teacher half of the score buffer is released as
-// soon as the dS warps have loaded it, so the next step's teacher score MMAs can start
-// while the student half is still being read.
-#ifndef SKL_BWD_TFREE
-#define SKL_BWD_TFREE 0
-#endif
-static_assert(!SKL_BWD_TFREE || SKL_BWD_TFIRST, "the early teacher release needs SKL_BWD_TFIRST");
-// SKL_BWD_DQ3 (student gradient only): the S_S score MMAs read K_S from shared memory
-// instead of TMEM, and the 64 TMEM columns this frees hold a third dQ^T buffer, so a
-// step's dQ^T MMAs reuse the buffer of step s-3 (drained long before) instead of step s-2.
-// Measured at N = 16384, d = 128: -1.9 % (the S_S MMAs are on the teacher-first critical
-// path), so it is off. The trainable-teacher gradient cannot use it: its second staging
-// tile is the K_S tile, which the S_S MMAs would still be reading.
-#ifndef SKL_BWD_DQ3
-#define SKL_BWD_DQ3 0
-#endif
-// SKL_BWD_DQ3_T: the same for the trainable-teacher gradient, with a single dQ staging tile
-// (its second one would be the K_S tile, which the S_S MMAs then still read).
-#ifndef SKL_BWD_DQ3_T
-#define SKL_BWD_DQ3_T 0
-#endif
-static_assert(!(SKL_BWD_DQ3 || SKL_BWD_DQ3_T) || (SKL_BWD_LEANMMA && SKL_BWD_KTMEM && SKL_BWD_SPLIT),
-              "three dQ buffers assume the lean MMA issue, K_T in TMEM and 16 dS warps");
 
 // SKL_BWD_NSTG = 2: two fp32 staging tiles for the dQ reduce-adds, one per step parity (each
 // dS warpgroup drains into its own tile while the previous reduce is still reading the
@@ -182,10 +159,8 @@ struct BwdCfg {
   // K tile of the side that is not differentiated (second staging tile, see SKL_BWD_NSTG).
   static constexpr int OFF_KX = TEACHER ? OFF_KS : OFF_KT;
   static constexpr int KX_TILE = TEACHER ? KS_TILE : KT_TILE;
-  // SKL_BWD_DQ3(_T): S_S reads K_S from shared memory (third dQ^T buffer in TMEM)
-  static constexpr bool DQ3 = TEACHER ? SKL_BWD_DQ3_T != 0 : SKL_BWD_DQ3 != 0;
-  static constexpr int NSTG =  // staging tiles; the K_S tile is not free with DQ3
-      (SKL_BWD_NSTG == 2 && SKL_BWD_KTMEM && KX_TILE >= STG_TILE && !(TEACHER && DQ3)) ? 2 : 1;
+  static constexpr int NSTG =
+      (SKL_BWD_NSTG == 2 && SKL_BWD_KTMEM && KX_TILE >= STG_TILE) ? 2 : 1;  // staging tiles
   // Staging tile of use p (dQ part of step p, or dK round p - n_steps).
   static __device__ __forceinline__ uint32_t stg_off(int p) {
     return (NSTG == 2 && (p & 1)) ? OFF_KX : OFF_STG;
@@ -198,13 +173,11 @@ struct BwdCfg {
   static constexpr int NSB = SKL_BWD_KTMEM ? 1 : 2;  // score-tile buffers
   static constexpr int TM_S = 0;          // buffer b: [128b, 128b+64) S_T, [+64, +128) S_S
   static constexpr int TM_DK = 128 * NSB; // d_G columns
-  static constexpr int NDQ = DQ3 ? 3 : 2;  // dQ^T buffers in TMEM
   static constexpr int TM_DQ = TM_DK + DG;  // buffer b: + 64 b
-  static constexpr int TM_KT = TM_DQ + NDQ * BM;  // SKL_BWD_KTMEM: K_T rows, d_T/2 columns
-  static constexpr int TM_KS = TM_KT + DT / 2;    // K_S rows, d_S/2 columns (not DQ3)
+  static constexpr int TM_KT = TM_DQ + 2 * BM;  // SKL_BWD_KTMEM: K_T rows, d_T/2 columns
+  static constexpr int TM_KS = TM_KT + DT / 2;  //                K_S rows, d_S/2 columns
   static constexpr int DQ_M = DG;         // M of the dQ^T MMA (64 uses half the lanes)
-  static_assert((SKL_BWD_KTMEM ? TM_KS + (DQ3 ? 0 : DS / 2) : TM_DQ + 2 * BM) <= 512,
-                "TMEM budget");
+  static_assert((SKL_BWD_KTMEM ? TM_KS + DS / 2 : TM_DQ + 2 * BM) <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -214,9 +187,8 @@ struct BwdBars {
   uint64_t stg_full[2], stg_free[2];  // indexed by step parity
   uint64_t s_full[2], s_free[2];
   uint64_t t_full[2];  // SKL_BWD_TFIRST: teacher scores of the step (parity) are ready
-  uint64_t t_free[2];  // SKL_BWD_TFREE: teacher scores of the step (parity) have been read
   uint64_t ds_full[2], ds_empty[2];
-  uint64_t dq_full[3], dq_free[3];  // indexed by dQ^T buffer
+  uint64_t dq_full[2], dq_free[2];
   uint64_t dk_full;
   uint64_t k_tmem;  // SKL_BWD_KTMEM: the K rows are in tensor memory (8 warps arrive)
   uint64_t drain;
@@ -292,12 +264,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&bars->s_full[b]), 1);
       mbar_init(smem_u32(&bars->t_full[b]), 1);
-      mbar_init(smem_u32(&bars->t_free[b]), kBwdArrive);
       mbar_init(smem_u32(&bars->s_free[b]), kBwdArrive);
       mbar_init(smem_u32(&bars->ds_full[b]), kBwdArrive);
       mbar_init(smem_u32(&bars->ds_empty[b]), 1);
-    }
-    for (int b = 0; b < C::NDQ; ++b) {
       mbar_init(smem_u32(&bars->dq_full[b]), 1);
       mbar_init(smem_u32(&bars->dq_free[b]), kBwdArrive);
     }
@@ -484,18 +453,14 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         const uint32_t lds_k0 = sdesc_lo(sb + C::OFF_DS, 16);           // dS^T buffer 0 as A
         const uint32_t lds_n0 = sdesc_lo(sb + C::OFF_DS, C::BN * 128);  // dS^T buffer 0 as B
         const uint32_t lkg = sdesc_lo(TEACHER ? s_kt : s_ks, C::BN * 128);  // K^T as A
-        const uint32_t lks = sdesc_lo(s_ks, 16);  // SKL_BWD_DQ3: K_S as the A of S_S, K-major
         constexpr uint32_t kQ16 = C::Q_STAGE >> 4, kDs16 = C::DS_TILE >> 4;
         const uint32_t t_st = tmem + C::TM_S, t_ss = t_st + 64, t_dk = tmem + C::TM_DK;
         const uint32_t t_kt = tmem + C::TM_KT, t_ks = tmem + C::TM_KS, t_dq = tmem + C::TM_DQ;
         int s_st = 0;      // query stage of the next score step
         uint32_t s_ph = 0;  // and the phase of its q_full barrier
-        constexpr bool kTFree = SKL_BWD_TFREE && !TEACHER;
         auto issue_scores = [&](int s) -> bool {
           if (!mbar_wait(smem_u32(&bars->q_full[s_st]), s_ph)) return false;
-          if (s > 0 && !mbar_wait(smem_u32(kTFree ? &bars->t_free[(s - 1) & 1]
-                                                  : &bars->s_free[(s - 1) & 1]),
-                                  ((s - 1) >> 1) & 1))
+          if (s > 0 && !mbar_wait(smem_u32(&bars->s_free[(s - 1) & 1]), ((s - 1) >> 1) & 1))
             return false;
           tc_fence_after();
           const uint32_t lq = lq0 + (uint32_t)s_st * kQ16;
@@ -505,19 +470,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
             umma_bf16_ts_lh(t_st, t_kt + kk * 8, lq + qa, hi, idesc_st, kk > 0);
           }
           if (SKL_BWD_TFIRST && !TEACHER) umma_commit(smem_u32(&bars->t_full[s & 1]));
-          if (kTFree && s > 0) {
-            if (!mbar_wait(smem_u32(&bars->s_free[(s - 1) & 1]), ((s - 1) >> 1) & 1)) return false;
-            tc_fence_after();
-          }
     #pragma unroll
           for (int kk = 0; kk < DS / 16; ++kk) {
             const uint32_t qa = (C::QT_TILE + (kk >> 2) * (C::BM * 128) + (kk & 3) * 32) >> 4;
-            if (C::DQ3) {
-              const uint32_t ka = ((kk >> 2) * (C::BN * 128) + (kk & 3) * 32) >> 4;
-              umma_bf16_ss_lh(t_ss, lks + ka, lq + qa, hi, idesc_ss, kk > 0);
-            } else {
-              umma_bf16_ts_lh(t_ss, t_ks + kk * 8, lq + qa, hi, idesc_ss, kk > 0);
-            }
+            umma_bf16_ts_lh(t_ss, t_ks + kk * 8, lq + qa, hi, idesc_ss, kk > 0);
           }
           umma_commit(smem_u32(&bars->s_full[s & 1]));
           if (++s_st == C::NQST) {
@@ -526,9 +482,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
           }
           return true;
         };
-        int pst = 0;       // query stage of step p
-        int pq = 0;        // dQ^T buffer of step p
-        uint32_t pq_ph = 0;  // and the phase of its barriers
+        int pst = 0;  // query stage of step p
         if (ok && n_steps > 0) ok = issue_scores(0);
         for (int p = 0; ok && p < n_steps; ++p) {
           const int pb = p & 1;
@@ -543,20 +497,16 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
             umma_bf16_ss_lh(t_dk, la + kk * 2, lb + kk * 128, hi, idesc_dk,
                             (p > 0 || kk > 0) ? 1u : 0u);
           umma_commit(smem_u32(&bars->q_empty[pst]));
-          if (!mbar_wait(smem_u32(&bars->dq_free[pq]), pq_ph ^ 1)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&bars->dq_free[pb]), ((p >> 1) & 1) ^ 1)) { ok = false; break; }
           tc_fence_after();
           // dQ^T = K^T dS^T : A = K [keys][d] MN-major, B = dS^T [keys][queries] MN-major.
-          const uint32_t lbq = lds_n0 + (pb ? kDs16 : 0u), t_dqb = t_dq + pq * C::BM;
+          const uint32_t lbq = lds_n0 + (pb ? kDs16 : 0u), t_dqb = t_dq + (pb ? C::BM : 0);
     #pragma unroll
           for (int kk = 0; kk < C::BN / 16; ++kk)
             umma_bf16_ss_lh(t_dqb, lkg + kk * 128, lbq + kk * 128, hi, idesc_dq, kk > 0);
           umma_commit(smem_u32(&bars->ds_empty[pb]));
-          umma_commit(smem_u32(&bars->dq_full[pq]));
+          umma_commit(smem_u32(&bars->dq_full[pb]));
           if (++pst == C::NQST) pst = 0;
-          if (++pq == C::NDQ) {
-            pq = 0;
-            pq_ph ^= 1u;
-          }
         }
     #else
     #if SKL_BWD_KTMEM
@@ -700,21 +650,18 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
     // dQ^T part of step p (TMEM) -> staging tile (dQ row layout: 32-column boxes of
     // 64 rows x 128 bytes, 128-byte swizzle) -> one bulk reduce-add by the reduce warp.
     auto drain_dq = [&](int p) -> bool {
-      // dQ^T buffer of step p and the phase of its barriers (two buffers: the step parity)
-      const int qb = C::NDQ == 3 ? p % 3 : wg;
-      const uint32_t qph = C::NDQ == 3 ? (uint32_t)(p / 3) & 1u : (uint32_t)(p >> 1) & 1u;
-      if (!mbar_wait(smem_u32(&bars->dq_full[qb]), qph)) return false;
+      if (!mbar_wait(smem_u32(&bars->dq_full[wg]), (p >> 1) & 1)) return false;
       tc_fence_after();
       uint32_t v[NC];  // this warp's query columns c0 .. c0+NC-1 of the dQ^T part
       if constexpr (NC == 64) {
-        tmem_ld_2x32_wait(tmem + lane_off + C::TM_DQ + qb * C::BM,
-                          tmem + lane_off + C::TM_DQ + qb * C::BM + 32, v);
+        tmem_ld_2x32_wait(tmem + lane_off + C::TM_DQ + wg * C::BM,
+                          tmem + lane_off + C::TM_DQ + wg * C::BM + 32, v);
       } else {
-        tmem_ld_32_wait(tmem + lane_off + C::TM_DQ + qb * C::BM + c0, v);
+        tmem_ld_32_wait(tmem + lane_off + C::TM_DQ + wg * C::BM + c0, v);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->dq_free[qb]));
+      if (lane == 0) mbar_arrive(smem_u32(&bars->dq_free[wg]));
       if (!stg_wait(p)) return false;
       if (dq_lane_ok) {
         const uint32_t col = sb + C::stg_off(p) + (dq_d >> 5) * (C::BM * 128) + ((dq_d & 3) << 2);
@@ -741,7 +688,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
       } else if (mbar_wait(smem_u32(&bars->k_full), 0)) {
         if (wg == 0)
           row_to_tmem<DT>(sb + C::OFF_KT + kl * 128, tmem + lane_off + C::TM_KT, kl);
-        else if (!C::DQ3)
+        else
           row_to_tmem<DS>(sb + C::OFF_KS + kl * 128, tmem + lane_off + C::TM_KS, kl);
       } else {
         ok = false;
@@ -766,11 +713,6 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap map_qt,
         tc_fence_after();
         uint32_t vt[NC];
         tmem_ld_32_wait(tmem + lane_off + C::TM_S + sbuf * 128 + c0, vt);
-#if SKL_BWD_TFREE
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->t_free[wg]));
-#endif
         if (!mbar_wait(smem_u32(&bars->st_full[s & 1]), (s >> 1) & 1)) { ok = false; break; }
         const float* sts = stats + (s & 1) * (4 * C::BM);
         float pt[NC];
