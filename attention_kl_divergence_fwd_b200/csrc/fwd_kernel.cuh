@@ -7,16 +7,20 @@
 //
 // CTA = two 128-row query tiles of one (batch, head). Key tiles of 64 rows stream
 // through a TMA ring. Per key tile and query tile the tensor core computes the teacher
-// and student score tiles into TMEM (two buffers per query tile, so the next tile is
-// computed while the current one is folded). Each query row is folded by two threads
-// (one per 32-key half of every tile), each keeping its own online state
-//     m_T, m_S   running maxima of t = s * log2(e)
+// and student score tiles into TMEM, with the query tiles themselves held in TMEM as the
+// MMA's A operand (SKL_FWD_QTMEM; one score buffer per query tile, whose next tile is
+// computed as soon as the current one has been read, so the fold overlaps those MMAs).
+// Each query row is folded by two threads (one per 32-key half of every tile), each
+// keeping its own online state
+//     m_T, m_S   reference maxima of t = s * log2(e) (at most the running maxima)
 //     l_T, l_S   running sums of 2^(t - m)
 //     A          running sum of 2^(t_T - m_T) * (t_T - t_S)
 // which merge at the end, so that KL = ln2 * A / l_T - LSE_T + LSE_S. Per tile a thread
 // reads its 64 scores from TMEM in one round trip and releases the buffer at once; the
 // fp32 work is issued as packed pairs, with a share of the exponentials on the FMA pipe.
-// Unmasked tiles are folded against the running maxima as they stand (no per-tile max).
+// Unmasked tiles are folded against the reference maxima as they stand (no per-tile max;
+// the state is exact for any reference); masked tiles, a row's first tile and a tile
+// whose exponentials would reach 2^64 raise the references to the running maxima first.
 // Nothing of size N_Q x N_K ever leaves the SM.
 //
 // Warp roles (640 threads, SKL_FWD_SPLIT): warps 0-7 query tile 0 and 8-15 query tile 1
