@@ -77,10 +77,6 @@ WORKLOADS: Dict[str, Workload] = {
 WORKLOAD_LIST = sorted(WORKLOADS.values(), key=lambda w: w.index)
 
 
-def by_index(k: int) -> Workload:
-    return WORKLOAD_LIST[k - 1]
-
-
 def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
     """Draw the inputs of workload ``w`` on the CPU.
 
