@@ -179,11 +179,13 @@ streamkl_fwd_persistent_kernel(const __grid_constant__ CUtensorMap map_qt,
       }
 
       // Half 1 hands its row state to half 0 through 8 columns of this query tile's score
-      // buffer. Nothing writes that buffer between this unit's last score MMA on the tile
-      // (completed: its scores were read) and the next unit's first, which the MMA thread
-      // issues only after every statistics warp has copied the next unit's query rows,
-      // i.e. after half 0 has read the state below.
-      const uint32_t tx = tmem + lane_off + C::tm_s(q, 0);
+      // buffer: the first 8 of its own teacher columns (32 .. 39), which it has already read
+      // and half 0 never reads (half 0 may still be loading its columns of the last tile
+      // when half 1 gets here). No MMA writes that buffer between this unit's last score
+      // MMA on the tile (completed: its scores were read) and the next unit's first, which
+      // the MMA thread issues only after every statistics warp has copied the next unit's
+      // query rows, i.e. after half 0 has read the state below.
+      const uint32_t tx = tmem + lane_off + C::tm_s(q, 0) + 32;
       if (half == 1) {
         const uint32_t xs[8] = {__float_as_uint(st.mT), __float_as_uint(st.mS),
                                 __float_as_uint(st.lT), __float_as_uint(st.lS),
